@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the GDN recurrence on B200: tokens*heads/s and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one gdn_forward call over the whole workload (default: the 720p
+bidirectional workload, B=2, H=16, T=75600, dk=dv=128, bf16 inputs, fp32
+state), inputs resident in HBM.  Inputs total 4.4 GB, far above the 126 MB
+L2, so no flush is needed between steps.  Timing: W warm-up steps, then a
+barrier + device synchronise, K steps bracketed by CUDA events on the
+launching stream, synchronise + barrier, max over ranks.  With N > 1 (one
+process per GPU under torchrun) every rank runs its own full workload: the
+scans are independent, there is no collective on the data path (weak scaling).
+
+Also measured, and printed on the same JSON line:
+  e2e          the same metric through the library's host-buffer entry point
+               (pinned host inputs; host->device copies, the kernels, and the
+               device->host copy of o and the states inside the timed region);
+  roofline     the main kernel's algorithmic bytes / its average event-timed
+               duration, against the measured HBM copy bandwidth;
+  cpu_baseline the fp64 CPU oracle on a bounded sample of the same workload
+               (rank 0, N = 1 only);
+  clocks       nvidia-smi samples taken during the timed region.
+--impl reference times the CPU oracle alone (the reference arm of this build:
+there is no upstream code to run).
+"""
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN tokens*heads/s (bf16, 1xB200)"
+UNIT = "tokens*heads/s"
+
+
+def algorithmic_bytes(wl):
+    """Bytes a perfect kernel moves once: q, k, v, gates read and o written once
+    per scan direction, plus the fp32 states (in if present, out always)."""
+    es = 2 if wl.dtype == "bf16" else 4
+    ndir = 2 if wl.bidi else 1
+    per_tok = ndir * ((2 * wl.dk + wl.dv) * es + 8) + wl.dv * es
+    st = wl.dk * wl.dv * 4
+    n_heads = wl.B * wl.H
+    states = n_heads * st * (ndir + (1 if wl.state0 else 0))
+    return wl.B * wl.H * wl.T * wl.n_chunks * per_tok + states * wl.n_chunks
+
+
+def algorithmic_flops(wl, C=64):
+    """Useful chunkwise MMA FLOPs (triangles counted half) per token*head*direction:
+    3*C*dk + 2*C*dv + C^2/3 + 6*dk*dv."""
+    ndir = 2 if wl.bidi else 1
+    per = 3 * C * wl.dk + 2 * C * wl.dv + C * C / 3 + 6 * wl.dk * wl.dv
+    return wl.token_heads * ndir * per
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in ("gdn_chunk_tc.cu", "gdn_recurrent.cu"):
+        p = os.path.join(ROOT, "gated_delta_rule_149_b200", "csrc", name)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, sha):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload)
+    if not d or d.get("kernel_source_sha") != sha:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.f is None:
+            return None
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.lower() in ("active", "1"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# CPU oracle baseline (a bounded sample of the workload)
+# --------------------------------------------------------------------------
+
+def oracle_sample_throughput(wl, target_s=15.0):
+    """Times the fp64 oracle on whole heads of the workload truncated to a
+    token prefix sized for ~target_s seconds on the host cores."""
+    import numpy as np
+    import oracle
+    from gated_delta_rule_149_b200.inputs import Workload, make_inputs
+    nproc = os.cpu_count() or 1
+    ndir = 2 if wl.bidi else 1
+    n_heads = max(1, min(wl.B * wl.H, max(1, nproc // ndir)))
+    threads = min(nproc, n_heads * ndir)
+
+    def run(T):
+        sub = Workload(wl.name + "_sample", B=1, H=n_heads, T=T, dk=wl.dk, dv=wl.dv,
+                       dtype=wl.dtype, bidi=wl.bidi, decay_shift=wl.decay_shift, seed=wl.seed)
+        inp = make_inputs(sub)
+        args = [inp.q.double().numpy(), inp.k.double().numpy(), inp.v.double().numpy(),
+                inp.beta.double().numpy(), inp.decay.double().numpy()]
+        t0 = time.perf_counter()
+        oracle.gdn_forward(*args, bidi=wl.bidi, n_threads=threads)
+        return time.perf_counter() - t0
+
+    t_small = run(256)
+    per_tok = t_small / 256.0
+    T = int(max(512, min(wl.T, target_s / max(per_tok, 1e-9))))
+    el = run(T)
+    value = n_heads * T / el
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n_heads} heads x first {T} tokens of {wl.name} "
+                      f"({'both directions' if wl.bidi else 'causal'}), fp64, {el:.1f} s wall",
+            "elapsed_s": el, "cpu": _cpu_model()}
+
+
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_reference(args, world, rank):
+    from gated_delta_rule_149_b200.inputs import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if rank != 0:
+        return 0
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample_throughput(wl, target_s=args.ref_seconds)
+        if i >= args.warmup:
+            vals.append(r)
+    value = statistics.median(v["value"] for v in vals)
+    el = sum(v["elapsed_s"] for v in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / len(vals), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk,
+                       "dv": wl.dv, "mode": "bidi" if wl.bidi else "causal"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"],
+                             "kind": "oracle", "sample": vals[0]["sample"],
+                             "cpu": vals[0]["cpu"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+
+def run_gpu(args, world, rank, local):
+    import torch
+    from gated_delta_rule_149_b200 import gdn, gdn_forward, gdn_forward_host, gdn_device_status
+    from gated_delta_rule_149_b200.inputs import WORKLOADS, make_inputs
+
+    wl = WORKLOADS[args.workload]
+    assert wl.n_chunks == 1, "the benchmark times single-call workloads"
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_inputs(wl)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    beta, decay = inp.beta.to(dev), inp.decay.to(dev)
+    s0 = None if inp.state0 is None else inp.state0.to(dev)
+    o = torch.empty(wl.B, wl.H, wl.T, wl.dv, dtype=q.dtype, device=dev)
+    s_out = torch.empty(((2,) if wl.bidi else ()) + (wl.B, wl.H, wl.dk, wl.dv),
+                        dtype=torch.float32, device=dev)
+    recurrent = args.recurrent or wl.dtype == "fp32"
+    stream = torch.cuda.current_stream(dev)
+    lib = gdn.load_library()
+
+    def step():
+        gdn_forward(q, k, v, beta, decay, s0, bidi=wl.bidi, recurrent=recurrent, o=o,
+                    state_out=s_out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    gdn_device_status(stream)
+    torch.cuda.synchronize()
+
+    launches0 = lib.gdn_kernel_launches()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_all0 = torch.cuda.Event(enable_timing=True)
+        t_all1 = torch.cuda.Event(enable_timing=True)
+        t_all0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_all1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = lib.gdn_kernel_launches() - launches0
+    gdn_device_status(stream)
+    total_ms = t_all0.elapsed_time(t_all1)
+    per_call = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    value = world * wl.token_heads / (ms_per_step * 1e-3)
+
+    # roofline of the main kernel (the call is one main kernel plus a tiny memset)
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+    call_s = statistics.mean(per_call) * 1e-3
+    bytes_ = algorithmic_bytes(wl)
+    achieved = bytes_ / call_s / 1e9
+    sha = kernel_source_sha()
+    traffic = recorded_traffic(wl.name, sha)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": traffic,
+                "peak_kind": peak_kind, "algorithmic_bytes": bytes_,
+                "tensor_tflops": algorithmic_flops(wl) / call_s / 1e12,
+                "tensor_frac": algorithmic_flops(wl) / call_s / 1e12 / tc_peak,
+                "kernel_source_sha": sha}
+
+    # end to end through the host-buffer entry point
+    pin = lambda t: t.pin_memory()
+    hq, hk, hv, hb, ha = map(pin, (inp.q, inp.k, inp.v, inp.beta, inp.decay))
+    hs0 = None if inp.state0 is None else pin(inp.state0)
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hso = torch.empty(s_out.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        gdn_forward_host(hq, hk, hv, hb, ha, hs0, bidi=wl.bidi, recurrent=recurrent, o=ho,
+                         state_out=hso, stream=stream)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    nbytes = lambda *ts: sum(t.numel() * t.element_size() for t in ts if t is not None)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk,
+                       "dv": wl.dv, "mode": "bidi" if wl.bidi else "causal",
+                       "kernel": "recurrent" if recurrent else "chunk_tc",
+                       "token_heads_per_gpu": wl.token_heads,
+                       "l2": "no flush: inputs of %.2f GB per step exceed the 126 MB L2"
+                             % (bytes_ / 1e9),
+                       "parallelism": f"replicas x{world} (independent scans, no collective)"},
+            "e2e": {"value": world * wl.token_heads / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": nbytes(hq, hk, hv, hb, ha, hs0),
+                    "d2h_bytes_per_step": nbytes(ho, hso)},
+            "gpu_launches": int(launches),
+            "roofline": roofline,
+            "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample_throughput(wl, target_s=args.ref_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="bidi_720p")
+    ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
+    ap.add_argument("--recurrent", action="store_true",
+                    help="time the token-by-token SIMT kernel instead of the chunkwise one")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        return run_reference(args, world, rank)
+    world, rank, local = dist_setup()
+    try:
+        return run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,241 @@
+// libgdn C ABI: argument checks, dispatch, rollout threading, host-buffer
+// entry point, device error word.  No C++ exception crosses this boundary
+// (the catch-at-the-boundary convention of the librediffusion PR #21 C-API,
+// and the reason-string prechecks of the SANA-WM camera-GDN backend error
+// record), and every argument error is caught before anything is launched.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/gdn.h"
+#include "gdn_internal.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok()
+{
+    g_msg[0] = '\0';
+    return GDN_OK;
+}
+
+bool misaligned(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+// Shape / dtype / pointer checks shared by gdn_forward and gdn_rollout.
+int check_common(const void *q, const void *k, const void *v, const float *beta,
+                 const float *decay, const float *state_in, const float *state_out,
+                 const void *o, int B, int H, int T, int dk, int dv, int mode,
+                 const char *T_name)
+{
+    if (!q || !k || !v || !beta || !decay || !o)
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v, beta, decay and o must be non-NULL");
+    if (B <= 0 || H <= 0 || T <= 0)
+        return fail(GDN_ERR_INVALID_ARG, "B, H and %s must be positive (got %d, %d, %d)",
+                    T_name, B, H, T);
+    if (mode & ~(GDN_BIDI | GDN_FP32 | GDN_RECURRENT))
+        return fail(GDN_ERR_INVALID_ARG, "unknown mode bits 0x%x", mode);
+    if ((long long)B * H > 65535)
+        return fail(GDN_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535", (long long)B * H);
+    if (dk <= 0 || dv <= 0 || dk % 32 || dv % 32 || dk > 128 || dv > 128)
+        return fail(GDN_ERR_UNSUPPORTED,
+                    "dk and dv must be multiples of 32 in [32, 128] (got dk=%d, dv=%d)", dk, dv);
+    const void *ptrs[] = {q, k, v, beta, decay, state_in, state_out, o};
+    const char *names[] = {"q", "k", "v", "beta", "decay", "state_in", "state_out", "o"};
+    for (int i = 0; i < 8; ++i)
+        if (misaligned(ptrs[i]))
+            return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    return GDN_OK;
+}
+
+gdn::FwdArgs make_args(const void *q, const void *k, const void *v, const float *beta,
+                       const float *decay, const float *state_in, float *state_out, void *o,
+                       int B, int H, int T, int dk, int dv, int mode)
+{
+    gdn::FwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.decay = decay;
+    a.state_in = state_in; a.state_out = state_out; a.o = o;
+    a.B = B; a.H = H; a.T = T; a.dk = dk; a.dv = dv;
+    a.bidi = (mode & GDN_BIDI) != 0;
+    a.fp32 = (mode & GDN_FP32) != 0;
+    return a;
+}
+
+// Picks the kernel for validated arguments and launches it.
+int dispatch(const gdn::FwdArgs &a, int mode, cudaStream_t stream)
+{
+    const bool recurrent = a.fp32 || (mode & GDN_RECURRENT);
+    cudaError_t err;
+    if (recurrent) {
+        err = gdn::launch_recurrent(a, stream);
+    } else if (gdn::chunk_tc_supported(a)) {
+        err = gdn::launch_chunk_tc(a, stream);
+    } else {
+        return fail(GDN_ERR_UNSUPPORTED,
+                    "bf16 chunkwise kernel needs dk = 128 and dv in {64, 128} (got dk=%d, dv=%d); "
+                    "GDN_RECURRENT runs other sizes", a.dk, a.dv);
+    }
+    if (err != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "launch failed: %s", cudaGetErrorString(err));
+    return ok();
+}
+
+size_t dtype_size(int mode) { return (mode & GDN_FP32) ? 4 : 2; }
+
+}  // namespace
+
+extern "C" {
+
+int gdn_version(void) { return 10000; }
+
+const char *gdn_last_error(void) { return g_msg; }
+
+int gdn_forward(const void *q, const void *k, const void *v, const float *beta,
+                const float *decay, const float *state_in, float *state_out, void *o,
+                int B, int H, int T, int dk, int dv, int mode, void *stream)
+{
+    try {
+        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                              mode, "T");
+        if (rc != GDN_OK) return rc;
+        gdn::FwdArgs a = make_args(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                                   mode);
+        return dispatch(a, mode, static_cast<cudaStream_t>(stream));
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in gdn_forward");
+    }
+}
+
+int gdn_rollout(const void *q, const void *k, const void *v, const float *beta,
+                const float *decay, const float *state_in, float *state_out,
+                float *chunk_states, void *o, int B, int H, int n_chunks, int Tc, int dk,
+                int dv, int mode, void *stream_)
+{
+    try {
+        if (n_chunks <= 0) return fail(GDN_ERR_INVALID_ARG, "n_chunks must be positive");
+        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, Tc, dk, dv,
+                              mode, "Tc");
+        if (rc != GDN_OK) return rc;
+        if (misaligned(chunk_states))
+            return fail(GDN_ERR_MISALIGNED, "chunk_states is not 16-byte aligned");
+        if (mode & GDN_BIDI)
+            return fail(GDN_ERR_UNSUPPORTED, "gdn_rollout is causal only (GDN_BIDI given)");
+        cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+        const size_t BH = (size_t)B * H;
+        const size_t st = (size_t)dk * dv;
+        const size_t es = dtype_size(mode);
+        const size_t tok = BH * (size_t)Tc;
+
+        float *ws = nullptr;   // ping-pong states when the caller keeps none
+        if (n_chunks > 1 && !chunk_states) {
+            cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * BH * st * sizeof(float),
+                                            stream);
+            if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "workspace: %s", cudaGetErrorString(e));
+        }
+        const float *cur = state_in;
+        rc = GDN_OK;
+        for (int c = 0; c < n_chunks && rc == GDN_OK; ++c) {
+            float *dst;
+            if (chunk_states) dst = chunk_states + (size_t)c * BH * st;
+            else if (c == n_chunks - 1) dst = state_out;
+            else dst = ws + (size_t)(c & 1) * BH * st;
+            const size_t off = (size_t)c * tok;
+            gdn::FwdArgs a = make_args(
+                static_cast<const char *>(q) + off * dk * es, static_cast<const char *>(k) + off * dk * es,
+                static_cast<const char *>(v) + off * dv * es, beta + off, decay + off, cur, dst,
+                static_cast<char *>(o) + off * dv * es, B, H, Tc, dk, dv, mode);
+            rc = dispatch(a, mode, stream);
+            cur = dst;
+        }
+        if (rc == GDN_OK && chunk_states && state_out) {
+            cudaError_t e = cudaMemcpyAsync(state_out, chunk_states + (size_t)(n_chunks - 1) * BH * st,
+                                            BH * st * sizeof(float), cudaMemcpyDeviceToDevice, stream);
+            if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "state copy: %s", cudaGetErrorString(e));
+        }
+        if (ws) {
+            cudaError_t e = cudaFreeAsync(ws, stream);
+            if (rc == GDN_OK && e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "workspace free: %s", cudaGetErrorString(e));
+        }
+        return rc == GDN_OK ? ok() : rc;
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in gdn_rollout");
+    }
+}
+
+int gdn_forward_host(const void *q, const void *k, const void *v, const float *beta,
+                     const float *decay, const float *state_in, float *state_out, void *o,
+                     int B, int H, int T, int dk, int dv, int mode, void *stream_)
+{
+    try {
+        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                              mode, "T");
+        if (rc != GDN_OK) return rc;
+        cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+        const size_t BH = (size_t)B * H, es = dtype_size(mode);
+        const size_t nqk = BH * T * dk * es, nv = BH * T * dv * es, ng = BH * T * sizeof(float);
+        const size_t nst = BH * (size_t)dk * dv * sizeof(float);
+        const size_t nso = nst * ((mode & GDN_BIDI) ? 2 : 1);
+        // one device block, 256-byte aligned sub-buffers
+        auto up = [](size_t n) { return (n + 255) & ~(size_t)255; };
+        const size_t total = 2 * up(nqk) + 2 * up(nv) + 2 * up(ng) + (state_in ? up(nst) : 0) +
+                             (state_out ? up(nso) : 0);
+        char *base = nullptr;
+        cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&base), total, stream);
+        if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device buffers: %s", cudaGetErrorString(e));
+        char *p = base;
+        auto take = [&p, &up](size_t n) { char *r = p; p += up(n); return r; };
+        char *dq = take(nqk), *dk_ = take(nqk), *dv_ = take(nv), *dout = take(nv);
+        float *db = reinterpret_cast<float *>(take(ng)), *da = reinterpret_cast<float *>(take(ng));
+        float *dsi = state_in ? reinterpret_cast<float *>(take(nst)) : nullptr;
+        float *dso = state_out ? reinterpret_cast<float *>(take(nso)) : nullptr;
+
+        struct Cp { void *dst; const void *src; size_t n; };
+        const Cp h2d[] = {{dq, q, nqk}, {dk_, k, nqk}, {dv_, v, nv}, {db, beta, ng}, {da, decay, ng},
+                          {dsi, state_in, dsi ? nst : 0}};
+        for (const Cp &c : h2d)
+            if (c.n && e == cudaSuccess)
+                e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, stream);
+        if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "host->device copy: %s", cudaGetErrorString(e));
+        if (rc == GDN_OK) {
+            gdn::FwdArgs a = make_args(dq, dk_, dv_, db, da, dsi, dso, dout, B, H, T, dk, dv, mode);
+            rc = dispatch(a, mode, stream);
+        }
+        if (rc == GDN_OK) {
+            e = cudaMemcpyAsync(o, dout, nv, cudaMemcpyDeviceToHost, stream);
+            if (e == cudaSuccess && dso)
+                e = cudaMemcpyAsync(state_out, dso, nso, cudaMemcpyDeviceToHost, stream);
+            if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "device->host copy: %s", cudaGetErrorString(e));
+        }
+        e = cudaFreeAsync(base, stream);
+        cudaError_t es2 = cudaStreamSynchronize(stream);
+        if (rc == GDN_OK && (e != cudaSuccess || es2 != cudaSuccess))
+            rc = fail(GDN_ERR_CUDA, "gdn_forward_host: %s",
+                      cudaGetErrorString(e != cudaSuccess ? e : es2));
+        return rc == GDN_OK ? ok() : rc;
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in gdn_forward_host");
+    }
+}
+
+int gdn_device_status(void *stream)
+{
+    int err = 0;
+    cudaError_t e = gdn::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &err);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device status: %s", cudaGetErrorString(e));
+    if (err) return fail(GDN_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (code %d)", err);
+    return ok();
+}
+
+}  // extern "C"

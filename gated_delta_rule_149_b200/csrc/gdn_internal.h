@@ -1,0 +1,35 @@
+// Internal declarations shared by the libgdn translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace gdn {
+
+// One forward/bidi pass, already validated on the host.
+struct FwdArgs {
+    const void *q, *k, *v;
+    const float *beta, *decay;
+    const float *state_in;    // [B,H,dk,dv] or nullptr
+    float *state_out;         // causal [B,H,dk,dv]; bidi [2,B,H,dk,dv]; or nullptr
+    void *o;                  // [B,H,T,dv]
+    int B, H, T, dk, dv;
+    bool bidi;
+    bool fp32;                // q/k/v/o dtype: fp32 (else bf16)
+};
+
+// Token-by-token fp32 SIMT kernel (any dtype; dk, dv multiples of 32, <= 128).
+cudaError_t launch_recurrent(const FwdArgs &a, cudaStream_t stream);
+
+// Chunkwise tcgen05 kernel (bf16; dk = 128; dv in {64, 128}).
+bool chunk_tc_supported(const FwdArgs &a);
+cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream);
+
+// Device-side error word (set by bounded waits that gave up).
+cudaError_t device_error_word(int **ptr);
+
+// Launch accounting (gdn_kernel_launches).
+void count_launches(int n);
+cudaError_t read_and_clear_device_error(cudaStream_t stream, int *err);
+
+}  // namespace gdn

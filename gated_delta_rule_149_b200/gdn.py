@@ -1,0 +1,190 @@
+"""Thin ctypes binding of libgdn's C ABI (argument marshalling only).
+
+Every function takes torch tensors, checks dtype/shape/device/contiguity,
+and passes raw pointers and sizes to the library; all computation happens in
+the library's CUDA kernels.  There is no CPU or fallback path: if libgdn.so
+cannot be loaded, calls raise.
+"""
+import ctypes
+import os
+
+import torch
+
+GDN_CAUSAL = 0
+GDN_BIDI = 1
+GDN_BF16 = 0
+GDN_FP32 = 2
+GDN_RECURRENT = 4
+
+_STATUS = {0: "GDN_OK", -1: "GDN_ERR_INVALID_ARG", -2: "GDN_ERR_UNSUPPORTED",
+           -3: "GDN_ERR_MISALIGNED", -4: "GDN_ERR_CUDA", -5: "GDN_ERR_DEVICE_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+
+class GDNError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{_STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+def lib_path():
+    return os.environ.get("GDN_LIB", os.path.join(_HERE, "lib", "libgdn.so"))
+
+
+def load_library():
+    """Loads libgdn.so and declares the ABI's argument types."""
+    global _lib
+    if _lib is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise GDNError(-4, f"libgdn.so not found at {path}; run "
+                               f"`python -m gated_delta_rule_149_b200.build` first")
+        lib = ctypes.CDLL(path)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        lib.gdn_forward.argtypes = [vp] * 8 + [i] * 6 + [vp]
+        lib.gdn_forward.restype = i
+        lib.gdn_forward_host.argtypes = [vp] * 8 + [i] * 6 + [vp]
+        lib.gdn_forward_host.restype = i
+        lib.gdn_rollout.argtypes = [vp] * 9 + [i] * 7 + [vp]
+        lib.gdn_rollout.restype = i
+        lib.gdn_device_status.argtypes = [vp]
+        lib.gdn_device_status.restype = i
+        lib.gdn_last_error.argtypes = []
+        lib.gdn_last_error.restype = ctypes.c_char_p
+        lib.gdn_version.argtypes = []
+        lib.gdn_version.restype = i
+        lib.gdn_kernel_launches.argtypes = []
+        lib.gdn_kernel_launches.restype = ctypes.c_longlong
+        _lib = lib
+    return _lib
+
+
+def _check(rc):
+    if rc != 0:
+        raise GDNError(rc, load_library().gdn_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _mode(q, bidi, recurrent):
+    if q.dtype == torch.float32:
+        m = GDN_FP32
+    elif q.dtype == torch.bfloat16:
+        m = GDN_BF16
+    else:
+        raise TypeError(f"q/k/v must be bf16 or fp32, got {q.dtype}")
+    return m | (GDN_BIDI if bidi else 0) | (GDN_RECURRENT if recurrent else 0)
+
+
+def _expect(t, name, shape, dtype, device):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def gdn_forward(q, k, v, beta, decay, state_in=None, *, bidi=False, recurrent=False,
+                o=None, state_out=None, want_state=True, stream=None):
+    """o, state_out = gdn_forward(q, k, v, beta, decay, state_in) on CUDA tensors.
+
+    q, k [B,H,T,dk] and v [B,H,T,dv] (bf16 or fp32, same dtype); beta, decay
+    [B,H,T] fp32; state_in [B,H,dk,dv] fp32 or None.  Returns o [B,H,T,dv]
+    (dtype of q) and the final state ([B,H,dk,dv], or [2,B,H,dk,dv] for bidi:
+    forward then reverse), or None if want_state is False.
+    """
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_forward runs on CUDA tensors only")
+    _expect(k, "k", (B, H, T, dk), q.dtype, dev)
+    _expect(v, "v", (B, H, T, dv), q.dtype, dev)
+    _expect(beta, "beta", (B, H, T), torch.float32, dev)
+    _expect(decay, "decay", (B, H, T), torch.float32, dev)
+    _expect(q, "q", (B, H, T, dk), q.dtype, dev)
+    if state_in is not None:
+        _expect(state_in, "state_in", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=dev)
+    _expect(o, "o", (B, H, T, dv), q.dtype, dev)
+    s_shape = ((2,) if bidi else ()) + (B, H, dk, dv)
+    if state_out is None and want_state:
+        state_out = torch.empty(s_shape, dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _expect(state_out, "state_out", s_shape, torch.float32, dev)
+    lib = load_library()
+    _check(lib.gdn_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(state_in),
+                           _ptr(state_out), _ptr(o), B, H, T, dk, dv,
+                           _mode(q, bidi, recurrent), _stream_handle(stream, dev)))
+    return o, state_out
+
+
+def gdn_rollout(q, k, v, beta, decay, state_in=None, *, recurrent=False, chunk_states=False,
+                o=None, state_out=None, stream=None):
+    """Streaming rollout over chunk-major inputs q,k [n,B,H,Tc,dk], v [n,B,H,Tc,dv],
+    gates [n,B,H,Tc].  Returns (o, state_out, chunk_states or None)."""
+    n, B, H, Tc, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_rollout runs on CUDA tensors only")
+    _expect(k, "k", (n, B, H, Tc, dk), q.dtype, dev)
+    _expect(v, "v", (n, B, H, Tc, dv), q.dtype, dev)
+    _expect(beta, "beta", (n, B, H, Tc), torch.float32, dev)
+    _expect(decay, "decay", (n, B, H, Tc), torch.float32, dev)
+    _expect(q, "q", (n, B, H, Tc, dk), q.dtype, dev)
+    if state_in is not None:
+        _expect(state_in, "state_in", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(n, B, H, Tc, dv, dtype=q.dtype, device=dev)
+    if state_out is None:
+        state_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    cs = torch.empty(n, B, H, dk, dv, dtype=torch.float32, device=dev) if chunk_states else None
+    lib = load_library()
+    _check(lib.gdn_rollout(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(state_in),
+                           _ptr(state_out), _ptr(cs), _ptr(o), B, H, n, Tc, dk, dv,
+                           _mode(q, False, recurrent), _stream_handle(stream, dev)))
+    return o, state_out, cs
+
+
+def gdn_forward_host(q, k, v, beta, decay, state_in=None, *, bidi=False, recurrent=False,
+                     o=None, state_out=None, want_state=True, stream=None, device=None):
+    """gdn_forward on CPU (ideally pinned) tensors through the library's host-buffer
+    entry point: the library copies inputs in, runs, copies o/state back and
+    synchronises.  Returns CPU tensors."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("beta", beta), ("decay", decay)):
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, pin_memory=q.is_pinned())
+    s_shape = ((2,) if bidi else ()) + (B, H, dk, dv)
+    if state_out is None and want_state:
+        state_out = torch.empty(s_shape, dtype=torch.float32, pin_memory=q.is_pinned())
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    lib = load_library()
+    _check(lib.gdn_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay),
+                                _ptr(state_in), _ptr(state_out), _ptr(o), B, H, T, dk, dv,
+                                _mode(q, bidi, recurrent), _stream_handle(stream, dev)))
+    return o, state_out
+
+
+def gdn_device_status(stream=None, device=None):
+    """Synchronises the stream and raises GDNError if a bounded device wait gave up."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _check(load_library().gdn_device_status(_stream_handle(stream, dev)))

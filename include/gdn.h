@@ -1,0 +1,137 @@
+/*
+ * gdn.h -- C ABI of libgdn, the Gated-Delta-Net (GDN) linear-attention
+ * recurrence on NVIDIA B200 (sm_100a).
+ *
+ * The operation (the "GDN (Gated-Delta-Net) linear-attention recurrence" of the
+ * librediffusion PR #21 page, "What's added"; the streaming/bidirectional
+ * forms of the flashdreams SANA-WM page, "Bidirectional variant", and the
+ * causal linear-attention KV cache of the LongSANA diffusers PR #12723 page,
+ * "PR feature"), per batch b and head h, with a dv x dk state S:
+ *
+ *     S_t = a_t * S_{t-1} * (I - b_t k_t k_t^T) + b_t v_t k_t^T
+ *     o_t = S_t q_t
+ *
+ * a_t = decay[b,h,t], b_t = beta[b,h,t].  The stored state is H = S^T, a
+ * row-major [dk][dv] fp32 matrix per head.  No 1/sqrt(dk) factor is applied.
+ *
+ * Layouts (all row-major, contiguous, element strides implied by the sizes):
+ *   q, k        [B, H, T, dk]      bf16 or fp32 (mode bit GDN_FP32)
+ *   v, o        [B, H, T, dv]      same dtype as q
+ *   beta, decay [B, H, T]          fp32; decay in (0, 1], beta in [0, 1] typical
+ *   state_in    [B, H, dk, dv]     fp32, or NULL for a zero initial state
+ *   state_out   causal: [B, H, dk, dv];  bidi: [2, B, H, dk, dv] =
+ *               {forward final state, reverse final state}; or NULL to skip
+ *
+ * Modes (bit flags, OR-ed):
+ *   GDN_CAUSAL (0) / GDN_BIDI (1): causal scan, or bidirectional
+ *       o = fwd(x).o + flip_t(fwd(flip_t(x)).o), flip_t reversing q, k, v,
+ *       beta and decay together along T; the reverse scan starts from zero and
+ *       state_in applies to the forward scan only.
+ *   GDN_BF16 (0) / GDN_FP32 (2): dtype of q, k, v and o.  The state and all
+ *       accumulation are fp32 in both cases.
+ *   GDN_RECURRENT (4): run the token-by-token fp32 SIMT kernel even for bf16
+ *       inputs (a slower cross-check of the chunkwise tensor-core kernel).
+ *
+ * Ownership and asynchrony: every pointer is device memory owned by the
+ * caller (except gdn_forward_host, which takes host memory).  Calls enqueue
+ * work on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ * return without synchronising.  Temporary workspace is taken stream-ordered
+ * (cudaMallocAsync / cudaFreeAsync on `stream`); nothing persists between
+ * calls.  state_in == state_out is allowed.  Inputs must not overlap outputs
+ * otherwise.
+ *
+ * Errors: every call returns GDN_OK (0) or a negative code below, and records
+ * a message readable with gdn_last_error() (thread-local).  All argument
+ * errors are detected on the host before anything is launched.  No C++
+ * exception crosses this boundary.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum gdn_mode_bits {
+    GDN_CAUSAL = 0,
+    GDN_BIDI = 1,
+    GDN_BF16 = 0,
+    GDN_FP32 = 2,
+    GDN_RECURRENT = 4
+};
+
+enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = -1,    /* NULL required pointer, B/H/T/n_chunks <= 0, bad mode bits */
+    GDN_ERR_UNSUPPORTED = -2,    /* shape/dtype combination the kernels do not implement      */
+    GDN_ERR_MISALIGNED = -3,     /* a pointer not 16-byte aligned                              */
+    GDN_ERR_CUDA = -4,           /* a CUDA runtime/driver call or kernel launch failed         */
+    GDN_ERR_DEVICE_TIMEOUT = -5  /* a bounded device-side wait gave up (gdn_device_status)     */
+};
+
+/*
+ * gdn_forward -- one causal or bidirectional pass over T tokens.
+ *
+ * Supported shapes:
+ *   bf16 (chunkwise tensor-core kernel): dk = 128, dv in {64, 128}.
+ *   fp32, or any dtype with GDN_RECURRENT: dk, dv multiples of 32, <= 128.
+ * T >= 1 of any value (a ragged last chunk is handled).  B*H <= 65535.
+ */
+int gdn_forward(const void *q, const void *k, const void *v,
+                const float *beta, const float *decay,
+                const float *state_in, float *state_out, void *o,
+                int B, int H, int T, int dk, int dv, int mode, void *stream);
+
+/*
+ * gdn_rollout -- n_chunks consecutive causal chunks of Tc tokens, the final
+ * state of chunk c being the initial state of chunk c+1 (the streaming
+ * linear-attention cache).  Equal to n_chunks gdn_forward(GDN_CAUSAL) calls
+ * with the state threaded between them.
+ *   q, k [n_chunks, B, H, Tc, dk]; v, o [n_chunks, B, H, Tc, dv];
+ *   beta, decay [n_chunks, B, H, Tc]; state_in/state_out [B, H, dk, dv] (NULL
+ *   allowed); chunk_states NULL or [n_chunks, B, H, dk, dv]: the state after
+ *   each chunk.  GDN_BIDI is rejected (GDN_ERR_UNSUPPORTED).
+ */
+int gdn_rollout(const void *q, const void *k, const void *v,
+                const float *beta, const float *decay,
+                const float *state_in, float *state_out, float *chunk_states,
+                void *o, int B, int H, int n_chunks, int Tc, int dk, int dv,
+                int mode, void *stream);
+
+/*
+ * gdn_forward_host -- gdn_forward on HOST buffers (same layouts).  Copies the
+ * inputs to the device, runs gdn_forward, copies o (and state_out if given)
+ * back, and synchronises `stream` before returning.  Device buffers are taken
+ * stream-ordered and released before return.  Pinned host memory gives
+ * asynchronous copies; pageable memory works but is slower.
+ */
+int gdn_forward_host(const void *q, const void *k, const void *v,
+                     const float *beta, const float *decay,
+                     const float *state_in, float *state_out, void *o,
+                     int B, int H, int T, int dk, int dv, int mode, void *stream);
+
+/*
+ * gdn_device_status -- synchronises `stream` and reports (and clears) the
+ * library's device-side error word: GDN_OK, or GDN_ERR_DEVICE_TIMEOUT if a
+ * bounded wait inside a kernel gave up since the last call, or GDN_ERR_CUDA.
+ */
+int gdn_device_status(void *stream);
+
+/* Message for the last non-zero return on this thread ("" if none). */
+const char *gdn_last_error(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+/*
+ * gdn_kernel_launches -- number of CUDA kernels this library has launched in
+ * this process (all devices, all threads).  For launch accounting in
+ * benchmarks and tests; reading it has no side effects.
+ */
+long long gdn_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,84 @@
+"""ctypes wrapper around the fp64 C oracle (test infrastructure only).
+
+Inputs are numpy arrays in the library's layouts; they are converted to
+contiguous float64 before the call, and results come back as float64.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_gdn_forward.argtypes = [dp] * 8 + [ctypes.c_int] * 7
+        lib.oracle_gdn_forward.restype = ctypes.c_int
+        lib.oracle_gdn_rollout.argtypes = [dp] * 9 + [ctypes.c_int] * 7
+        lib.oracle_gdn_rollout.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    return x.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_threads():
+    return max(1, os.cpu_count() or 1)
+
+
+def gdn_forward(q, k, v, beta, decay, state_in=None, bidi=False, n_threads=None):
+    """q,k [B,H,T,dk]; v [B,H,T,dv]; beta, decay [B,H,T]; state_in [B,H,dk,dv] or None.
+
+    Returns (o [B,H,T,dv], state_out [B,H,dk,dv] causal or [2,B,H,dk,dv] bidi).
+    """
+    q, k, v, beta, decay = map(_f64, (q, k, v, beta, decay))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and v.shape[:3] == (B, H, T)
+    assert beta.shape == (B, H, T) and decay.shape == (B, H, T)
+    s_in = None if state_in is None else _f64(state_in)
+    if s_in is not None:
+        assert s_in.shape == (B, H, dk, dv)
+    o = np.zeros((B, H, T, dv), dtype=np.float64)
+    s_out = np.zeros(((2,) if bidi else ()) + (B, H, dk, dv), dtype=np.float64)
+    rc = load().oracle_gdn_forward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(s_in), _ptr(s_out),
+        _ptr(o), B, H, T, dk, dv, 1 if bidi else 0, n_threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle_gdn_forward failed ({rc})")
+    return o, s_out
+
+
+def gdn_rollout(q, k, v, beta, decay, state_in=None, n_threads=None):
+    """Chunk-major inputs q,k [n,B,H,Tc,dk]; v [n,B,H,Tc,dv]; gates [n,B,H,Tc].
+
+    Returns (o [n,B,H,Tc,dv], state_out [B,H,dk,dv], chunk_states [n,B,H,dk,dv]).
+    """
+    q, k, v, beta, decay = map(_f64, (q, k, v, beta, decay))
+    n, B, H, Tc, dk = q.shape
+    dv = v.shape[-1]
+    s_in = None if state_in is None else _f64(state_in)
+    o = np.zeros((n, B, H, Tc, dv), dtype=np.float64)
+    s_out = np.zeros((B, H, dk, dv), dtype=np.float64)
+    cs = np.zeros((n, B, H, dk, dv), dtype=np.float64)
+    rc = load().oracle_gdn_rollout(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(s_in), _ptr(s_out),
+        _ptr(cs), _ptr(o), B, H, n, Tc, dk, dv, n_threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle_gdn_rollout failed ({rc})")
+    return o, s_out, cs

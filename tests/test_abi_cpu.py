@@ -1,0 +1,100 @@
+"""Host-only checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments with the documented codes before
+launching anything.  No call here reaches a CUDA API (every case fails
+validation first), so these run without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_149_b200 import build, gdn
+    build.build()
+    return gdn.load_library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w ]*[\s*]+(gdn_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_device_status", "gdn_kernel_launches",
+              "gdn_last_error", "gdn_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/gdn.h but not exported"
+
+
+def test_version(lib):
+    assert lib.gdn_version() >= 10000
+
+
+# Fake but 16-byte-aligned addresses: never dereferenced, because every case
+# below fails host-side validation before any CUDA call.
+P = ctypes.c_void_p(0x10000)
+PM = ctypes.c_void_p(0x10008)   # misaligned
+
+
+def fwd(lib, q=P, k=P, v=P, beta=P, decay=P, sin=None, sout=None, o=P,
+        B=1, H=1, T=64, dk=128, dv=128, mode=0):
+    return lib.gdn_forward(q, k, v, beta, decay, sin, sout, o, B, H, T, dk, dv, mode, None)
+
+
+@pytest.mark.parametrize("which", ["q", "k", "v", "beta", "decay", "o"])
+def test_null_required_pointer(lib, which):
+    rc = fwd(lib, **{which: None})
+    assert rc == -1 and b"non-NULL" in lib.gdn_last_error()
+
+
+@pytest.mark.parametrize("B,H,T", [(0, 1, 1), (1, 0, 1), (1, 1, 0), (1, 1, -5), (-1, 2, 3)])
+def test_nonpositive_sizes(lib, B, H, T):
+    assert fwd(lib, B=B, H=H, T=T) == -1
+
+
+def test_bad_mode_bits(lib):
+    assert fwd(lib, mode=8) == -1
+    assert b"mode" in lib.gdn_last_error()
+
+
+@pytest.mark.parametrize("dk,dv", [(48, 128), (128, 40), (160, 128), (128, 256), (0, 64), (16, 16)])
+def test_unsupported_head_dims(lib, dk, dv):
+    assert fwd(lib, dk=dk, dv=dv) == -2
+
+
+def test_too_many_heads(lib):
+    assert fwd(lib, B=256, H=256) == -2
+
+
+@pytest.mark.parametrize("which", ["q", "k", "v", "beta", "decay", "o", "sin", "sout"])
+def test_misaligned_pointer(lib, which):
+    rc = fwd(lib, **{which: PM})
+    assert rc == -3 and b"aligned" in lib.gdn_last_error()
+
+
+def test_rollout_rejects_bidi_and_bad_chunks(lib):
+    r = lambda **kw: lib.gdn_rollout(P, P, P, P, P, None, None, kw.get("cs"), P, 1, 1,
+                                     kw.get("n", 2), 64, 128, 128, kw.get("mode", 0), None)
+    assert r(mode=1) == -2
+    assert r(n=0) == -1
+    assert r(cs=PM) == -3
+
+
+def test_host_entry_validates_first(lib):
+    rc = lib.gdn_forward_host(None, P, P, P, P, None, None, P, 1, 1, 64, 128, 128, 0, None)
+    assert rc == -1
+
+
+def test_last_error_is_per_call(lib):
+    fwd(lib, B=0)
+    assert lib.gdn_last_error() != b""
