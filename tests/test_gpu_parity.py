@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 
 # which kernels serve bf16 inputs: the chunkwise tensor-core kernel (default)
 # and the token-by-token cross-check kernel
-BF16_KERNELS = ["recurrent"]
+BF16_KERNELS = ["tc", "recurrent"]
 
 
 def run_gpu(inp, bidi, recurrent):
