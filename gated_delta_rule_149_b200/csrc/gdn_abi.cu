@@ -229,6 +229,40 @@ int gdn_forward_host(const void *q, const void *k, const void *v, const float *b
     }
 }
 
+int gdn_forward_noalloc(const void *q, const void *k, const void *v, const float *beta,
+                        const float *decay, const float *state_in, float *state_out, void *o,
+                        int B, int H, int T, int dk, int dv, int mode, void *stream)
+{
+    try {
+        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                              mode, "T");
+        if (rc != GDN_OK) return rc;
+        if (mode & (GDN_FP32 | GDN_RECURRENT))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_noalloc runs the bf16 chunkwise kernel only (no GDN_FP32 / "
+                        "GDN_RECURRENT)");
+        gdn::FwdArgs a = make_args(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                                   mode);
+        if (!gdn::chunk_tc_supported(a))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_noalloc needs dk = 128 and dv in {64, 128} (got dk=%d, dv=%d)",
+                        dk, dv);
+        if (a.bidi) {
+            const size_t need = (size_t)B * H * (size_t)((T + 63) / 64) * (size_t)(dv / 64);
+            if (need > gdn::noalloc_capacity())
+                return fail(GDN_ERR_UNSUPPORTED,
+                            "gdn_forward_noalloc: bidirectional call needs %zu arrival counters "
+                            "(B*H*ceil(T/64)*dv/64) but the static scratch holds %zu; split the "
+                            "batch or use gdn_forward", need, gdn::noalloc_capacity());
+        }
+        cudaError_t err = gdn::launch_chunk_tc_noalloc(a, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return fail(GDN_ERR_CUDA, "launch failed: %s", cudaGetErrorString(err));
+        return ok();
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in gdn_forward_noalloc");
+    }
+}
+
 int gdn_device_status(void *stream)
 {
     int err = 0;

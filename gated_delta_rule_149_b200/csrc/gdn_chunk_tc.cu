@@ -738,6 +738,81 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
     return err;
 }
 
+// ------------------------------------------------------ allocation-free variant
+//
+// Some callers cannot allocate device memory while they run this library:
+// plugins hosted by a framework that owns every byte of device memory (media
+// and real-time video pipelines, inference engines with a fixed memory plan),
+// and streaming loops that must not touch an allocator mid-run because a pool
+// allocation can block or grow the footprint at an unpredictable moment.  For
+// them the bidirectional arrival counters (the only scratch this kernel needs)
+// live in a fixed file-scope device array instead of a stream-ordered
+// allocation.  Every device that loads this library holds the array (1 MiB)
+// until the process exits.
+
+constexpr size_t kNoAllocCounters = (size_t)1 << 18;   // 262,144 counters = 1 MiB
+static __device__ __align__(256) int g_noalloc_counters[kNoAllocCounters];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+int *g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+size_t noalloc_capacity() { return kNoAllocCounters; }
+
+cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream)
+{
+    CUtensorMap mq, mk, mv;
+    const int BH = a.B * a.H;
+    if (!make_map(&mq, a.q, a.dk, a.T, BH) || !make_map(&mk, a.k, a.dk, a.T, BH) ||
+        !make_map(&mv, a.v, a.dv, a.T, BH))
+        return cudaErrorInvalidValue;
+
+    TcParams p;
+    p.beta = a.beta; p.decay = a.decay; p.state_in = a.state_in; p.state_out = a.state_out;
+    p.o = static_cast<__nv_bfloat16 *>(a.o);
+    p.BH = BH; p.T = a.T; p.dv = a.dv;
+    p.n_chunks = (a.T + kC - 1) / kC;
+    p.n_slices = a.dv / kDVS;
+    p.counters = nullptr;
+    p.debug = nullptr;
+    cudaError_t err = device_error_word(&p.err);
+    if (err != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSmemAlloc);
+    if (err != cudaSuccess) return err;
+
+    if (a.bidi) {
+        const size_t n_cnt = (size_t)BH * p.n_chunks * p.n_slices;
+        if (n_cnt > kNoAllocCounters) return cudaErrorInvalidValue;   // checked by the caller too
+        int dev = 0;
+        err = cudaGetDevice(&dev);
+        if (err != cudaSuccess) return err;
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        {
+            // Host code cannot use the array's name as a device address: look the
+            // address up once per device, with that device current.
+            std::lock_guard<std::mutex> lock(g_noalloc_mu);
+            if (!g_noalloc_ptr[dev]) {
+                void *ptr = nullptr;
+                err = cudaGetSymbolAddress(&ptr, g_noalloc_counters);
+                if (err != cudaSuccess) return err;
+                g_noalloc_ptr[dev] = static_cast<int *>(ptr);
+            }
+            p.counters = g_noalloc_ptr[dev];
+        }
+        // the array keeps the previous call's contents: the counters must start at zero
+        err = cudaMemsetAsync(p.counters, 0, n_cnt * sizeof(int), stream);
+        if (err != cudaSuccess) return err;
+    }
+    dim3 grid(p.n_slices, a.bidi ? 2 : 1, BH);
+    gdn_chunk_tc_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, p);
+    err = cudaGetLastError();
+    if (err == cudaSuccess) count_launches(1);
+    return err;
+}
+
 }  // namespace gdn
 
 // Test hook (not part of the documented ABI): when set to a device buffer of

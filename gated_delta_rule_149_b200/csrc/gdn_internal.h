@@ -25,6 +25,11 @@ cudaError_t launch_recurrent(const FwdArgs &a, cudaStream_t stream);
 bool chunk_tc_supported(const FwdArgs &a);
 cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream);
 
+// Allocation-free variant of launch_chunk_tc: the bidirectional arrival
+// counters come from a fixed static device array of noalloc_capacity() ints.
+size_t noalloc_capacity();
+cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream);
+
 // Device-side error word (set by bounded waits that gave up).
 cudaError_t device_error_word(int **ptr);
 

@@ -47,6 +47,8 @@ def load_library():
         lib.gdn_forward.restype = i
         lib.gdn_forward_host.argtypes = [vp] * 8 + [i] * 6 + [vp]
         lib.gdn_forward_host.restype = i
+        lib.gdn_forward_noalloc.argtypes = [vp] * 8 + [i] * 6 + [vp]
+        lib.gdn_forward_noalloc.restype = i
         lib.gdn_rollout.argtypes = [vp] * 9 + [i] * 7 + [vp]
         lib.gdn_rollout.restype = i
         lib.gdn_device_status.argtypes = [vp]

@@ -111,6 +111,38 @@ int gdn_forward_host(const void *q, const void *k, const void *v,
                      int B, int H, int T, int dk, int dv, int mode, void *stream);
 
 /*
+ * gdn_forward_noalloc -- gdn_forward that allocates no device memory.
+ *
+ * The paper has no counterpart: this entry point exists for callers that
+ * cannot allocate device memory while they run this library -- plugins hosted
+ * by a framework that owns all device memory (media and real-time video
+ * pipelines, inference engines with a fixed memory plan) and streaming loops
+ * that must never wait on an allocator mid-run.  gdn_forward takes its only
+ * workspace (the bidirectional arrival counters) stream-ordered; this variant
+ * uses a fixed 1 MiB static device array instead, which every device that
+ * loads the library holds until the process exits.
+ *
+ * Same arguments and layouts as gdn_forward; the caller still provides every
+ * input and output buffer.  Limits: bf16 chunkwise kernel only (dk = 128,
+ * dv in {64, 128}; GDN_FP32 and GDN_RECURRENT return GDN_ERR_UNSUPPORTED);
+ * a bidirectional call needs B*H*ceil(T/64)*(dv/64) <= 262144 counters, and a
+ * larger one returns GDN_ERR_UNSUPPORTED with the sizes in gdn_last_error()
+ * before anything is launched.  Causal calls need no scratch.
+ *
+ * The first call on a device looks up the array's device address (and may
+ * load the library's device code): make that first call before any stream
+ * capture.  All calls share the one array; the library clears the counters a
+ * call uses before its kernel runs, so back-to-back calls on one stream are
+ * fine, but calls that overlap on the GPU (other streams, other threads) race
+ * on it and give wrong results.  Never allocates, frees or calls an allocating
+ * library routine.
+ */
+int gdn_forward_noalloc(const void *q, const void *k, const void *v,
+                        const float *beta, const float *decay,
+                        const float *state_in, float *state_out, void *o,
+                        int B, int H, int T, int dk, int dv, int mode, void *stream);
+
+/*
  * gdn_device_status -- synchronises `stream` and reports (and clears) the
  * library's device-side error word: GDN_OK, or GDN_ERR_DEVICE_TIMEOUT if a
  * bounded wait inside a kernel gave up since the last call, or GDN_ERR_CUDA.

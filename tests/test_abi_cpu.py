@@ -26,7 +26,8 @@ def declared_functions():
 
 def test_header_declares_the_abi():
     names = declared_functions()
-    for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_device_status", "gdn_kernel_launches",
+    for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_forward_noalloc",
+              "gdn_device_status", "gdn_kernel_launches",
               "gdn_last_error", "gdn_version"):
         assert n in names
 
@@ -98,3 +99,16 @@ def test_host_entry_validates_first(lib):
 def test_last_error_is_per_call(lib):
     fwd(lib, B=0)
     assert lib.gdn_last_error() != b""
+
+
+def test_noalloc_rejects_before_launch(lib):
+    """The allocation-free entry point refuses what its static scratch cannot
+    hold, and the modes it does not run, before any CUDA call."""
+    f = lambda T=64, dk=128, dv=128, mode=1: lib.gdn_forward_noalloc(
+        P, P, P, P, P, None, None, P, 1, 1, T, dk, dv, mode, None)
+    assert f(T=64 * 262145) == -2                      # 524290 counters > 262144
+    assert b"262144" in lib.gdn_last_error()
+    assert f(mode=1 | 2) == -2                          # fp32
+    assert f(mode=1 | 4) == -2                          # recurrent kernel
+    assert f(dk=64) == -2
+    assert f(T=0) == -1
