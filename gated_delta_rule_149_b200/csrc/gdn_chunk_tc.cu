@@ -16,20 +16,23 @@
 //     U    = U~ - W H_prev                                       (serial step)
 //     O    = diag(gamma) Q H_prev + P U
 //     H    = gamma_end H_prev + K^T diag(2^(G_end - G)) U          (serial step)
-// Only 2^(G_i - G_j) with j at or before i is used.  It is formed as
-// 2^(G_i - G_m) * 2^(G_m - G_j) around the chunk's mid-range G_m when the
-// chunk's total decay is at most 2^-240 (each factor then stays a normal
-// float), and directly otherwise, so nothing overflows however strong the decay.
+// Only 2^(G_i - G_j) with j at or before i is used.  It is formed as a product
+// of a row and a column factor: around the middle of the half-chunk when i and
+// j lie in the same 32-token half, around the boundary between the halves
+// when they do not (both factors are then <= 1); when a half-chunk decays by
+// more than 2^-240 (a factor could leave the normal range) it is formed
+// directly, so nothing overflows however strong the decay.
 //
-// One CTA per (64-wide dv slice, direction, batch*head), 10 warps:
-//   warps 0-3  chain:  fp32 state in registers (thread d owns row d of the
-//                      dk x 64 slice); U, state and output epilogues;
-//   warps 4-7  prep:   gates, masks, the triangular solve (16x16 diagonal
+// One CTA per (64-wide dv slice, direction, batch*head), 19 warps:
+//   warps 0-7   chain: fp32 state in registers (each thread owns 32 columns
+//                      of one row of the dk x 64 slice); U, state and output
+//                      epilogues;
+//   warps 8-15  prep:  gates, masks, the triangular solve (16x16 diagonal
 //                      blocks by substitution, the rest with tf32 mma.sync),
 //                      T1 = T diag(b gamma), T2 = T diag(b), gamma*Q, W;
-//   warp 8     TMA:    q, k and the v slice of each chunk, three stages ahead;
-//   warp 9     MMA:    issues every tcgen05.mma from one thread, in whatever
-//                      order the mbarriers allow (serial-chain products first).
+//   warp 16     TMA:   q, k and the v slice of each chunk, three stages ahead;
+//   warp 17     MMA:   issues the state-independent products ([Q;K]K^T, W, U~);
+//   warp 18     MMA:   issues the serial-chain products (W H, Q H, K^T Ubar, P U).
 // Tensor-core products (bf16 operands, fp32 accumulation in TMEM):
 //     [Q;K] K^T        M=128 N=64  K=dk     -> QK^T, KK^T
 //     W^T = K^T T1^T   M=128 N=64  K=64
@@ -55,6 +58,7 @@
 namespace gdn {
 
 extern float *g_debug_dump;
+extern long long *g_prof_buf;
 
 namespace {
 
@@ -63,10 +67,11 @@ using namespace ptx;
 constexpr int kC = 64;           // chunk length
 constexpr int kDK = 128;         // key dim served by this kernel
 constexpr int kDVS = 64;         // dv columns per CTA
-constexpr int kThreads = 320;    // 4 chain + 4 prep + TMA + MMA warps
+constexpr int kThreads = 608;    // 8 chain + 8 prep + TMA + 2 MMA-issue warps
+constexpr int kChainThreads = 256, kPrepThreads = 256;
 constexpr int kNS = 3;           // input stages
 constexpr int kLDA = 68;         // fp32 row stride of the solve buffers
-constexpr int kBarPrep = 1, kBarChain = 2;   // named barriers, 128 threads each
+constexpr int kBarPrep = 1, kBarChain = 2;   // named barriers of the prep and chain groups
 
 // TMEM columns (fp32 accumulators)
 constexpr uint32_t kColD1 = 0;     // [Q;K] K^T   (M=128)
@@ -88,17 +93,19 @@ constexpr uint32_t kOffA = kOffH + 16384;              // fp32 [64][68], scan or
 constexpr uint32_t kOffT1 = kOffA;                     // T1, T2 (bf16) reuse A after the solve
 constexpr uint32_t kOffT2 = kOffA + 8192;
 constexpr uint32_t kOffT = kOffA + 64 * kLDA * 4;      // fp32 [64][68], scan order
-constexpr uint32_t kOffY = kOffT + 64 * kLDA * 4;      // 4 warps x 16 x 8 fp32
-constexpr uint32_t kGateFloats = 9 * 64;               // per buffer, see GateIdx
-constexpr uint32_t kOffGates = kOffY + 4 * 512;        // 2 buffers
+constexpr uint32_t kGateFloats = 10 * 64;              // per buffer, see GateIdx
+constexpr uint32_t kOffGates = kOffT + 64 * kLDA * 4;  // 2 buffers
 constexpr uint32_t kOffBar = kOffGates + 2 * kGateFloats * 4;
-constexpr uint32_t kSmemBytes = kOffBar + 512;
+constexpr uint32_t kOffProf = kOffBar + 512;            // 32 x 8 B (profiling builds)
+constexpr uint32_t kSmemBytes = kOffProf + 256;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;     // alignment slack
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(kOffA % 1024 == 0 && kOffT2 % 1024 == 0 && kOffP % 1024 == 0, "tile alignment");
 
 // gate arrays (64 floats each, physical token order unless noted)
-enum GateIdx { gG = 0, gGam, gBet, gBG, gEb, gRf, gCf, gCfl /* scan order */, gScal };
+// G (log2 cumulative decay), gamma = 2^G, beta, beta*gamma, 2^(G_end - G), row/column
+// factors of the decay products (A: same half of the chunk, B: across halves), scalars
+enum GateIdx { gG = 0, gGam, gBet, gBG, gEb, gRA, gRB, gCA, gCB, gScal };
 
 constexpr uint32_t kIdM1 = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdW = idesc_bf16(128, 64, true, false);
@@ -117,8 +124,41 @@ struct TcParams {
     int *counters;       // bidi arrival counters [BH][n_chunks][n_slices], zeroed
     int *err;            // device error word
     float *debug;        // optional: first-chunk intermediates of CTA (0,0,0)
+    long long *prof;     // optional (profiling builds): per-phase cycle counts of CTA (0,0,0)
     int BH, T, dv, n_chunks, n_slices;
+    int predict;         // bidi: all CTAs resident, first writer of each tile known in advance
 };
+
+// Phase timers for profiling builds (-DGDN_PROFILE): each role's leader
+// thread in CTA (0,0,0) adds the cycles since its previous mark to a slot.
+#ifdef GDN_PROFILE
+// Per-slot cycle accumulators live in shared memory (kOffProf); the leader
+// thread of each role adds the cycles since its previous mark.
+#define PROF_DECL(lead)                                                                     \
+    const bool prof_on = p.prof != nullptr && (lead) && blockIdx.x == 0 && blockIdx.y == 0 && \
+                         blockIdx.z == 0;                                                   \
+    long long prof_t = clock64();                                                           \
+    long long *prof_s = reinterpret_cast<long long *>(x.smem + kOffProf);
+#define PROF_MARK(slot)                                \
+    do {                                               \
+        if (prof_on) {                                 \
+            const long long prof_n = clock64();        \
+            prof_s[slot] += prof_n - prof_t;           \
+            prof_t = prof_n;                           \
+        }                                              \
+    } while (0)
+#define PROF_FLUSH() \
+    do {             \
+    } while (0)
+#else
+#define PROF_DECL(lead)
+#define PROF_MARK(slot) \
+    do {                \
+    } while (0)
+#define PROF_FLUSH() \
+    do {             \
+    } while (0)
+#endif
 
 // Debug dump layout (floats): 6 TMEM snapshots of 128 lanes x 64 columns
 // (D1, W^T, U~, U, O, D_S) then the 64 x 64 solve result in scan order.
@@ -128,8 +168,8 @@ constexpr int kDbgD1 = 0, kDbgW = 8192, kDbgUt = 16384, kDbgU = 24576, kDbgO = 3
 // mbarriers
 struct Bars {
     uint64_t stage_full[kNS], stage_empty[kNS];
-    uint64_t d1_full, d1_empty, tp_full, wu_full, wmn_full, wmn_empty;
-    uint64_t chain_full, u_full, s_full, h_full, drain;
+    uint64_t d1_full, d1_empty, tp_full, wu_full, wmn_full, dw_empty;
+    uint64_t chain_full, u_full, s_full, h_full, drain, drain2;
     uint64_t o_full[2], do_empty[2], du_empty[2], p_empty[2], g_full[2], g_empty[2];
     uint32_t tmem_slot;
     int abort_flag;
@@ -143,16 +183,6 @@ __device__ __forceinline__ unsigned long long globaltimer()
     unsigned long long t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
     return t;
-}
-
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    return ok != 0;
 }
 
 // Bounded wait on an mbarrier phase; on timeout records the error and raises
@@ -173,21 +203,21 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     return false;
 }
 
-__device__ __forceinline__ void named_bar(int id)
+__device__ __forceinline__ void named_bar(int id, int count)
 {
-    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Named barrier over a 128-thread group that also ORs a predicate across it,
 // so that every thread of the group takes the same abort decision.
-__device__ __forceinline__ bool named_bar_any(int id, bool pred)
+__device__ __forceinline__ bool named_bar_any(int id, int count, bool pred)
 {
     uint32_t r;
     asm volatile("{\n\t.reg .pred p, q;\n\t"
                  "setp.ne.u32 p, %1, 0;\n\t"
-                 "bar.red.or.pred q, %2, 128, p;\n\t"
+                 "bar.red.or.pred q, %2, %3, p;\n\t"
                  "selp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r) : "r"((uint32_t)pred), "r"(id) : "memory");
+                 : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(count) : "memory");
     return r != 0;
 }
 
@@ -204,27 +234,21 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  "r"(d) : "memory");
 }
 
-// Writes 64 fp32 values as one 128-byte bf16 row of a 128B-swizzled tile.
-__device__ __forceinline__ void store_row_bf16(uint32_t tile, uint32_t row, const float *x)
+// Writes 32 fp32 values as half (64 bytes, 16-byte chunks 4h..4h+3) of a
+// 128-byte bf16 row of a 128B-swizzled tile.
+__device__ __forceinline__ void store_half_row_bf16(uint32_t tile, uint32_t row, int h, const float *x)
 {
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-        st_shared_v4(tile + sw128_off(row, 8 * q), pack_bf16(x[8 * q + 0], x[8 * q + 1]),
+    for (int q = 0; q < 4; ++q)
+        st_shared_v4(tile + sw128_off(row, 32 * h + 8 * q), pack_bf16(x[8 * q + 0], x[8 * q + 1]),
                      pack_bf16(x[8 * q + 2], x[8 * q + 3]), pack_bf16(x[8 * q + 4], x[8 * q + 5]),
                      pack_bf16(x[8 * q + 6], x[8 * q + 7]));
 }
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float *x)
-{
-    tmem_ld32(taddr, x);
-    tmem_ld32(taddr + 32, x + 32);
-    tmem_wait_ld();
-}
-
-__device__ __forceinline__ void dbg_rows(float *dst, int row, const float *x)
+__device__ __forceinline__ void dbg_half(float *dst, int row, int h, const float *x)
 {
 #pragma unroll
-    for (int e = 0; e < 64; ++e) dst[row * 64 + e] = x[e];
+    for (int e = 0; e < 32; ++e) dst[row * 64 + 32 * h + e] = x[e];
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float x)
@@ -244,78 +268,113 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 }
 
 // T = (I + A)^-1 for a strictly lower-triangular 64 x 64 fp32 A (scan order),
-// by the 128 prep threads.  16 x 16 diagonal blocks by forward substitution
-// (one column per thread), then the off-diagonal blocks by distance from the
-// diagonal, T_ab = -T_aa sum_{m=b}^{a-1} A_am T_mb, on tf32 tensor cores
-// (one 16 x 8 column strip per warp and step).  The upper triangle of Ts is
-// zero on entry and stays zero.
-__device__ void solve_unit_lower(const float *As, float *Ts, float *Yall, int pt)
+// by the 256 prep threads, in four barrier-separated steps:
+//   1. the four 16 x 16 diagonal blocks D_a by forward substitution (one
+//      column per thread, right-looking so one FMA per step is serial);
+//   2. the two 16 x 16 blocks below them inside each 32 x 32 half,
+//      T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2 (tf32 mma.sync);
+//   3. Y = A[32:64, 0:32] T[0:32, 0:32]                  (tf32 mma.sync)
+//   4. T[32:64, 0:32] = -T[32:64, 32:64] Y               (tf32 mma.sync)
+// Products skip the k-steps that the triangular factors make zero.  The
+// upper-right 32 x 32 block of Ts is scratch for the intermediate products;
+// every other upper-triangular entry of Ts stays zero (callers mask the
+// scratch block out when they read T).
+__device__ __forceinline__ void solve_diag_blocks(const float *As, float *Ts, int pt)
 {
     if (pt < 64) {
         const int a = pt >> 4, c = pt & 15;
         const float *Ab = As + (16 * a) * kLDA + 16 * a;
-        float x[16];
+        float x[16], acc[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) acc[r] = 0.f;
 #pragma unroll
-        for (int r = 1; r < 16; ++r) {
-            float s = 0.f;
+        for (int m = 0; m < 16; ++m) {
+            x[m] = (m == c) ? 1.f : ((m > c) ? -acc[m] : 0.f);
 #pragma unroll
-            for (int m = 0; m < r; ++m) s = fmaf(Ab[r * kLDA + m], x[m], s);
-            if (r > c) x[r] = -s;
+            for (int r = m + 1; r < 16; ++r) acc[r] = fmaf(Ab[r * kLDA + m], x[m], acc[r]);
         }
         float *Tb = Ts + (16 * a) * kLDA + 16 * a;
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tb[r * kLDA + c] = x[r];
     }
-    named_bar(kBarPrep);
-    const int pw = pt >> 5, lane = pt & 31, g = lane >> 2, q = lane & 3;
-    float *Y = Yall + pw * 128;   // 16 x 8, row-major
-    for (int dist = 1; dist <= 3; ++dist) {
-        const int items = (4 - dist) * 2;
-        for (int it = pw; it < items; it += 4) {
-            const int blk = it >> 1, nt = it & 1, a = dist + blk, b = blk;
-            const int col0 = 16 * b + 8 * nt;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int kk = 16 * b; kk < 16 * a; kk += 8) {
-                uint32_t af[4], bf[2];
-                const float *Ar = As + (16 * a + g) * kLDA + kk + q;
-                af[0] = to_tf32(Ar[0]);
-                af[1] = to_tf32(Ar[8 * kLDA]);
-                af[2] = to_tf32(Ar[4]);
-                af[3] = to_tf32(Ar[8 * kLDA + 4]);
-                const float *Br = Ts + (kk + q) * kLDA + col0 + g;
-                bf[0] = to_tf32(Br[0]);
-                bf[1] = to_tf32(Br[4 * kLDA]);
-                mma_tf32(d, af, bf);
-            }
-            Y[g * 8 + 2 * q] = d[0];
-            Y[g * 8 + 2 * q + 1] = d[1];
-            Y[(g + 8) * 8 + 2 * q] = d[2];
-            Y[(g + 8) * 8 + 2 * q + 1] = d[3];
-            __syncwarp();
-            float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kk = 0; kk < 16; kk += 8) {
-                uint32_t af[4], bf[2];
-                const float *Dr = Ts + (16 * a + g) * kLDA + 16 * a + kk + q;
-                af[0] = to_tf32(Dr[0]);
-                af[1] = to_tf32(Dr[8 * kLDA]);
-                af[2] = to_tf32(Dr[4]);
-                af[3] = to_tf32(Dr[8 * kLDA + 4]);
-                bf[0] = to_tf32(Y[(kk + q) * 8 + g]);
-                bf[1] = to_tf32(Y[(kk + q + 4) * 8 + g]);
-                mma_tf32(e, af, bf);
-            }
-            float *Tr = Ts + (16 * a + g) * kLDA + col0 + 2 * q;
-            Tr[0] = -e[0];
-            Tr[1] = -e[1];
-            Tr[8 * kLDA] = -e[2];
-            Tr[8 * kLDA + 1] = -e[3];
-            __syncwarp();
-        }
-        named_bar(kBarPrep);
+    named_bar(kBarPrep, kPrepThreads);
+}
+
+// D(16x8) += A[rows r0.., cols k0..k0+8*nk) * B[rows k0.., cols c0..c0+8), fp32 smem, tf32 MMA
+__device__ __forceinline__ void mma_strip(float (&d)[4], const float *Am, int r0, const float *Bm,
+                                          int c0, int k0, int nk, int g, int q)
+{
+    for (int s = 0; s < nk; ++s) {
+        const int kk = k0 + 8 * s;
+        uint32_t af[4], bf[2];
+        const float *Ar = Am + (r0 + g) * kLDA + kk + q;
+        af[0] = to_tf32(Ar[0]);
+        af[1] = to_tf32(Ar[8 * kLDA]);
+        af[2] = to_tf32(Ar[4]);
+        af[3] = to_tf32(Ar[8 * kLDA + 4]);
+        const float *Br = Bm + (kk + q) * kLDA + c0 + g;
+        bf[0] = to_tf32(Br[0]);
+        bf[1] = to_tf32(Br[4 * kLDA]);
+        mma_tf32(d, af, bf);
     }
+}
+
+// writes a 16 x 8 accumulator strip (times sgn) at rows r0.., cols c0.. of M
+__device__ __forceinline__ void store_strip(float *M, int r0, int c0, const float (&d)[4], float sgn,
+                                            int g, int q)
+{
+    float *Mr = M + (r0 + g) * kLDA + c0 + 2 * q;
+    Mr[0] = sgn * d[0];
+    Mr[1] = sgn * d[1];
+    Mr[8 * kLDA] = sgn * d[2];
+    Mr[8 * kLDA + 1] = sgn * d[3];
+}
+
+__device__ __forceinline__ void solve_off_diag(const float *As, float *Ts, int pt)
+{
+    const int pw = pt >> 5, lane = pt & 31, g = lane >> 2, q = lane & 3;
+    // step 2: T_ab, (a,b) in {(1,0), (3,2)}; warp = (block, 8-column strip)
+    if (pw < 4) {
+        const int a = (pw >> 1) ? 3 : 1, b = a - 1, nt = pw & 1;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_strip(y, As, 16 * a, Ts, 16 * b + 8 * nt, 16 * b + 8 * nt, 2 - nt, g, q);   // A_ab D_b
+        // Y strip (16 x 8) parked in the scratch block: rows 0..15, cols 32 + 8 pw
+        store_strip(Ts, 0, 32 + 8 * pw, y, 1.f, g, q);
+        __syncwarp();
+        float e[4] = {0.f, 0.f, 0.f, 0.f};
+        // -D_a Y : D_a = T[16a.., 16a..], Y rows are the k index
+        for (int s = 0; s < 2; ++s) {
+            const int kk = 8 * s;
+            uint32_t af[4], bf[2];
+            const float *Dr = Ts + (16 * a + g) * kLDA + 16 * a + kk + q;
+            af[0] = to_tf32(Dr[0]);
+            af[1] = to_tf32(Dr[8 * kLDA]);
+            af[2] = to_tf32(Dr[4]);
+            af[3] = to_tf32(Dr[8 * kLDA + 4]);
+            const float *Yr = Ts + (kk + q) * kLDA + 32 + 8 * pw + g;
+            bf[0] = to_tf32(Yr[0]);
+            bf[1] = to_tf32(Yr[4 * kLDA]);
+            mma_tf32(e, af, bf);
+        }
+        store_strip(Ts, 16 * a, 16 * b + 8 * nt, e, -1.f, g, q);
+    }
+    named_bar(kBarPrep, kPrepThreads);
+    // step 3: Y = A[32:64, 0:32] T[0:32, 0:32] -> scratch rows 0..31, cols 32..63
+    {
+        const int mt = pw >> 2, nt = pw & 3;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_strip(y, As, 32 + 16 * mt, Ts, 8 * nt, 8 * nt, 4 - nt, g, q);
+        store_strip(Ts, 16 * mt, 32 + 8 * nt, y, 1.f, g, q);
+    }
+    named_bar(kBarPrep, kPrepThreads);
+    // step 4: T[32:64, 0:32] = -T[32:64, 32:64] Y
+    {
+        const int mt = pw >> 2, nt = pw & 3;
+        float e[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_strip(e, Ts + 32, 32 + 16 * mt, Ts + 32, 8 * nt, 0, 2 * mt + 2, g, q);
+        store_strip(Ts, 32 + 16 * mt, 8 * nt, e, -1.f, g, q);
+    }
+    named_bar(kBarPrep, kPrepThreads);
 }
 
 struct Ctx {
@@ -328,19 +387,24 @@ struct Ctx {
 };
 
 __device__ __forceinline__ uint32_t stage_addr(const Ctx &x, int i) { return x.sbase + kOffStage + (uint32_t)(i % kNS) * kStageBytes; }
-__device__ __forceinline__ int chunk_of(const Ctx &x, int i) { return x.dir ? (x.NC - 1 - i) : i; }
+template <int DIR>
+__device__ __forceinline__ int chunk_of(const Ctx &x, int i) { return DIR ? (x.NC - 1 - i) : i; }
 __device__ __forceinline__ float *gates_buf(const Ctx &x, int b) { return reinterpret_cast<float *>(x.smem + kOffGates) + b * kGateFloats; }
 
 // ------------------------------------------------------------------ TMA warp
-__device__ void tma_role(const Ctx &x, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+template <int DIR>
+__device__ __forceinline__ void tma_role(const Ctx &x, const CUtensorMap *tmQ, const CUtensorMap *tmK,
                          const CUtensorMap *tmV, const TcParams &p)
 {
     Bars &B = *x.bars;
     int issued = 0;
+    PROF_DECL(true);
     for (int i = 0; i < x.NC; ++i) {
         const int s = i % kNS;
+        PROF_MARK(1);
         if (i >= kNS && !wait_bar(&B.stage_empty[s], ((i / kNS) + 1) & 1, x.abort_flag, p.err, 1)) break;
-        const int c = chunk_of(x, i);
+        PROF_MARK(0);
+        const int c = chunk_of<DIR>(x, i);
         uint8_t *st = x.smem + (stage_addr(x, i) - x.sbase);
         mbar_arrive_expect_tx(&B.stage_full[s], 5 * 8192);
         for (int kb = 0; kb < 2; ++kb) {
@@ -350,6 +414,7 @@ __device__ void tma_role(const Ctx &x, const CUtensorMap *tmQ, const CUtensorMap
         tma_load_3d(st + 32768, tmV, &B.stage_full[s], x.slice * kDVS, c * kC, x.bh);
         issued = i + 1;
     }
+    PROF_FLUSH();
     if (*x.abort_flag) {   // let copies in flight land before the CTA exits
         for (int i = (issued > kNS ? issued - kNS : 0); i < issued; ++i) {
             const unsigned long long t0 = globaltimer();
@@ -359,115 +424,125 @@ __device__ void tma_role(const Ctx &x, const CUtensorMap *tmQ, const CUtensorMap
     }
 }
 
-// ------------------------------------------------------------------ MMA warp
-__device__ void mma_role(const Ctx &x, const TcParams &p)
+// ------------------------------------------------------------------ MMA warps
+// Two issuing threads, each waiting (suspended) on its next products' inputs in
+// a fixed order: one for the state-independent products of the prep pipeline,
+// one for the serial-chain products.  tcgen05.commit tracks the MMAs of the
+// issuing thread only; the mbarrier protocol orders the two streams.
+
+// [Q;K] K^T, then W^T = K^T T1^T and U~ = T2 V, chunk after chunk.
+__device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
 {
     Bars &B = *x.bars;
     const uint32_t tm = x.tmem;
-    const uint32_t sP = x.sbase + kOffP, sW = x.sbase + kOffW, sU = x.sbase + kOffU;
-    const uint32_t sUb = x.sbase + kOffUb, sH = x.sbase + kOffH;
     const uint32_t sT1 = x.sbase + kOffT1, sT2 = x.sbase + kOffT2;
-    int nm1 = 0, nwu = 0, nch = 0, nst = 0;
-    unsigned long long t_last = globaltimer();
-    while (nst < x.NC) {
-        if (*x.abort_flag) break;
-        bool did = false;
-        if (nst < nch && mbar_test(&B.u_full, nst & 1)) {
-            // ---- state products of chunk nst: D_S = K^T Ubar, then O += P U
-            const int i = nst, b = i & 1;
-            const uint32_t sQK = stage_addr(x, i);
-            tc_fence_after();
+    PROF_DECL(true);
+    for (int i = 0; i < x.NC; ++i) {
+        const int b = i & 1;
+        const uint32_t sQK = stage_addr(x, i), sV = sQK + 32768;
+        PROF_MARK(6);
+        if (!wait_bar(&B.stage_full[i % kNS], (i / kNS) & 1, x.abort_flag, p.err, 11)) break;
+        if (i > 0 && !wait_bar(&B.d1_empty, (i - 1) & 1, x.abort_flag, p.err, 12)) break;
+        PROF_MARK(2);
+        tc_fence_after();
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + kColS, sw128_desc(sQK + 8192 + ks * 2048, 16384, 1024),
-                         sw128_desc(sUb + ks * 2048, 8192, 1024), kIdS, ks != 0);
-            mma_commit(&B.s_full);
+                mma_bf16(tm + kColD1, sw128_desc(sQK + kb * 16384 + ks * 32, 16, 1024),
+                         sw128_desc(sQK + kb * 16384 + 8192 + ks * 32, 16, 1024), kIdM1, (kb | ks) != 0);
+        mma_commit(&B.d1_full);
+        PROF_MARK(6);
+        if (!wait_bar(&B.tp_full, i & 1, x.abort_flag, p.err, 13)) break;
+        if (i >= 2 && !wait_bar(&B.du_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 14)) break;
+        if (i >= 1 && !wait_bar(&B.dw_empty, (i - 1) & 1, x.abort_flag, p.err, 19)) break;
+        PROF_MARK(2);
+        tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + kColO0 + 64 * b, sw128_desc(sP + b * 8192 + ks * 32, 16, 1024),
-                         sw128_desc(sU + ks * 2048, 8192, 1024), kIdPU, 1);
-            mma_commit(&B.o_full[b]);
-            mma_commit(&B.p_empty[b]);
-            mma_commit(&B.stage_empty[i % kNS]);
-            ++nst;
-            did = true;
-        } else if (nch < nwu && mbar_test(&B.wmn_full, nch & 1) && mbar_test(&B.h_full, nch & 1) &&
-                   (nch < 2 || mbar_test(&B.do_empty[nch & 1], ((nch >> 1) + 1) & 1))) {
-            // ---- serial-chain products of chunk nch: U -= W H ; O = (gamma Q) H
-            const int i = nch, b = i & 1;
-            const uint32_t sQK = stage_addr(x, i);
-            tc_fence_after();
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tm + kColW, sw128_desc(sQK + 8192 + ks * 2048, 16384, 1024),
+                     sw128_desc(sT1 + ks * 32, 16, 1024), kIdW, ks != 0);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sW + ks * 2048, 8192, 1024),
-                         sw128_desc(sH + ks * 2048, 8192, 1024), kIdUc, 1);
-            mma_commit(&B.chain_full);
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tm + kColO0 + 64 * b, sw128_desc(sQK + kb * 16384 + ks * 32, 16, 1024),
-                             sw128_desc(sH + (kb * 4 + ks) * 2048, 8192, 1024), kIdOq, (kb | ks) != 0);
-            mma_commit(&B.wmn_empty);
-            ++nch;
-            did = true;
-        } else if (nwu < nm1 && mbar_test(&B.tp_full, nwu & 1) &&
-                   (nwu < 2 || mbar_test(&B.du_empty[nwu & 1], ((nwu >> 1) + 1) & 1))) {
-            // ---- W^T = K^T T1^T ; U~ = T2 V
-            const int i = nwu, b = i & 1;
-            const uint32_t sQK = stage_addr(x, i), sV = sQK + 32768;
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + kColW, sw128_desc(sQK + 8192 + ks * 2048, 16384, 1024),
-                         sw128_desc(sT1 + ks * 32, 16, 1024), kIdW, ks != 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sT2 + ks * 32, 16, 1024),
-                         sw128_desc(sV + ks * 2048, 8192, 1024), kIdUt, ks != 0);
-            mma_commit(&B.wu_full);
-            ++nwu;
-            did = true;
-        } else if (nm1 < x.NC && mbar_test(&B.stage_full[nm1 % kNS], (nm1 / kNS) & 1) &&
-                   (nm1 == 0 || mbar_test(&B.d1_empty, (nm1 - 1) & 1))) {
-            // ---- [Q;K] K^T
-            const uint32_t sQK = stage_addr(x, nm1);
-            tc_fence_after();
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tm + kColD1, sw128_desc(sQK + kb * 16384 + ks * 32, 16, 1024),
-                             sw128_desc(sQK + kb * 16384 + 8192 + ks * 32, 16, 1024), kIdM1, (kb | ks) != 0);
-            mma_commit(&B.d1_full);
-            ++nm1;
-            did = true;
-        }
-        if (did) {
-            t_last = globaltimer();
-        } else if (globaltimer() - t_last > kWaitLimitNs) {
-            atomicOr(p.err, 16);
-            *x.abort_flag = 1;
-            break;
-        }
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sT2 + ks * 32, 16, 1024),
+                     sw128_desc(sV + ks * 2048, 8192, 1024), kIdUt, ks != 0);
+        mma_commit(&B.wu_full);
     }
+    PROF_MARK(5);
+    PROF_FLUSH();
     // every issued MMA completes before the CTA releases its TMEM
     mma_commit(&B.drain);
     const unsigned long long t0 = globaltimer();
     while (!mbar_try_wait(&B.drain, 0) && globaltimer() - t0 < kWaitLimitNs) {}
 }
 
-// ------------------------------------------------------------------ prep warps
-__device__ void prep_role(const Ctx &x, const TcParams &p, int pt)
+// U -= W H and O = (gamma Q) H, then D_S = K^T Ubar and O += P U.
+__device__ __forceinline__ void mma_chain_role(const Ctx &x, const TcParams &p)
 {
     Bars &B = *x.bars;
-    const int pw = pt >> 5, lane = pt & 31;
+    const uint32_t tm = x.tmem;
+    const uint32_t sP = x.sbase + kOffP, sW = x.sbase + kOffW, sU = x.sbase + kOffU;
+    const uint32_t sUb = x.sbase + kOffUb, sH = x.sbase + kOffH;
+    PROF_DECL(true);
+    for (int i = 0; i < x.NC; ++i) {
+        const int b = i & 1;
+        const uint32_t sQK = stage_addr(x, i);
+        PROF_MARK(28);
+        if (!wait_bar(&B.wmn_full, i & 1, x.abort_flag, p.err, 15)) break;
+        if (!wait_bar(&B.h_full, i & 1, x.abort_flag, p.err, 16)) break;
+        if (i >= 2 && !wait_bar(&B.do_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 17)) break;
+        PROF_MARK(26);
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sW + ks * 2048, 8192, 1024),
+                     sw128_desc(sH + ks * 2048, 8192, 1024), kIdUc, 1);
+        mma_commit(&B.chain_full);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + kColO0 + 64 * b, sw128_desc(sQK + kb * 16384 + ks * 32, 16, 1024),
+                         sw128_desc(sH + (kb * 4 + ks) * 2048, 8192, 1024), kIdOq, (kb | ks) != 0);
+        PROF_MARK(4);
+        if (!wait_bar(&B.u_full, i & 1, x.abort_flag, p.err, 18)) break;
+        PROF_MARK(27);
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tm + kColS, sw128_desc(sQK + 8192 + ks * 2048, 16384, 1024),
+                     sw128_desc(sUb + ks * 2048, 8192, 1024), kIdS, ks != 0);
+        mma_commit(&B.s_full);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tm + kColO0 + 64 * b, sw128_desc(sP + b * 8192 + ks * 32, 16, 1024),
+                     sw128_desc(sU + ks * 2048, 8192, 1024), kIdPU, 1);
+        mma_commit(&B.o_full[b]);
+        mma_commit(&B.p_empty[b]);
+        mma_commit(&B.stage_empty[i % kNS]);
+        PROF_MARK(3);
+    }
+    PROF_FLUSH();
+    mma_commit(&B.drain2);
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(&B.drain2, 0) && globaltimer() - t0 < kWaitLimitNs) {}
+}
+
+// ------------------------------------------------------------------ prep warps
+// 8 warps (256 threads).  Warp pw reads TMEM lane quarter pw & 3 and handles
+// columns [32 * (pw >> 2), +32) of each row it owns.
+template <int DIR>
+__device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int pt)
+{
+    Bars &B = *x.bars;
+    const int pw = pt >> 5, lane = pt & 31, qd = pw & 3, hf = pw >> 2;
     float *As = reinterpret_cast<float *>(x.smem + kOffA);
     float *Ts = reinterpret_cast<float *>(x.smem + kOffT);
-    float *Yall = reinterpret_cast<float *>(x.smem + kOffY);
-    const uint32_t tm_lane = (uint32_t)(pw * 32) << 16;
+    const uint32_t tm_lane = (uint32_t)(qd * 32) << 16;
     const float *beta_h = p.beta + (size_t)x.bh * x.T;
     const float *decay_h = p.decay + (size_t)x.bh * x.T;
+    // the logical (scan-order) half that this warp's 32 physical columns fall in
+    const bool col_h1 = DIR ? (hf == 1) : (hf == 0);
 
     // raw gates of the next chunk, fetched one chunk ahead (thread pt < 64
     // handles scan position pt)
@@ -476,8 +551,8 @@ __device__ void prep_role(const Ctx &x, const TcParams &p, int pt)
         ra = 1.f;
         rb = 0.f;
         if (pt < 64 && i < x.NC) {
-            const int pp = x.dir ? (63 - pt) : pt;
-            const int t = chunk_of(x, i) * kC + pp;
+            const int pp = DIR ? (63 - pt) : pt;
+            const int t = chunk_of<DIR>(x, i) * kC + pp;
             if (t < x.T) {
                 ra = __ldg(decay_h + t);
                 rb = __ldg(beta_h + t);
@@ -485,16 +560,20 @@ __device__ void prep_role(const Ctx &x, const TcParams &p, int pt)
         }
     };
     load_raw(0);
+    PROF_DECL(pt == 0);
 
     for (int i = 0; i < x.NC; ++i) {
         const int b = i & 1;
         float *gt = gates_buf(x, b);
         const bool dbg = p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
                          blockIdx.z == 0;
+        PROF_MARK(16);
 
         // ---- gates (log2 domain) for chunk i
         if (i >= 2) wait_bar(&B.g_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 2);
-        float gsum = 0.f, bcur = rb;
+        PROF_MARK(8);
+        float gsum = 0.f;
+        const float bcur = rb;
         if (pt < 64) {
             float v = fmaxf(log2f(ra), -120.f);   // decay below 2^-120 acts as 2^-120
 #pragma unroll
@@ -506,222 +585,364 @@ __device__ void prep_role(const Ctx &x, const TcParams &p, int pt)
             gsum = v;
         }
         load_raw(i + 1);
-        if (named_bar_any(kBarPrep, *x.abort_flag)) return;
+        if (named_bar_any(kBarPrep, kPrepThreads, *x.abort_flag)) return;
         if (pt < 64) {
             const float G = (pt >= 32) ? gsum + x.bars->s_wsum : gsum;
-            const int pp = x.dir ? (63 - pt) : pt;
+            const int pp = DIR ? (63 - pt) : pt;
             gt[gG * 64 + pp] = G;
             const float gam = exp2f(G);
             gt[gGam * 64 + pp] = gam;
             gt[gBet * 64 + pp] = bcur;
             gt[gBG * 64 + pp] = bcur * gam;
-            if (pt == 63) gt[gScal * 64] = G;   // G_end
         }
-        named_bar(kBarPrep);
-        const float Gend = gt[gScal * 64];
-        const float Gm = 0.5f * Gend;
-        const bool fact = Gend >= -240.f;
+        named_bar(kBarPrep, kPrepThreads);
+        // references: scan positions 15 (first half), 47 (second half), 31 (boundary)
+        const float R1 = gt[gG * 64 + (DIR ? 48 : 15)];
+        const float R2 = gt[gG * 64 + (DIR ? 16 : 47)];
+        const float Rm = gt[gG * 64 + (DIR ? 32 : 31)];
+        const float G0 = gt[gG * 64 + (DIR ? 63 : 0)];
+        const float G32 = gt[gG * 64 + (DIR ? 31 : 32)];
+        const float Gend = gt[gG * 64 + (DIR ? 0 : 63)];
+        // factorised decay products are exact while every factor is a normal float
+        const bool fact = (G0 - R1) <= 120.f && (R1 - Rm) <= 120.f && (G32 - R2) <= 120.f &&
+                          (R2 - Gend) <= 120.f;
         if (pt < 64) {
             const float G = gt[gG * 64 + pt];
+            const int lp = DIR ? 63 - pt : pt;
+            const float Rh = (lp >= 32) ? R2 : R1;
             gt[gEb * 64 + pt] = exp2f(Gend - G);
-            gt[gRf * 64 + pt] = exp2f(G - Gm);
-            const float cf = exp2f(Gm - G);
-            gt[gCf * 64 + pt] = cf;
-            gt[gCfl * 64 + (x.dir ? 63 - pt : pt)] = cf;
+            gt[gRA * 64 + pt] = exp2f(G - Rh);
+            gt[gCA * 64 + pt] = exp2f(Rh - G);
+            gt[gRB * 64 + pt] = exp2f(G - Rm);
+            gt[gCB * 64 + pt] = exp2f(Rm - G);
+            if (pt == 0) gt[gScal * 64] = Gend;
         }
-        named_bar(kBarPrep);
+        named_bar(kBarPrep, kPrepThreads);
         if (pt == 0) mbar_arrive(&B.g_full[b]);
+        PROF_MARK(9);
 
         // ---- masks: P (rows of QK^T) and A (rows of KK^T, scan order)
         wait_bar(&B.d1_full, i & 1, x.abort_flag, p.err, 3);
         if (i >= 2) wait_bar(&B.p_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 4);
+        // A shares space with T1/T2 of chunk i-1: their products must be done
+        if (i >= 1) wait_bar(&B.wu_full, (i - 1) & 1, x.abort_flag, p.err, 6);
+        PROF_MARK(10);
         tc_fence_after();
         {
-            float xv[64];
-            tmem_ld64(x.tmem + tm_lane + kColD1, xv);
-            if (dbg) dbg_rows(p.debug + kDbgD1, pt, xv);
-            if (pw < 2) {
-                const int r = pt;                        // physical row of P
-                const int lr = x.dir ? 63 - r : r;
+            float xv[32];
+            tmem_ld32(x.tmem + tm_lane + kColD1 + 32 * hf, xv);
+            tmem_wait_ld();
+            if (dbg) dbg_half(p.debug + kDbgD1, qd * 32 + lane, hf, xv);
+            const int r = (qd & 1) * 32 + lane;            // physical token row
+            const int lr = DIR ? 63 - r : r;
+            const bool useB = lr >= 32 && col_h1;           // cross-half pairs
+            const float *cf = gt + (useB ? gCB : gCA) * 64 + 32 * hf;
+            const float *Gj = gt + gG * 64 + 32 * hf;
+            if (qd < 2) {
+                // P row r: keep j at or before r in scan order
                 if (fact) {
-                    const float rf = gt[gRf * 64 + r];
+                    const float rf = gt[(useB ? gRB : gRA) * 64 + r];
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        const int lj = x.dir ? 63 - j : j;
-                        xv[j] = (lj <= lr) ? rf * gt[gCf * 64 + j] * xv[j] : 0.f;
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = 32 * hf + e;
+                        const bool keep = DIR ? (j >= r) : (j <= r);
+                        xv[e] = keep ? rf * cf[e] * xv[e] : 0.f;
                     }
                 } else {
                     const float Gr = gt[gG * 64 + r];
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        const int lj = x.dir ? 63 - j : j;
-                        xv[j] = (lj <= lr) ? exp2f(Gr - gt[gG * 64 + j]) * xv[j] : 0.f;
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = 32 * hf + e;
+                        const bool keep = DIR ? (j >= r) : (j <= r);
+                        xv[e] = keep ? exp2f(Gr - Gj[e]) * xv[e] : 0.f;
                     }
                 }
-                store_row_bf16(x.sbase + kOffP + b * 8192, r, xv);
+                store_half_row_bf16(x.sbase + kOffP + b * 8192, r, hf, xv);
             } else {
-                const int r = pt - 64;
-                const int lr = x.dir ? 63 - r : r;
+                // A row r, written in scan order: row lr, columns lj
                 const float br = gt[gBet * 64 + r];
-                float *Arow = As + lr * kLDA;
-                if (fact) {
-                    const float rf = br * gt[gRf * 64 + r];
+                const float rf = br * gt[(useB ? gRB : gRA) * 64 + r];
+                const float Gr = gt[gG * 64 + r];
+                float4 *Arow = reinterpret_cast<float4 *>(As + lr * kLDA + (DIR ? 32 * (1 - hf) : 32 * hf));
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        float o4[4];
+                for (int m = 0; m < 8; ++m) {
+                    float o4[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int lj = 4 * m + u;
-                            const float xj = x.dir ? xv[63 - lj] : xv[lj];
-                            o4[u] = (lj < lr) ? rf * gt[gCfl * 64 + lj] * xj : 0.f;
-                        }
-                        *reinterpret_cast<float4 *>(Arow + 4 * m) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;   // physical column 32 hf + e
+                        const int lj = DIR ? 63 - (32 * hf + e) : 32 * hf + e;
+                        const float f = fact ? rf * cf[e] : br * exp2f(Gr - Gj[e]);
+                        o4[u] = (lj < lr) ? f * xv[e] : 0.f;
                     }
-                } else {
-                    const float Gr = gt[gG * 64 + r];
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        float o4[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int lj = 4 * m + u;
-                            const int j = x.dir ? 63 - lj : lj;
-                            const float xj = x.dir ? xv[63 - lj] : xv[lj];
-                            o4[u] = (lj < lr) ? br * exp2f(Gr - gt[gG * 64 + j]) * xj : 0.f;
-                        }
-                        *reinterpret_cast<float4 *>(Arow + 4 * m) = make_float4(o4[0], o4[1], o4[2], o4[3]);
-                    }
+                    Arow[m] = make_float4(o4[0], o4[1], o4[2], o4[3]);
                 }
             }
         }
         tc_fence_before();
         fence_proxy_async_smem();
-        if (named_bar_any(kBarPrep, *x.abort_flag)) return;
+        PROF_MARK(11);
+        if (named_bar_any(kBarPrep, kPrepThreads, *x.abort_flag)) return;
         if (pt == 0) mbar_arrive(&B.d1_empty);
 
-        // ---- gamma-scale Q in place (the unscaled Q is no longer needed)
-        {
-            const int r = pt >> 1, kb = pt & 1;
-            const float gr = gt[gGam * 64 + r];
-            const uint32_t rowbase = stage_addr(x, i) + kb * 16384;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint32_t addr = rowbase + sw128_off(r, 8 * q);
-                uint32_t w[4];
-                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[u]));
-                    w[u] = pack_bf16(f.x * gr, f.y * gr);
-                }
-                st_shared_v4(addr, w[0], w[1], w[2], w[3]);
-            }
-        }
-
         // ---- T = (I + A)^-1
-        solve_unit_lower(As, Ts, Yall, pt);
+        solve_diag_blocks(As, Ts, pt);
+        PROF_MARK(13);
+        solve_off_diag(As, Ts, pt);
+        PROF_MARK(17);
         if (dbg)
-            for (int e = pt; e < 64 * 64; e += 128) p.debug[kDbgT + e] = Ts[(e >> 6) * kLDA + (e & 63)];
+            for (int e = pt; e < 64 * 64; e += kPrepThreads) {
+                const int rr = e >> 6, cc = e & 63;
+                p.debug[kDbgT + e] = (cc <= rr) ? Ts[rr * kLDA + cc] : 0.f;
+            }
 
         // ---- T1 = T diag(b gamma), T2 = T diag(b), physical order, into A's space
         {
-            const int r = pt & 63;
-            const bool second = pt >= 64;
-            const int lr = x.dir ? 63 - r : r;
-            const float *Trow = Ts + lr * kLDA;
-            const float *scale = gt + (second ? gBet : gBG) * 64;
-            float xv[64];
+            const int second = pt >> 7, r = (pt >> 1) & 63, h2 = pt & 1;
+            const int lr = DIR ? 63 - r : r;
+            // scan-order columns of physical half h2
+            const float4 *Trow = reinterpret_cast<const float4 *>(Ts + lr * kLDA + (DIR ? 32 * (1 - h2) : 32 * h2));
+            const float *sc = gt + (second ? gBet : gBG) * 64 + 32 * h2;
+            float xv[32];
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float4 t4 = *reinterpret_cast<const float4 *>(Trow + 4 * m);   // scan cols 4m..4m+3
+            for (int m = 0; m < 8; ++m) {
+                const float4 t4 = Trow[m];
                 const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int lj = 4 * m + u;
-                    if (x.dir) xv[63 - lj] = tv[u];
-                    else xv[lj] = tv[u];
+                    const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;
+                    const int lj = DIR ? 63 - (32 * h2 + e) : 32 * h2 + e;
+                    xv[e] = (lj <= lr) ? tv[u] * sc[e] : 0.f;    // upper triangle: zero
                 }
             }
-#pragma unroll
-            for (int j = 0; j < 64; ++j) xv[j] *= scale[j];
-            store_row_bf16(x.sbase + (second ? kOffT2 : kOffT1), r, xv);
+            store_half_row_bf16(x.sbase + (second ? kOffT2 : kOffT1), r, h2, xv);
         }
         fence_proxy_async_smem();
-        if (named_bar_any(kBarPrep, *x.abort_flag)) return;
+        PROF_MARK(14);
+        if (named_bar_any(kBarPrep, kPrepThreads, *x.abort_flag)) return;
         if (pt == 0) mbar_arrive(&B.tp_full);
 
-        // ---- W (MN-major, row d = key index) to shared memory
-        wait_bar(&B.wu_full, i & 1, x.abort_flag, p.err, 5);
-        if (i >= 1) wait_bar(&B.wmn_empty, (i - 1) & 1, x.abort_flag, p.err, 6);
-        tc_fence_after();
-        {
-            float xv[64];
-            tmem_ld64(x.tmem + tm_lane + kColW, xv);
-            if (dbg) {
-                dbg_rows(p.debug + kDbgW, pt, xv);
-                float yv[64];
-                tmem_ld64(x.tmem + tm_lane + kColU0 + 64 * b, yv);
-                dbg_rows(p.debug + kDbgUt, pt, yv);
-            }
-            store_row_bf16(x.sbase + kOffW, pt, xv);
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        if (named_bar_any(kBarPrep, *x.abort_flag)) return;
-        if (pt == 0) mbar_arrive(&B.wmn_full);
     }
+    PROF_FLUSH();
 }
 
 // ------------------------------------------------------------------ chain warps
-__device__ void chain_role(const Ctx &x, const TcParams &p, int ct)
+// 8 warps (256 threads).  Thread (warp cw, lane) owns state row
+// d = 32 * (cw & 3) + lane, columns [32 * (cw >> 2), +32) of the slice.
+// Per chunk i, in this order (so that the serial-chain products of chunk i can
+// start while the output tile of chunk i-1 is written):
+//   W and gamma*Q of chunk i  ->  output tile of chunk i-1  ->  U of chunk i
+//   ->  state update of chunk i.
+template <int DIR>
+__device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int ct)
 {
     Bars &B = *x.bars;
-    const int warp = ct >> 5, lane = ct & 31;
-    const uint32_t tm_lane = (uint32_t)(warp * 32) << 16;
+    const int cw = ct >> 5, lane = ct & 31, cq = cw & 3, chf = cw >> 2;
+    const uint32_t tm_lane = (uint32_t)(cq * 32) << 16;
+    const int d = cq * 32 + lane;
+    const int r = cq * 16 + lane;   // M=64 accumulators: lanes 0-15 of quarter cq hold rows 16 cq ..
 
-    float h[kDVS];
+    float h[32];
     {
-        const float *s0 = (x.dir == 0 && p.state_in)
-                              ? p.state_in + ((size_t)x.bh * kDK + ct) * x.dv + x.slice * kDVS
+        const float *s0 = (DIR == 0 && p.state_in)
+                              ? p.state_in + ((size_t)x.bh * kDK + d) * x.dv + x.slice * kDVS + 32 * chf
                               : nullptr;
 #pragma unroll
-        for (int e = 0; e < kDVS; e += 4) {
+        for (int e = 0; e < 32; e += 4) {
             const float4 v4 = s0 ? *reinterpret_cast<const float4 *>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
             h[e] = v4.x; h[e + 1] = v4.y; h[e + 2] = v4.z; h[e + 3] = v4.w;
         }
-        store_row_bf16(x.sbase + kOffH, ct, h);
+        store_half_row_bf16(x.sbase + kOffH, d, chf, h);
     }
     fence_proxy_async_smem();
-    named_bar(kBarChain);
+    named_bar(kBarChain, kChainThreads);
     if (ct == 0) mbar_arrive(&B.h_full);
+    PROF_DECL(ct == 0);
+
+    // output tile of chunk j: O = (gamma Q) H_prev + P U, from TMEM to o
+    // (bidirectional: combined with the other direction's partial)
+    auto out_tile = [&](int j) -> bool {
+        const int bj = j & 1, c = chunk_of<DIR>(x, j);
+        wait_bar(&B.o_full[bj], (j >> 1) & 1, x.abort_flag, p.err, 10);
+        PROF_MARK(24);
+        tc_fence_after();
+        float xv[32];
+        tmem_ld32(x.tmem + tm_lane + kColO0 + 64 * bj + 32 * chf, xv);
+        tmem_wait_ld();
+        if (p.debug != nullptr && j == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+            dbg_half(p.debug + kDbgO, d, chf, xv);
+        const int t = c * kC + r;
+        const bool mine = lane < 16 && t < x.T;
+        __nv_bfloat16 *orow = p.o + ((size_t)x.bh * x.T + (mine ? t : 0)) * x.dv + x.slice * kDVS + 32 * chf;
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = pack_bf16(xv[2 * e], xv[2 * e + 1]);
+        auto store_own = [&]() {
+            if (mine)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        };
+        auto add_other = [&]() {
+            if (mine && !*x.abort_flag)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 o4 = __ldcg(reinterpret_cast<const uint4 *>(orow + 8 * q));
+                    const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
+                    uint32_t sw[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow[u]));
+                        sw[u] = pack_bf16(f.x + xv[8 * q + 2 * u], f.y + xv[8 * q + 2 * u + 1]);
+                    }
+                    *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+                }
+        };
+        // bounded wait (thread ct == 0) until the counter reaches `target`
+        auto wait_count = [&](int *cnt, int target) {
+            if (ct == 0) {
+                const unsigned long long t0 = globaltimer();
+                int seen = 0;
+                for (uint32_t it = 0; it < (1u << 30); ++it) {
+                    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(cnt) : "memory");
+                    if (seen >= target) break;
+                    if ((it & 255) == 255 && globaltimer() - t0 > kWaitLimitNs) break;
+                }
+                if (seen < target) {
+                    atomicOr(p.err, 32);
+                    *x.abort_flag = 1;
+                }
+            }
+        };
+        if (p.counters == nullptr) {
+            store_own();
+        } else {
+            int *cnt = p.counters + ((size_t)x.bh * x.NC + c) * p.n_slices + x.slice;
+            if (p.predict) {
+                // every CTA is resident: the direction that reaches chunk c
+                // first is known (forward for the first half of the chunks)
+                const int first = (2 * c < x.NC) ? 0 : 1;
+                if (DIR == first) {
+                    store_own();
+                    named_bar(kBarChain, kChainThreads);
+                    if (ct == 0) {
+                        __threadfence();
+                        atomicAdd(cnt, 1);
+                    }
+                } else {
+                    wait_count(cnt, 1);
+                    named_bar(kBarChain, kChainThreads);
+                    add_other();
+                }
+            } else {
+                // arrival order decided at run time: the first to arrive writes
+                // its partial, the second waits until it is written and adds
+                if (ct == 0) x.bars->s_old = atomicAdd(cnt, 1);
+                named_bar(kBarChain, kChainThreads);
+                if (x.bars->s_old == 0) {
+                    store_own();
+                    named_bar(kBarChain, kChainThreads);
+                    if (ct == 0) {
+                        __threadfence();
+                        atomicAdd(cnt, 1);
+                    }
+                } else {
+                    wait_count(cnt, 3);
+                    named_bar(kBarChain, kChainThreads);
+                    add_other();
+                }
+            }
+        }
+        tc_fence_before();
+        PROF_MARK(25);
+        if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return false;
+        if (ct == 0) mbar_arrive(&B.do_empty[bj]);
+        return true;
+    };
 
     for (int i = 0; i < x.NC; ++i) {
-        const int b = i & 1, c = chunk_of(x, i);
+        const int b = i & 1, c = chunk_of<DIR>(x, i);
         const float *gt = gates_buf(x, b);
         const bool dbg = p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
                          blockIdx.z == 0;
 
-        // ---- U and Ubar rows (M=64 layout: warp w, lanes 0-15 hold rows 16w..16w+15)
+        // ---- W (MN-major, row d = key index) and gamma-scaled Q of chunk i
         wait_bar(&B.g_full[b], (i >> 1) & 1, x.abort_flag, p.err, 7);
-        wait_bar(&B.chain_full, i & 1, x.abort_flag, p.err, 8);
+        wait_bar(&B.wu_full, i & 1, x.abort_flag, p.err, 5);
+        PROF_MARK(26);
         tc_fence_after();
         {
-            float xv[64];
-            tmem_ld64(x.tmem + tm_lane + kColU0 + 64 * b, xv);
-            if (dbg) dbg_rows(p.debug + kDbgU, ct, xv);
-            if (lane < 16) {
-                const int r = warp * 16 + lane;
-                store_row_bf16(x.sbase + kOffU, r, xv);
-                const float eb = gt[gEb * 64 + r];
+            float xv[32];
+            tmem_ld32(x.tmem + tm_lane + kColW + 32 * chf, xv);
+            tmem_wait_ld();
+            if (dbg) {
+                dbg_half(p.debug + kDbgW, d, chf, xv);
+                float yv[32];
+                tmem_ld32(x.tmem + tm_lane + kColU0 + 64 * b + 32 * chf, yv);
+                tmem_wait_ld();
+                dbg_half(p.debug + kDbgUt, d, chf, yv);
+            }
+            store_half_row_bf16(x.sbase + kOffW, d, chf, xv);
+        }
+        {
+            // gamma-scale Q in place (Q is no longer needed unscaled); bf16x2
+            // products: gamma is rounded to bf16 first, one more bf16 rounding
+            const int rq = ct >> 2, kb = (ct >> 1) & 1, part = ct & 1;
+            const __nv_bfloat162 g2 = __float2bfloat162_rn(gt[gGam * 64 + rq]);
+            const uint32_t rowbase = stage_addr(x, i) + kb * 16384;
+            uint32_t w[4][4];
 #pragma unroll
-                for (int e = 0; e < 64; ++e) xv[e] *= eb;
-                store_row_bf16(x.sbase + kOffUb, r, xv);
+            for (int q = 0; q < 4; ++q)
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(w[q][0]), "=r"(w[q][1]), "=r"(w[q][2]), "=r"(w[q][3])
+                             : "r"(rowbase + sw128_off(rq, 8 * (4 * part + q))));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    __nv_bfloat162 v = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&w[q][u]), g2);
+                    w[q][u] = *reinterpret_cast<uint32_t *>(&v);
+                }
+                st_shared_v4(rowbase + sw128_off(rq, 8 * (4 * part + q)), w[q][0], w[q][1], w[q][2], w[q][3]);
             }
         }
         tc_fence_before();
         fence_proxy_async_smem();
-        if (named_bar_any(kBarChain, *x.abort_flag)) return;
+        PROF_MARK(27);
+        if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return;
+        if (ct == 0) {
+            mbar_arrive(&B.wmn_full);
+            mbar_arrive(&B.dw_empty);
+        }
+
+        // ---- output tile of the previous chunk (overlaps this chunk's products)
+        if (i > 0 && !out_tile(i - 1)) return;
+
+        // ---- U and Ubar rows of chunk i
+        wait_bar(&B.chain_full, i & 1, x.abort_flag, p.err, 8);
+        PROF_MARK(20);
+        tc_fence_after();
+        {
+            float xv[32];
+            tmem_ld32(x.tmem + tm_lane + kColU0 + 64 * b + 32 * chf, xv);
+            tmem_wait_ld();
+            if (dbg) dbg_half(p.debug + kDbgU, d, chf, xv);
+            if (lane < 16) {
+                store_half_row_bf16(x.sbase + kOffU, r, chf, xv);
+                const float eb = gt[gEb * 64 + r];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) xv[e] *= eb;
+                store_half_row_bf16(x.sbase + kOffUb, r, chf, xv);
+                // bidirectional, second direction for this tile: pull the other
+                // direction's partial into L2 ahead of the output step
+                const int t = c * kC + r;
+                if (p.counters != nullptr && p.predict && t < x.T && DIR != ((2 * c < x.NC) ? 0 : 1))
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + ((size_t)x.bh * x.T + t) * x.dv + x.slice * kDVS + 32 * chf));
+            }
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        PROF_MARK(21);
+        if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return;
         if (ct == 0) {
             mbar_arrive(&B.u_full);
             mbar_arrive(&B.du_empty[b]);
@@ -729,99 +950,34 @@ __device__ void chain_role(const Ctx &x, const TcParams &p, int ct)
 
         // ---- state update (fp32 registers) and its bf16 copy
         wait_bar(&B.s_full, i & 1, x.abort_flag, p.err, 9);
+        PROF_MARK(22);
         tc_fence_after();
         {
-            float xv[64];
-            tmem_ld64(x.tmem + tm_lane + kColS, xv);
-            if (dbg) dbg_rows(p.debug + kDbgS, ct, xv);
+            float xv[32];
+            tmem_ld32(x.tmem + tm_lane + kColS + 32 * chf, xv);
+            tmem_wait_ld();
+            if (dbg) dbg_half(p.debug + kDbgS, d, chf, xv);
             const float ge = exp2f(gt[gScal * 64]);
 #pragma unroll
-            for (int e = 0; e < 64; ++e) h[e] = fmaf(ge, h[e], xv[e]);
-            store_row_bf16(x.sbase + kOffH, ct, h);
+            for (int e = 0; e < 32; ++e) h[e] = fmaf(ge, h[e], xv[e]);
+            store_half_row_bf16(x.sbase + kOffH, d, chf, h);
         }
         tc_fence_before();
         fence_proxy_async_smem();
-        if (named_bar_any(kBarChain, *x.abort_flag)) return;
+        PROF_MARK(23);
+        if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return;
         if (ct == 0) {
             mbar_arrive(&B.h_full);
             mbar_arrive(&B.g_empty[b]);
         }
-
-        // ---- output tile
-        wait_bar(&B.o_full[b], (i >> 1) & 1, x.abort_flag, p.err, 10);
-        tc_fence_after();
-        {
-            float xv[64];
-            tmem_ld64(x.tmem + tm_lane + kColO0 + 64 * b, xv);
-            if (dbg) dbg_rows(p.debug + kDbgO, ct, xv);
-            const int r = warp * 16 + lane;
-            const int t = c * kC + r;
-            const bool mine = lane < 16 && t < x.T;
-            __nv_bfloat16 *orow = p.o + ((size_t)x.bh * x.T + (mine ? t : 0)) * x.dv + x.slice * kDVS;
-            uint32_t w[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) w[e] = pack_bf16(xv[2 * e], xv[2 * e + 1]);
-            if (p.counters == nullptr) {
-                if (mine)
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-            } else {
-                int *cnt = p.counters + ((size_t)x.bh * x.NC + c) * p.n_slices + x.slice;
-                if (ct == 0) x.bars->s_old = atomicAdd(cnt, 1);
-                named_bar(kBarChain);
-                if (x.bars->s_old == 0) {
-                    if (mine)
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-                    named_bar(kBarChain);
-                    if (ct == 0) {
-                        __threadfence();
-                        atomicAdd(cnt, 1);
-                    }
-                } else {
-                    if (ct == 0) {
-                        const unsigned long long t0 = globaltimer();
-                        int seen = 0;
-                        for (uint32_t it = 0; it < (1u << 30); ++it) {
-                            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(cnt) : "memory");
-                            if (seen >= 3) break;
-                            if ((it & 255) == 255 && globaltimer() - t0 > kWaitLimitNs) break;
-                        }
-                        if (seen < 3) {
-                            atomicOr(p.err, 32);
-                            *x.abort_flag = 1;
-                        }
-                        __threadfence();
-                    }
-                    named_bar(kBarChain);
-                    if (mine && !*x.abort_flag) {
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const uint4 o4 = __ldcg(reinterpret_cast<const uint4 *>(orow + 8 * q));
-                            const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
-                            uint32_t sw[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow[u]));
-                                sw[u] = pack_bf16(f.x + xv[8 * q + 2 * u], f.y + xv[8 * q + 2 * u + 1]);
-                            }
-                            *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-                        }
-                    }
-                }
-            }
-        }
-        tc_fence_before();
-        if (named_bar_any(kBarChain, *x.abort_flag)) return;
-        if (ct == 0) mbar_arrive(&B.do_empty[b]);
     }
+    if (x.NC > 0 && !out_tile(x.NC - 1)) return;
+    PROF_FLUSH();
 
     if (p.state_out) {
-        float *so = p.state_out + (((size_t)x.dir * p.BH + x.bh) * kDK + ct) * x.dv + x.slice * kDVS;
+        float *so = p.state_out + (((size_t)DIR * p.BH + x.bh) * kDK + d) * x.dv + x.slice * kDVS + 32 * chf;
 #pragma unroll
-        for (int e = 0; e < kDVS; e += 4)
+        for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4 *>(so + e) = make_float4(h[e], h[e + 1], h[e + 2], h[e + 3]);
     }
 }
@@ -830,9 +986,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const TcParams p)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // Align by offsetting the shared array itself (not through an integer
+    // cast), so that every access below stays a shared-memory access.
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     Ctx x;
@@ -864,23 +1021,43 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     float *Ts = reinterpret_cast<float *>(smem + kOffT);
     for (int i = tid; i < 64 * kLDA; i += kThreads) Ts[i] = 0.f;
+    if (tid < 32) reinterpret_cast<long long *>(smem + kOffProf)[tid] = 0;
+#ifdef GDN_PROFILE
+    const unsigned long long prof_start = globaltimer();
+#endif
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     x.tmem = B.tmem_slot;
 
-    if (warp < 4) {
-        chain_role(x, p, tid);
-    } else if (warp < 8) {
-        prep_role(x, p, tid - 128);
-    } else if (warp == 8) {
-        if (lane == 0) tma_role(x, &tmQ, &tmK, &tmV, p);
+    if (warp < 8) {
+        if (x.dir) chain_role<1>(x, p, tid);
+        else chain_role<0>(x, p, tid);
+    } else if (warp < 16) {
+        if (x.dir) prep_role<1>(x, p, tid - kChainThreads);
+        else prep_role<0>(x, p, tid - kChainThreads);
+    } else if (warp == 16) {
+        if (lane == 0) {
+            if (x.dir) tma_role<1>(x, &tmQ, &tmK, &tmV, p);
+            else tma_role<0>(x, &tmQ, &tmK, &tmV, p);
+        }
+    } else if (warp == 17) {
+        if (lane == 0) mma_prep_role(x, p);
     } else {
-        if (lane == 0) mma_role(x, p);
+        if (lane == 0) mma_chain_role(x, p);
     }
 
     tc_fence_before();
     __syncthreads();
+#ifdef GDN_PROFILE
+    if (p.prof && tid < 32 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+        p.prof[tid] += reinterpret_cast<long long *>(smem + kOffProf)[tid];
+    if (p.prof && tid == 0) {
+        const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+        p.prof[32 + 2 * cta] = (long long)prof_start;
+        p.prof[33 + 2 * cta] = (long long)globaltimer();
+    }
+#endif
     if (warp == 0) tmem_dealloc(x.tmem, kTmemCols);
 }
 
@@ -920,9 +1097,22 @@ bool make_map(CUtensorMap *m, const void *base, int inner, int T, int BH)
     return r == CUDA_SUCCESS;
 }
 
+// Whether every CTA of the grid is resident at once (one CTA per SM, as the
+// shared-memory footprint forces), so that each bidirectional output tile's
+// first writer can be fixed in advance.
+cudaError_t all_resident(int n_ctas, int *out)
+{
+    int dev = 0, sms = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    *out = (err == cudaSuccess && n_ctas <= sms) ? 1 : 0;
+    return err;
+}
+
 }  // namespace
 
 float *g_debug_dump = nullptr;
+long long *g_prof_buf = nullptr;
 
 bool chunk_tc_supported(const FwdArgs &a)
 {
@@ -945,7 +1135,10 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
     p.n_slices = a.dv / kDVS;
     p.counters = nullptr;
     p.debug = g_debug_dump;
+    p.prof = g_prof_buf;
     cudaError_t err = device_error_word(&p.err);
+    if (err != cudaSuccess) return err;
+    err = all_resident(BH * (a.bidi ? 2 : 1) * p.n_slices, &p.predict);
     if (err != cudaSuccess) return err;
 
     err = cudaFuncSetAttribute(gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1009,7 +1202,10 @@ cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream)
     p.n_slices = a.dv / kDVS;
     p.counters = nullptr;
     p.debug = nullptr;
+    p.prof = nullptr;
     cudaError_t err = device_error_word(&p.err);
+    if (err != cudaSuccess) return err;
+    err = all_resident(BH * (a.bidi ? 2 : 1) * p.n_slices, &p.predict);
     if (err != cudaSuccess) return err;
     err = cudaFuncSetAttribute(gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kSmemAlloc);
@@ -1051,3 +1247,7 @@ cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream)
 // 53248 floats, the next chunkwise launches dump the first chunk's
 // intermediates of CTA (0,0,0) there.  NULL turns it off.
 extern "C" void gdn_debug_dump(float *device_buffer) { gdn::g_debug_dump = device_buffer; }
+
+// Test hook for profiling builds: per-phase cycle counters of CTA (0,0,0),
+// 32 long longs (zeroed by the caller).  Ignored unless built with GDN_PROFILE.
+extern "C" void gdn_debug_profile(long long *device_buffer) { gdn::g_prof_buf = device_buffer; }
