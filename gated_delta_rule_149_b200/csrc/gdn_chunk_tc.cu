@@ -71,7 +71,7 @@ constexpr int kThreads = 608;    // 8 chain + 8 prep + TMA + 2 MMA-issue warps
 constexpr int kChainThreads = 256, kPrepThreads = 256;
 constexpr int kNS = 3;           // input stages
 constexpr int kLDA = 68;         // fp32 row stride of the solve buffers
-constexpr int kBarPrep = 1, kBarChain = 2;   // named barriers of the prep and chain groups
+constexpr int kBarPrep = 1, kBarChain = 2, kBarGates = 3;   // named barriers (prep, chain, gate warps)
 
 // TMEM columns (fp32 accumulators)
 constexpr uint32_t kColD1 = 0;     // [Q;K] K^T   (M=128)
@@ -93,9 +93,10 @@ constexpr uint32_t kOffA = kOffH + 16384;              // fp32 [64][68], scan or
 constexpr uint32_t kOffT1 = kOffA;                     // T1, T2 (bf16) reuse A after the solve
 constexpr uint32_t kOffT2 = kOffA + 8192;
 constexpr uint32_t kOffT = kOffA + 64 * kLDA * 4;      // fp32 [64][68], scan order
-constexpr uint32_t kGateFloats = 10 * 64;              // per buffer, see GateIdx
-constexpr uint32_t kOffGates = kOffT + 64 * kLDA * 4;  // 2 buffers
-constexpr uint32_t kOffBar = kOffGates + 2 * kGateFloats * 4;
+constexpr int kNG = 3;                                 // gate buffers (prep runs ahead)
+constexpr uint32_t kGateFloats = 9 * 64;               // per buffer, see GateIdx
+constexpr uint32_t kOffGates = kOffT + 64 * kLDA * 4;
+constexpr uint32_t kOffBar = kOffGates + kNG * kGateFloats * 4;
 constexpr uint32_t kOffProf = kOffBar + 512;            // 32 x 8 B (profiling builds)
 constexpr uint32_t kSmemBytes = kOffProf + 256;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;     // alignment slack
@@ -104,8 +105,8 @@ static_assert(kOffA % 1024 == 0 && kOffT2 % 1024 == 0 && kOffP % 1024 == 0, "til
 
 // gate arrays (64 floats each, physical token order unless noted)
 // G (log2 cumulative decay), gamma = 2^G, beta, beta*gamma, 2^(G_end - G), row/column
-// factors of the decay products (A: same half of the chunk, B: across halves), scalars
-enum GateIdx { gG = 0, gGam, gBet, gBG, gEb, gRA, gRB, gCA, gCB, gScal };
+// factors of the decay products (A: same half of the chunk, B: across halves)
+enum GateIdx { gG = 0, gGam, gBet, gBG, gEb, gRA, gRB, gCA, gCB };
 
 constexpr uint32_t kIdM1 = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdW = idesc_bf16(128, 64, true, false);
@@ -170,7 +171,8 @@ struct Bars {
     uint64_t stage_full[kNS], stage_empty[kNS];
     uint64_t d1_full, d1_empty, tp_full, wu_full, wmn_full, dw_empty;
     uint64_t chain_full, u_full, s_full, h_full, drain, drain2;
-    uint64_t o_full[2], do_empty[2], du_empty[2], p_empty[2], g_full[2], g_empty[2];
+    uint64_t o_full[2], do_empty[2], du_empty[2], p_empty[2], g_full[kNG], g_empty[kNG];
+    float gscal[kNG][2];   // per gate buffer: G_end, factorised (1) or not (0)
     uint32_t tmem_slot;
     int abort_flag;
     int s_old;
@@ -389,7 +391,7 @@ struct Ctx {
 __device__ __forceinline__ uint32_t stage_addr(const Ctx &x, int i) { return x.sbase + kOffStage + (uint32_t)(i % kNS) * kStageBytes; }
 template <int DIR>
 __device__ __forceinline__ int chunk_of(const Ctx &x, int i) { return DIR ? (x.NC - 1 - i) : i; }
-__device__ __forceinline__ float *gates_buf(const Ctx &x, int b) { return reinterpret_cast<float *>(x.smem + kOffGates) + b * kGateFloats; }
+__device__ __forceinline__ float *gates_buf(const Ctx &x, int g) { return reinterpret_cast<float *>(x.smem + kOffGates) + g * kGateFloats; }
 
 // ------------------------------------------------------------------ TMA warp
 template <int DIR>
@@ -437,13 +439,12 @@ __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
     const uint32_t tm = x.tmem;
     const uint32_t sT1 = x.sbase + kOffT1, sT2 = x.sbase + kOffT2;
     PROF_DECL(true);
-    for (int i = 0; i < x.NC; ++i) {
-        const int b = i & 1;
-        const uint32_t sQK = stage_addr(x, i), sV = sQK + 32768;
-        PROF_MARK(6);
-        if (!wait_bar(&B.stage_full[i % kNS], (i / kNS) & 1, x.abort_flag, p.err, 11)) break;
-        if (i > 0 && !wait_bar(&B.d1_empty, (i - 1) & 1, x.abort_flag, p.err, 12)) break;
+    // [Q;K] K^T of chunk j (needs its stage loaded and D1 read out for chunk j-1)
+    auto issue_m1 = [&](int j) -> bool {
+        if (!wait_bar(&B.stage_full[j % kNS], (j / kNS) & 1, x.abort_flag, p.err, 11)) return false;
+        if (j > 0 && !wait_bar(&B.d1_empty, (j - 1) & 1, x.abort_flag, p.err, 12)) return false;
         PROF_MARK(2);
+        const uint32_t sQK = stage_addr(x, j);
         tc_fence_after();
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
@@ -453,10 +454,19 @@ __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
                          sw128_desc(sQK + kb * 16384 + 8192 + ks * 32, 16, 1024), kIdM1, (kb | ks) != 0);
         mma_commit(&B.d1_full);
         PROF_MARK(6);
+        return true;
+    };
+    bool ok = issue_m1(0);
+    // chunk i: issue the next chunk's [Q;K] K^T first (its inputs are usually
+    // ready long before this chunk's T1/T2), then W^T = K^T T1^T, U~ = T2 V
+    for (int i = 0; ok && i < x.NC; ++i) {
+        const int b = i & 1;
+        if (i + 1 < x.NC && !(ok = issue_m1(i + 1))) break;
         if (!wait_bar(&B.tp_full, i & 1, x.abort_flag, p.err, 13)) break;
         if (i >= 2 && !wait_bar(&B.du_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 14)) break;
         if (i >= 1 && !wait_bar(&B.dw_empty, (i - 1) & 1, x.abort_flag, p.err, 19)) break;
         PROF_MARK(2);
+        const uint32_t sQK = stage_addr(x, i), sV = sQK + 32768;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
@@ -467,8 +477,8 @@ __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
             mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sT2 + ks * 32, 16, 1024),
                      sw128_desc(sV + ks * 2048, 8192, 1024), kIdUt, ks != 0);
         mma_commit(&B.wu_full);
+        PROF_MARK(6);
     }
-    PROF_MARK(5);
     PROF_FLUSH();
     // every issued MMA completes before the CTA releases its TMEM
     mma_commit(&B.drain);
@@ -544,58 +554,49 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
     // the logical (scan-order) half that this warp's 32 physical columns fall in
     const bool col_h1 = DIR ? (hf == 1) : (hf == 0);
 
-    // raw gates of the next chunk, fetched one chunk ahead (thread pt < 64
-    // handles scan position pt)
+    // Gates are computed one chunk ahead by prep warps 2-3 (gate thread
+    // gpt = pt - 64 handles scan position gpt), on their own 64-thread
+    // barrier, while warps 0-1 run the diagonal blocks of the previous solve.
+    const bool gate_thr = pt >= 64 && pt < 128;
+    const int gpt = pt - 64;
     float ra = 1.f, rb = 0.f;
-    auto load_raw = [&](int i) {
+    auto load_raw = [&](int j) {
         ra = 1.f;
         rb = 0.f;
-        if (pt < 64 && i < x.NC) {
-            const int pp = DIR ? (63 - pt) : pt;
-            const int t = chunk_of<DIR>(x, i) * kC + pp;
+        if (gate_thr && j < x.NC) {
+            const int pp = DIR ? (63 - gpt) : gpt;
+            const int t = chunk_of<DIR>(x, j) * kC + pp;
             if (t < x.T) {
                 ra = __ldg(decay_h + t);
                 rb = __ldg(beta_h + t);
             }
         }
     };
-    load_raw(0);
-    PROF_DECL(pt == 0);
-
-    for (int i = 0; i < x.NC; ++i) {
-        const int b = i & 1;
-        float *gt = gates_buf(x, b);
-        const bool dbg = p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
-                         blockIdx.z == 0;
-        PROF_MARK(16);
-
-        // ---- gates (log2 domain) for chunk i
-        if (i >= 2) wait_bar(&B.g_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 2);
-        PROF_MARK(8);
-        float gsum = 0.f;
+    // gates (log2 domain) of chunk j into buffer j & 1; gate threads only
+    auto compute_gates = [&](int j) {
+        const int gj = j % kNG;
+        float *gt = gates_buf(x, gj);
+        if (j >= kNG) wait_bar(&B.g_empty[gj], ((j / kNG) + 1) & 1, x.abort_flag, p.err, 2);
+        float v = fmaxf(log2f(ra), -120.f);   // decay below 2^-120 acts as 2^-120
         const float bcur = rb;
-        if (pt < 64) {
-            float v = fmaxf(log2f(ra), -120.f);   // decay below 2^-120 acts as 2^-120
+        load_raw(j + 1);
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, v, off);
-                if (lane >= off) v += y;
-            }
-            if (pt == 31) x.bars->s_wsum = v;
-            gsum = v;
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += y;
         }
-        load_raw(i + 1);
-        if (named_bar_any(kBarPrep, kPrepThreads, *x.abort_flag)) return;
-        if (pt < 64) {
-            const float G = (pt >= 32) ? gsum + x.bars->s_wsum : gsum;
-            const int pp = DIR ? (63 - pt) : pt;
+        if (gpt == 31) x.bars->s_wsum = v;
+        named_bar(kBarGates, 64);
+        {
+            const float G = (gpt >= 32) ? v + x.bars->s_wsum : v;
+            const int pp = DIR ? (63 - gpt) : gpt;
             gt[gG * 64 + pp] = G;
             const float gam = exp2f(G);
             gt[gGam * 64 + pp] = gam;
             gt[gBet * 64 + pp] = bcur;
             gt[gBG * 64 + pp] = bcur * gam;
         }
-        named_bar(kBarPrep, kPrepThreads);
+        named_bar(kBarGates, 64);
         // references: scan positions 15 (first half), 47 (second half), 31 (boundary)
         const float R1 = gt[gG * 64 + (DIR ? 48 : 15)];
         const float R2 = gt[gG * 64 + (DIR ? 16 : 47)];
@@ -606,20 +607,35 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
         // factorised decay products are exact while every factor is a normal float
         const bool fact = (G0 - R1) <= 120.f && (R1 - Rm) <= 120.f && (G32 - R2) <= 120.f &&
                           (R2 - Gend) <= 120.f;
-        if (pt < 64) {
-            const float G = gt[gG * 64 + pt];
-            const int lp = DIR ? 63 - pt : pt;
+        {
+            const float G = gt[gG * 64 + gpt];
+            const int lp = DIR ? 63 - gpt : gpt;
             const float Rh = (lp >= 32) ? R2 : R1;
-            gt[gEb * 64 + pt] = exp2f(Gend - G);
-            gt[gRA * 64 + pt] = exp2f(G - Rh);
-            gt[gCA * 64 + pt] = exp2f(Rh - G);
-            gt[gRB * 64 + pt] = exp2f(G - Rm);
-            gt[gCB * 64 + pt] = exp2f(Rm - G);
-            if (pt == 0) gt[gScal * 64] = Gend;
+            gt[gEb * 64 + gpt] = exp2f(Gend - G);
+            gt[gRA * 64 + gpt] = exp2f(G - Rh);
+            gt[gCA * 64 + gpt] = exp2f(Rh - G);
+            gt[gRB * 64 + gpt] = exp2f(G - Rm);
+            gt[gCB * 64 + gpt] = exp2f(Rm - G);
+            if (gpt == 0) {
+                x.bars->gscal[gj][0] = Gend;
+                x.bars->gscal[gj][1] = fact ? 1.f : 0.f;
+            }
         }
-        named_bar(kBarPrep, kPrepThreads);
-        if (pt == 0) mbar_arrive(&B.g_full[b]);
-        PROF_MARK(9);
+        named_bar(kBarGates, 64);
+        if (gpt == 0) mbar_arrive(&B.g_full[gj]);
+    };
+    load_raw(0);
+    if (gate_thr) compute_gates(0);
+    named_bar(kBarPrep, kPrepThreads);
+    PROF_DECL(pt == 0);
+
+    for (int i = 0; i < x.NC; ++i) {
+        const int b = i & 1;
+        float *gt = gates_buf(x, i % kNG);
+        const bool dbg = p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
+                         blockIdx.z == 0;
+        const bool fact = x.bars->gscal[i % kNG][1] != 0.f;
+        PROF_MARK(16);
 
         // ---- masks: P (rows of QK^T) and A (rows of KK^T, scan order)
         wait_bar(&B.d1_full, i & 1, x.abort_flag, p.err, 3);
@@ -684,7 +700,8 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
         if (named_bar_any(kBarPrep, kPrepThreads, *x.abort_flag)) return;
         if (pt == 0) mbar_arrive(&B.d1_empty);
 
-        // ---- T = (I + A)^-1
+        // ---- T = (I + A)^-1 ; meanwhile warps 2-3 prepare the next chunk's gates
+        if (gate_thr && i + 1 < x.NC) compute_gates(i + 1);
         solve_diag_blocks(As, Ts, pt);
         PROF_MARK(13);
         solve_off_diag(As, Ts, pt);
@@ -860,13 +877,13 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
     };
 
     for (int i = 0; i < x.NC; ++i) {
-        const int b = i & 1, c = chunk_of<DIR>(x, i);
-        const float *gt = gates_buf(x, b);
+        const int b = i & 1, c = chunk_of<DIR>(x, i), gi = i % kNG;
+        const float *gt = gates_buf(x, gi);
         const bool dbg = p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
                          blockIdx.z == 0;
 
         // ---- W (MN-major, row d = key index) and gamma-scaled Q of chunk i
-        wait_bar(&B.g_full[b], (i >> 1) & 1, x.abort_flag, p.err, 7);
+        wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 7);
         wait_bar(&B.wu_full, i & 1, x.abort_flag, p.err, 5);
         PROF_MARK(26);
         tc_fence_after();
@@ -957,7 +974,7 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
             tmem_ld32(x.tmem + tm_lane + kColS + 32 * chf, xv);
             tmem_wait_ld();
             if (dbg) dbg_half(p.debug + kDbgS, d, chf, xv);
-            const float ge = exp2f(gt[gScal * 64]);
+            const float ge = exp2f(x.bars->gscal[gi][0]);
 #pragma unroll
             for (int e = 0; e < 32; ++e) h[e] = fmaf(ge, h[e], xv[e]);
             store_half_row_bf16(x.sbase + kOffH, d, chf, h);
@@ -968,7 +985,7 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
         if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return;
         if (ct == 0) {
             mbar_arrive(&B.h_full);
-            mbar_arrive(&B.g_empty[b]);
+            mbar_arrive(&B.g_empty[gi]);
         }
     }
     if (x.NC > 0 && !out_tile(x.NC - 1)) return;
@@ -1007,7 +1024,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
     if (tid == 0) {
         uint64_t *all = reinterpret_cast<uint64_t *>(&B);
-        const int nbar = (int)(offsetof(Bars, tmem_slot) / sizeof(uint64_t));
+        const int nbar = (int)(offsetof(Bars, gscal) / sizeof(uint64_t));
         for (int k = 0; k < nbar; ++k) mbar_init(&all[k], 1);
         B.abort_flag = 0;
         fence_mbar_init();
