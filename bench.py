@@ -183,35 +183,43 @@ def max_over_ranks(x, world):
 # CPU oracle baseline (a bounded sample of the workload)
 # --------------------------------------------------------------------------
 
-def oracle_sample_throughput(wl, target_s=15.0):
-    """Times the fp64 oracle on whole heads of the workload truncated to a
-    token prefix sized for ~target_s seconds on the host cores."""
-    import numpy as np
+def oracle_sample_throughput(wl, inp=None, target_s=15.0):
+    """Times the fp64 oracle on a bounded sample of the workload's own inputs:
+    whole heads (both scan directions for bidi) truncated to a token prefix,
+    sized for about target_s seconds of wall time on the host cores."""
+    import math
     import oracle
-    from gated_delta_rule_149_b200.inputs import Workload, make_inputs
+    from gated_delta_rule_149_b200.inputs import make_inputs
+    if inp is None:
+        inp = make_inputs(wl)
     nproc = os.cpu_count() or 1
     ndir = 2 if wl.bidi else 1
-    n_heads = max(1, min(wl.B * wl.H, max(1, nproc // ndir)))
-    threads = min(nproc, n_heads * ndir)
+    BH = wl.B * wl.H
+    flat = lambda t: t.reshape(BH, *t.shape[2:])
 
-    def run(T):
-        sub = Workload(wl.name + "_sample", B=1, H=n_heads, T=T, dk=wl.dk, dv=wl.dv,
-                       dtype=wl.dtype, bidi=wl.bidi, decay_shift=wl.decay_shift, seed=wl.seed)
-        inp = make_inputs(sub)
-        args = [inp.q.double().numpy(), inp.k.double().numpy(), inp.v.double().numpy(),
-                inp.beta.double().numpy(), inp.decay.double().numpy()]
+    def run(n_heads, T):
+        sl = lambda t: flat(t)[:n_heads, :T].double().numpy()[None]
+        args = [sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.beta), sl(inp.decay)]
+        s0 = None if inp.state0 is None else flat(inp.state0)[:n_heads].double().numpy()[None]
         t0 = time.perf_counter()
-        oracle.gdn_forward(*args, bidi=wl.bidi, n_threads=threads)
+        oracle.gdn_forward(*args, state_in=s0, bidi=wl.bidi, n_threads=nproc)
         return time.perf_counter() - t0
 
-    t_small = run(256)
-    per_tok = t_small / 256.0
-    T = int(max(512, min(wl.T, target_s / max(per_tok, 1e-9))))
-    el = run(T)
+    per_wave = max(1, nproc // ndir)            # heads whose scans fill the cores once
+    n_heads = min(BH, per_wave)
+    T_cal = min(wl.T, 2048)
+    per_tok = run(n_heads, T_cal) / T_cal       # seconds per token for one wave
+    T = int(min(wl.T, max(256, target_s / per_tok)))
+    if T == wl.T:                               # whole heads are cheap: add waves
+        waves = max(1, int(target_s / (per_tok * T)))
+        n_heads = min(BH, per_wave * waves)
+    el = run(n_heads, T)
     value = n_heads * T / el
+    threads = min(nproc, n_heads * ndir)
     return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n_heads} heads x first {T} tokens of {wl.name} "
-                      f"({'both directions' if wl.bidi else 'causal'}), fp64, {el:.1f} s wall",
+            "sample": f"{n_heads} of {BH} heads x first {T} of {wl.T} tokens of {wl.name} "
+                      f"({'both scan directions' if wl.bidi else 'causal'}), fp64, "
+                      f"{el:.1f} s wall on {threads} threads",
             "elapsed_s": el, "cpu": _cpu_model()}
 
 
@@ -230,9 +238,11 @@ def run_reference(args, world, rank):
     wl = WORKLOADS[args.workload]
     if rank != 0:
         return 0
+    from gated_delta_rule_149_b200.inputs import make_inputs
+    inp = make_inputs(wl)
     vals = []
     for i in range(args.warmup + args.steps):
-        r = oracle_sample_throughput(wl, target_s=args.ref_seconds)
+        r = oracle_sample_throughput(wl, inp, target_s=args.ref_seconds)
         if i >= args.warmup:
             vals.append(r)
     value = statistics.median(v["value"] for v in vals)
@@ -364,7 +374,7 @@ def run_gpu(args, world, rank, local):
             "roofline": roofline,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample_throughput(wl, target_s=args.ref_seconds)
+        line["cpu_baseline"] = oracle_sample_throughput(wl, inp, target_s=args.ref_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -380,10 +390,13 @@ def main():
     ap.add_argument("--recurrent", action="store_true",
                     help="time the token-by-token SIMT kernel instead of the chunkwise one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="seconds of CPU work per oracle sample (default 15; 8 for --impl reference)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.ref_seconds is None:
+        args.ref_seconds = 8.0 if args.impl == "reference" else 15.0
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
