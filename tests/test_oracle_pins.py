@@ -285,3 +285,18 @@ def test_threads_do_not_change_bits(oracle_mod):
     o1, s1 = oracle_mod.gdn_forward(q, k, v, b, a, bidi=True, n_threads=1)
     o8, s8 = oracle_mod.gdn_forward(q, k, v, b, a, bidi=True, n_threads=8)
     assert np.array_equal(o1, o8) and np.array_equal(s1, s8)
+
+
+def test_oracle_regression_record(oracle_mod):
+    """The oracle still reproduces its committed tiny record (tests/golden)."""
+    import json
+    import os
+    rec = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "oracle_tiny.json")))
+    inp = {n: np.array(x) for n, x in rec["inputs"].items()}
+    args = [inp[n] for n in ("q", "k", "v", "beta", "decay")]
+    o, s = oracle_mod.gdn_forward(*args, state_in=inp["state0"])
+    np.testing.assert_allclose(o, np.array(rec["causal"]["o"]), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(s, np.array(rec["causal"]["state"]), rtol=1e-14, atol=1e-15)
+    o, s = oracle_mod.gdn_forward(*args, state_in=inp["state0"], bidi=True)
+    np.testing.assert_allclose(o, np.array(rec["bidi"]["o"]), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(s, np.array(rec["bidi"]["state"]), rtol=1e-14, atol=1e-15)
