@@ -161,6 +161,13 @@ struct TcParams {
     } while (0)
 #endif
 
+// First-chunk intermediates can be dumped for debugging in builds with
+// GDN_DEBUG_DUMP; production builds compile the dump code out.
+#ifdef GDN_DEBUG_DUMP
+constexpr bool kDbgOn = true;
+#else
+constexpr bool kDbgOn = false;
+#endif
 // Debug dump layout (floats): 6 TMEM snapshots of 128 lanes x 64 columns
 // (D1, W^T, U~, U, O, D_S) then the 64 x 64 solve result in scan order.
 constexpr int kDbgD1 = 0, kDbgW = 8192, kDbgUt = 16384, kDbgU = 24576, kDbgO = 32768,
@@ -632,7 +639,7 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
     for (int i = 0; i < x.NC; ++i) {
         const int b = i & 1;
         float *gt = gates_buf(x, i % kNG);
-        const bool dbg = p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
+        const bool dbg = kDbgOn && p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
                          blockIdx.z == 0;
         const bool fact = x.bars->gscal[i % kNG][1] != 0.f;
         PROF_MARK(16);
@@ -664,7 +671,7 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
                         const bool keep = DIR ? (j >= r) : (j <= r);
                         xv[e] = keep ? rf * cf[e] * xv[e] : 0.f;
                     }
-                } else {
+                } else {   // rare: a half-chunk decays by more than 2^-240
                     const float Gr = gt[gG * 64 + r];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -680,17 +687,30 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
                 const float rf = br * gt[(useB ? gRB : gRA) * 64 + r];
                 const float Gr = gt[gG * 64 + r];
                 float4 *Arow = reinterpret_cast<float4 *>(As + lr * kLDA + (DIR ? 32 * (1 - hf) : 32 * hf));
+                if (fact) {
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    float o4[4];
+                    for (int m = 0; m < 8; ++m) {
+                        float o4[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;   // physical column 32 hf + e
-                        const int lj = DIR ? 63 - (32 * hf + e) : 32 * hf + e;
-                        const float f = fact ? rf * cf[e] : br * exp2f(Gr - Gj[e]);
-                        o4[u] = (lj < lr) ? f * xv[e] : 0.f;
+                        for (int u = 0; u < 4; ++u) {
+                            const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;   // physical column 32 hf + e
+                            const int lj = DIR ? 63 - (32 * hf + e) : 32 * hf + e;
+                            o4[u] = (lj < lr) ? rf * cf[e] * xv[e] : 0.f;
+                        }
+                        Arow[m] = make_float4(o4[0], o4[1], o4[2], o4[3]);
                     }
-                    Arow[m] = make_float4(o4[0], o4[1], o4[2], o4[3]);
+                } else {   // rare: a half-chunk decays by more than 2^-240
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        float o4[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;
+                            const int lj = DIR ? 63 - (32 * hf + e) : 32 * hf + e;
+                            o4[u] = (lj < lr) ? br * exp2f(Gr - Gj[e]) * xv[e] : 0.f;
+                        }
+                        Arow[m] = make_float4(o4[0], o4[1], o4[2], o4[3]);
+                    }
                 }
             }
         }
@@ -785,7 +805,7 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
         float xv[32];
         tmem_ld32(x.tmem + tm_lane + kColO0 + 64 * bj + 32 * chf, xv);
         tmem_wait_ld();
-        if (p.debug != nullptr && j == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+        if (kDbgOn && p.debug != nullptr && j == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
             dbg_half(p.debug + kDbgO, d, chf, xv);
         const int t = c * kC + r;
         const bool mine = lane < 16 && t < x.T;
@@ -879,7 +899,7 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
     for (int i = 0; i < x.NC; ++i) {
         const int b = i & 1, c = chunk_of<DIR>(x, i), gi = i % kNG;
         const float *gt = gates_buf(x, gi);
-        const bool dbg = p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
+        const bool dbg = kDbgOn && p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
                          blockIdx.z == 0;
 
         // ---- W (MN-major, row d = key index) and gamma-scaled Q of chunk i
