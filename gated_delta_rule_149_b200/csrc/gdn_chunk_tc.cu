@@ -197,10 +197,9 @@ __device__ __forceinline__ unsigned long long globaltimer()
 // Bounded wait on an mbarrier phase; on timeout records the error and raises
 // the CTA's abort flag (callers then reach their group's next barrier and
 // leave together).
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                         int *err, int code)
+__device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int *err, int code)
 {
-    if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t it = 0; it < (1u << 30); ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -210,6 +209,15 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     atomicOr(err, code);
     *abort_flag = 1;
     return false;
+}
+
+// The first try covers almost every wait; the loop with its timer and error
+// path is kept out of line so that it does not crowd the instruction cache.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         int *err, int code)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, abort_flag, err, code);
 }
 
 __device__ __forceinline__ void named_bar(int id, int count)
@@ -463,12 +471,14 @@ __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
         PROF_MARK(6);
         return true;
     };
-    bool ok = issue_m1(0);
-    // chunk i: issue the next chunk's [Q;K] K^T first (its inputs are usually
-    // ready long before this chunk's T1/T2), then W^T = K^T T1^T, U~ = T2 V
-    for (int i = 0; ok && i < x.NC; ++i) {
-        const int b = i & 1;
-        if (i + 1 < x.NC && !(ok = issue_m1(i + 1))) break;
+    // step j: [Q;K] K^T of chunk j first (its inputs are usually ready long
+    // before the T1/T2 of chunk j - 1), then W^T = K^T T1^T, U~ = T2 V of
+    // chunk i = j - 1
+#pragma unroll 1
+    for (int j = 0; j <= x.NC; ++j) {
+        if (j < x.NC && !issue_m1(j)) break;
+        if (j == 0) continue;
+        const int i = j - 1, b = i & 1;
         if (!wait_bar(&B.tp_full, i & 1, x.abort_flag, p.err, 13)) break;
         if (i >= 2 && !wait_bar(&B.du_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 14)) break;
         if (i >= 1 && !wait_bar(&B.dw_empty, (i - 1) & 1, x.abort_flag, p.err, 19)) break;
@@ -548,6 +558,46 @@ __device__ __forceinline__ void mma_chain_role(const Ctx &x, const TcParams &p)
 // ------------------------------------------------------------------ prep warps
 // 8 warps (256 threads).  Warp pw reads TMEM lane quarter pw & 3 and handles
 // columns [32 * (pw >> 2), +32) of each row it owns.
+// Mask epilogue of one half row of [Q;K] K^T with every decay ratio taken as
+// one exp2 of a difference (the factorised form would leave the normal float
+// range: some half-chunk decays by more than 2^-120).  Rare, so it is kept out
+// of line; it reads its TMEM half row itself.
+template <int DIR>
+__device__ __noinline__ void m1_epi_direct(uint32_t taddr, const float *gt, float *As, uint32_t sP,
+                                           int qd, int lane, int hf)
+{
+    float xv[32];
+    tmem_ld32(taddr, xv);
+    tmem_wait_ld();
+    const int r = (qd & 1) * 32 + lane;
+    const int lr = DIR ? 63 - r : r;
+    const float Gr = gt[gG * 64 + r];
+    const float *Gj = gt + gG * 64 + 32 * hf;
+    if (qd < 2) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int j = 32 * hf + e;
+            const bool keep = DIR ? (j >= r) : (j <= r);
+            xv[e] = keep ? exp2f(Gr - Gj[e]) * xv[e] : 0.f;
+        }
+        store_half_row_bf16(sP, r, hf, xv);
+    } else {
+        const float br = gt[gBet * 64 + r];
+        float4 *Arow = reinterpret_cast<float4 *>(As + lr * kLDA + (DIR ? 32 * (1 - hf) : 32 * hf));
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            float o4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;
+                const int lj = DIR ? 63 - (32 * hf + e) : 32 * hf + e;
+                o4[u] = (lj < lr) ? br * exp2f(Gr - Gj[e]) * xv[e] : 0.f;
+            }
+            Arow[m] = make_float4(o4[0], o4[1], o4[2], o4[3]);
+        }
+    }
+}
+
 template <int DIR>
 __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int pt)
 {
@@ -632,66 +682,57 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
         if (gpt == 0) mbar_arrive(&B.g_full[gj]);
     };
     load_raw(0);
-    if (gate_thr) compute_gates(0);
-    named_bar(kBarPrep, kPrepThreads);
     PROF_DECL(pt == 0);
 
-    for (int i = 0; i < x.NC; ++i) {
+    // step i = -1 only computes the gates of chunk 0
+#pragma unroll 1
+    for (int i = -1; i < x.NC; ++i) {
         const int b = i & 1;
-        float *gt = gates_buf(x, i % kNG);
+        const int gi = (i + kNG) % kNG;
+        float *gt = gates_buf(x, gi);
         const bool dbg = kDbgOn && p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
                          blockIdx.z == 0;
-        const bool fact = x.bars->gscal[i % kNG][1] != 0.f;
-        PROF_MARK(16);
+        if (i >= 0) {
+            const bool fact = x.bars->gscal[gi][1] != 0.f;
+            PROF_MARK(16);
 
-        // ---- masks: P (rows of QK^T) and A (rows of KK^T, scan order)
-        wait_bar(&B.d1_full, i & 1, x.abort_flag, p.err, 3);
-        if (i >= 2) wait_bar(&B.p_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 4);
-        // A shares space with T1/T2 of chunk i-1: their products must be done
-        if (i >= 1) wait_bar(&B.wu_full, (i - 1) & 1, x.abort_flag, p.err, 6);
-        PROF_MARK(10);
-        tc_fence_after();
-        {
-            float xv[32];
-            tmem_ld32(x.tmem + tm_lane + kColD1 + 32 * hf, xv);
-            tmem_wait_ld();
-            if (dbg) dbg_half(p.debug + kDbgD1, qd * 32 + lane, hf, xv);
-            const int r = (qd & 1) * 32 + lane;            // physical token row
-            const int lr = DIR ? 63 - r : r;
-            const bool useB = lr >= 32 && col_h1;           // cross-half pairs
-            const float *cf = gt + (useB ? gCB : gCA) * 64 + 32 * hf;
-            const float *Gj = gt + gG * 64 + 32 * hf;
-            if (qd < 2) {
-                // P row r: keep j at or before r in scan order
-                if (fact) {
+            // ---- masks: P (rows of QK^T) and A (rows of KK^T, scan order)
+            wait_bar(&B.d1_full, i & 1, x.abort_flag, p.err, 3);
+            if (i >= 2) wait_bar(&B.p_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 4);
+            // A shares space with T1/T2 of chunk i-1: their products must be done
+            if (i >= 1) wait_bar(&B.wu_full, (i - 1) & 1, x.abort_flag, p.err, 6);
+            PROF_MARK(10);
+            tc_fence_after();
+            if (!fact) {
+                m1_epi_direct<DIR>(x.tmem + tm_lane + kColD1 + 32 * hf, gt, As, x.sbase + kOffP + b * 8192, qd,
+                                   lane, hf);
+            } else {
+                float xv[32];
+                tmem_ld32(x.tmem + tm_lane + kColD1 + 32 * hf, xv);
+                tmem_wait_ld();
+                if (dbg) dbg_half(p.debug + kDbgD1, qd * 32 + lane, hf, xv);
+                const int r = (qd & 1) * 32 + lane;            // physical token row
+                const int lr = DIR ? 63 - r : r;
+                const bool useB = lr >= 32 && col_h1;           // cross-half pairs
+                const float *cf = gt + (useB ? gCB : gCA) * 64 + 32 * hf;
+                if (qd < 2) {
+                    // P row r: keep j at or before r in scan order
                     const float rf = gt[(useB ? gRB : gRA) * 64 + r];
-#pragma unroll
+    #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int j = 32 * hf + e;
                         const bool keep = DIR ? (j >= r) : (j <= r);
                         xv[e] = keep ? rf * cf[e] * xv[e] : 0.f;
                     }
-                } else {   // rare: a half-chunk decays by more than 2^-240
-                    const float Gr = gt[gG * 64 + r];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = 32 * hf + e;
-                        const bool keep = DIR ? (j >= r) : (j <= r);
-                        xv[e] = keep ? exp2f(Gr - Gj[e]) * xv[e] : 0.f;
-                    }
-                }
-                store_half_row_bf16(x.sbase + kOffP + b * 8192, r, hf, xv);
-            } else {
-                // A row r, written in scan order: row lr, columns lj
-                const float br = gt[gBet * 64 + r];
-                const float rf = br * gt[(useB ? gRB : gRA) * 64 + r];
-                const float Gr = gt[gG * 64 + r];
-                float4 *Arow = reinterpret_cast<float4 *>(As + lr * kLDA + (DIR ? 32 * (1 - hf) : 32 * hf));
-                if (fact) {
-#pragma unroll
+                    store_half_row_bf16(x.sbase + kOffP + b * 8192, r, hf, xv);
+                } else {
+                    // A row r, written in scan order: row lr, columns lj
+                    const float rf = gt[gBet * 64 + r] * gt[(useB ? gRB : gRA) * 64 + r];
+                    float4 *Arow = reinterpret_cast<float4 *>(As + lr * kLDA + (DIR ? 32 * (1 - hf) : 32 * hf));
+    #pragma unroll
                     for (int m = 0; m < 8; ++m) {
                         float o4[4];
-#pragma unroll
+    #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;   // physical column 32 hf + e
                             const int lj = DIR ? 63 - (32 * hf + e) : 32 * hf + e;
@@ -699,29 +740,21 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
                         }
                         Arow[m] = make_float4(o4[0], o4[1], o4[2], o4[3]);
                     }
-                } else {   // rare: a half-chunk decays by more than 2^-240
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        float o4[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;
-                            const int lj = DIR ? 63 - (32 * hf + e) : 32 * hf + e;
-                            o4[u] = (lj < lr) ? br * exp2f(Gr - Gj[e]) * xv[e] : 0.f;
-                        }
-                        Arow[m] = make_float4(o4[0], o4[1], o4[2], o4[3]);
-                    }
                 }
             }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            PROF_MARK(11);
+            if (named_bar_any(kBarPrep, kPrepThreads, *x.abort_flag)) return;
+            if (pt == 0) mbar_arrive(&B.d1_empty);
         }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        PROF_MARK(11);
-        if (named_bar_any(kBarPrep, kPrepThreads, *x.abort_flag)) return;
-        if (pt == 0) mbar_arrive(&B.d1_empty);
 
         // ---- T = (I + A)^-1 ; meanwhile warps 2-3 prepare the next chunk's gates
         if (gate_thr && i + 1 < x.NC) compute_gates(i + 1);
+        if (i < 0) {
+            named_bar(kBarPrep, kPrepThreads);
+            continue;
+        }
         solve_diag_blocks(As, Ts, pt);
         PROF_MARK(13);
         solve_off_diag(As, Ts, pt);
@@ -850,44 +883,39 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
                 }
             }
         };
-        if (p.counters == nullptr) {
-            store_own();
-        } else {
-            int *cnt = p.counters + ((size_t)x.bh * x.NC + c) * p.n_slices + x.slice;
+        // causal: this CTA writes the tile.  Bidirectional: the direction
+        // that reaches the tile first writes its partial and counts it; the
+        // second waits for that count and adds its own partial.
+        bool first = true;
+        int *cnt = nullptr, target = 1;
+        if (p.counters != nullptr) {
+            cnt = p.counters + ((size_t)x.bh * x.NC + c) * p.n_slices + x.slice;
             if (p.predict) {
-                // every CTA is resident: the direction that reaches chunk c
-                // first is known (forward for the first half of the chunks)
-                const int first = (2 * c < x.NC) ? 0 : 1;
-                if (DIR == first) {
-                    store_own();
-                    named_bar(kBarChain, kChainThreads);
-                    if (ct == 0) {
-                        __threadfence();
-                        atomicAdd(cnt, 1);
-                    }
-                } else {
-                    wait_count(cnt, 1);
-                    named_bar(kBarChain, kChainThreads);
-                    add_other();
-                }
+                // every CTA is resident: the forward scan reaches the first
+                // half of the chunks first, the reverse scan the second half
+                first = DIR == ((2 * c < x.NC) ? 0 : 1);
             } else {
-                // arrival order decided at run time: the first to arrive writes
-                // its partial, the second waits until it is written and adds
+                // arrival order decided at run time by a claim on the counter
+                // (0 -> 1 -> 2), the partial's arrival brings it to 3
                 if (ct == 0) x.bars->s_old = atomicAdd(cnt, 1);
                 named_bar(kBarChain, kChainThreads);
-                if (x.bars->s_old == 0) {
-                    store_own();
-                    named_bar(kBarChain, kChainThreads);
-                    if (ct == 0) {
-                        __threadfence();
-                        atomicAdd(cnt, 1);
-                    }
-                } else {
-                    wait_count(cnt, 3);
-                    named_bar(kBarChain, kChainThreads);
-                    add_other();
+                first = x.bars->s_old == 0;
+                target = 3;
+            }
+        }
+        if (first) {
+            store_own();
+            if (cnt != nullptr) {
+                named_bar(kBarChain, kChainThreads);
+                if (ct == 0) {
+                    __threadfence();
+                    atomicAdd(cnt, 1);
                 }
             }
+        } else {
+            wait_count(cnt, target);
+            named_bar(kBarChain, kChainThreads);
+            add_other();
         }
         tc_fence_before();
         PROF_MARK(25);
@@ -896,63 +924,66 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
         return true;
     };
 
-    for (int i = 0; i < x.NC; ++i) {
+#pragma unroll 1
+    for (int i = 0; i <= x.NC; ++i) {
         const int b = i & 1, c = chunk_of<DIR>(x, i), gi = i % kNG;
         const float *gt = gates_buf(x, gi);
         const bool dbg = kDbgOn && p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
                          blockIdx.z == 0;
-
-        // ---- W (MN-major, row d = key index) and gamma-scaled Q of chunk i
-        wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 7);
-        wait_bar(&B.wu_full, i & 1, x.abort_flag, p.err, 5);
-        PROF_MARK(26);
-        tc_fence_after();
-        {
-            float xv[32];
-            tmem_ld32(x.tmem + tm_lane + kColW + 32 * chf, xv);
-            tmem_wait_ld();
-            if (dbg) {
-                dbg_half(p.debug + kDbgW, d, chf, xv);
-                float yv[32];
-                tmem_ld32(x.tmem + tm_lane + kColU0 + 64 * b + 32 * chf, yv);
+        if (i < x.NC) {
+            // ---- W (MN-major, row d = key index) and gamma-scaled Q of chunk i
+            wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 7);
+            wait_bar(&B.wu_full, i & 1, x.abort_flag, p.err, 5);
+            PROF_MARK(26);
+            tc_fence_after();
+            {
+                float xv[32];
+                tmem_ld32(x.tmem + tm_lane + kColW + 32 * chf, xv);
                 tmem_wait_ld();
-                dbg_half(p.debug + kDbgUt, d, chf, yv);
-            }
-            store_half_row_bf16(x.sbase + kOffW, d, chf, xv);
-        }
-        {
-            // gamma-scale Q in place (Q is no longer needed unscaled); bf16x2
-            // products: gamma is rounded to bf16 first, one more bf16 rounding
-            const int rq = ct >> 2, kb = (ct >> 1) & 1, part = ct & 1;
-            const __nv_bfloat162 g2 = __float2bfloat162_rn(gt[gGam * 64 + rq]);
-            const uint32_t rowbase = stage_addr(x, i) + kb * 16384;
-            uint32_t w[4][4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(w[q][0]), "=r"(w[q][1]), "=r"(w[q][2]), "=r"(w[q][3])
-                             : "r"(rowbase + sw128_off(rq, 8 * (4 * part + q))));
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    __nv_bfloat162 v = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&w[q][u]), g2);
-                    w[q][u] = *reinterpret_cast<uint32_t *>(&v);
+                if (dbg) {
+                    dbg_half(p.debug + kDbgW, d, chf, xv);
+                    float yv[32];
+                    tmem_ld32(x.tmem + tm_lane + kColU0 + 64 * b + 32 * chf, yv);
+                    tmem_wait_ld();
+                    dbg_half(p.debug + kDbgUt, d, chf, yv);
                 }
-                st_shared_v4(rowbase + sw128_off(rq, 8 * (4 * part + q)), w[q][0], w[q][1], w[q][2], w[q][3]);
+                store_half_row_bf16(x.sbase + kOffW, d, chf, xv);
             }
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        PROF_MARK(27);
-        if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return;
-        if (ct == 0) {
-            mbar_arrive(&B.wmn_full);
-            mbar_arrive(&B.dw_empty);
+            {
+                // gamma-scale Q in place (Q is no longer needed unscaled); bf16x2
+                // products: gamma is rounded to bf16 first, one more bf16 rounding
+                const int rq = ct >> 2, kb = (ct >> 1) & 1, part = ct & 1;
+                const __nv_bfloat162 g2 = __float2bfloat162_rn(gt[gGam * 64 + rq]);
+                const uint32_t rowbase = stage_addr(x, i) + kb * 16384;
+                uint32_t w[4][4];
+    #pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[q][0]), "=r"(w[q][1]), "=r"(w[q][2]), "=r"(w[q][3])
+                                 : "r"(rowbase + sw128_off(rq, 8 * (4 * part + q))));
+    #pragma unroll
+                for (int q = 0; q < 4; ++q) {
+    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        __nv_bfloat162 v = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&w[q][u]), g2);
+                        w[q][u] = *reinterpret_cast<uint32_t *>(&v);
+                    }
+                    st_shared_v4(rowbase + sw128_off(rq, 8 * (4 * part + q)), w[q][0], w[q][1], w[q][2], w[q][3]);
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            PROF_MARK(27);
+            if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return;
+            if (ct == 0) {
+                mbar_arrive(&B.wmn_full);
+                mbar_arrive(&B.dw_empty);
+            }
         }
 
         // ---- output tile of the previous chunk (overlaps this chunk's products)
         if (i > 0 && !out_tile(i - 1)) return;
+        if (i == x.NC) break;
 
         // ---- U and Ubar rows of chunk i
         wait_bar(&B.chain_full, i & 1, x.abort_flag, p.err, 8);
@@ -1008,7 +1039,6 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
             mbar_arrive(&B.g_empty[gi]);
         }
     }
-    if (x.NC > 0 && !out_tile(x.NC - 1)) return;
     PROF_FLUSH();
 
     if (p.state_out) {

@@ -83,6 +83,20 @@ def test_bf16_slow_decay_long(oracle_mod, kernel):
 
 
 @pytest.mark.parametrize("kernel", BF16_KERNELS)
+def test_bf16_fast_decay(oracle_mod, kernel):
+    """a ~ 2^-11 per token in the first 250 tokens, ~0.9 after: the early
+    chunks decay by far more than 2^-120 within a half chunk, so the kernel
+    cannot split their decay ratios into row and column factors and takes each
+    ratio as one exponential; the later chunks take the factorised form."""
+    inp = make_custom(1, 2, 500, 128, 128, dtype="bf16", seed=8, decay_shift=8.0, state0=True)
+    slow = make_custom(1, 2, 500, 128, 128, dtype="bf16", seed=9, decay_shift=-2.0)
+    inp.decay[..., 250:] = slow.decay[..., 250:]
+    assert float(inp.decay[..., :250].max()) < 0.05
+    check(oracle_mod, inp, False, recurrent=(kernel == "recurrent"))
+    check(oracle_mod, inp, True, recurrent=(kernel == "recurrent"))
+
+
+@pytest.mark.parametrize("kernel", BF16_KERNELS)
 def test_bf16_no_decay_unit_gates(oracle_mod, kernel):
     """a = 1, b = 1: the pure delta rule, the hardest case for carried error."""
     inp = make_custom(1, 2, 500, 128, 128, dtype="bf16", seed=6, state0=True)
