@@ -71,7 +71,7 @@ constexpr int kThreads = 608;    // 8 chain + 8 prep + TMA + 2 MMA-issue warps
 constexpr int kChainThreads = 256, kPrepThreads = 256;
 constexpr int kNS = 3;           // input stages
 constexpr int kLDA = 68;         // fp32 row stride of the solve buffers
-constexpr int kBarPrep = 1, kBarChain = 2, kBarGates = 3;   // named barriers (prep, chain, gate warps)
+constexpr int kBarPrep = 1, kBarChain = 2, kBarGates = 3, kBarSolve = 4;   // named barriers (prep, chain, gate warps)
 
 // TMEM columns (fp32 accumulators)
 constexpr uint32_t kColD1 = 0;     // [Q;K] K^T   (M=128)
@@ -89,19 +89,18 @@ constexpr uint32_t kOffW = kOffP + 16384;              // 16 KB bf16 [d][i]  (W,
 constexpr uint32_t kOffU = kOffW + 16384;              // 8 KB  bf16 [i][e]
 constexpr uint32_t kOffUb = kOffU + 8192;              // 8 KB
 constexpr uint32_t kOffH = kOffUb + 8192;              // 16 KB bf16 [d][e]
-constexpr uint32_t kOffA = kOffH + 16384;              // fp32 [64][68], scan order
-constexpr uint32_t kOffT1 = kOffA;                     // T1, T2 (bf16) reuse A after the solve
-constexpr uint32_t kOffT2 = kOffA + 8192;
-constexpr uint32_t kOffT = kOffA + 64 * kLDA * 4;      // fp32 [64][68], scan order
+constexpr uint32_t kOffA = kOffH + 16384;              // fp32 [64][68], scan order: A, then T in place
+constexpr uint32_t kOffT1 = kOffA + 64 * kLDA * 4;     // 8 KB bf16 [i][j]
+constexpr uint32_t kOffT2 = kOffT1 + 8192;             // 8 KB bf16 [i][j]
 constexpr int kNG = 3;                                 // gate buffers (prep runs ahead)
 constexpr uint32_t kGateFloats = 9 * 64;               // per buffer, see GateIdx
-constexpr uint32_t kOffGates = kOffT + 64 * kLDA * 4;
+constexpr uint32_t kOffGates = kOffT2 + 8192;
 constexpr uint32_t kOffBar = kOffGates + kNG * kGateFloats * 4;
 constexpr uint32_t kOffProf = kOffBar + 512;            // 32 x 8 B (profiling builds)
 constexpr uint32_t kSmemBytes = kOffProf + 256;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;     // alignment slack
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
-static_assert(kOffA % 1024 == 0 && kOffT2 % 1024 == 0 && kOffP % 1024 == 0, "tile alignment");
+static_assert(kOffT1 % 1024 == 0 && kOffT2 % 1024 == 0 && kOffP % 1024 == 0, "tile alignment");
 
 // gate arrays (64 floats each, physical token order unless noted)
 // G (log2 cumulative decay), gamma = 2^G, beta, beta*gamma, 2^(G_end - G), row/column
@@ -285,6 +284,7 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 }
 
 // T = (I + A)^-1 for a strictly lower-triangular 64 x 64 fp32 A (scan order),
+// in place (T overwrites A; each block of A is read before it is replaced),
 // by the 256 prep threads, in four barrier-separated steps:
 //   1. the four 16 x 16 diagonal blocks D_a by forward substitution (one
 //      column per thread, right-looking so one FMA per step is serial);
@@ -293,14 +293,13 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 //   3. Y = A[32:64, 0:32] T[0:32, 0:32]                  (tf32 mma.sync)
 //   4. T[32:64, 0:32] = -T[32:64, 32:64] Y               (tf32 mma.sync)
 // Products skip the k-steps that the triangular factors make zero.  The
-// upper-right 32 x 32 block of Ts is scratch for the intermediate products;
-// every other upper-triangular entry of Ts stays zero (callers mask the
-// scratch block out when they read T).
-__device__ __forceinline__ void solve_diag_blocks(const float *As, float *Ts, int pt)
+// upper-right 32 x 32 block (zero in A) is scratch for the intermediate
+// products, so callers mask it out when they read T.
+__device__ __forceinline__ void solve_diag_blocks(float *As, int pt)
 {
     if (pt < 64) {
         const int a = pt >> 4, c = pt & 15;
-        const float *Ab = As + (16 * a) * kLDA + 16 * a;
+        float *Ab = As + (16 * a) * kLDA + 16 * a;
         float x[16], acc[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) acc[r] = 0.f;
@@ -310,9 +309,9 @@ __device__ __forceinline__ void solve_diag_blocks(const float *As, float *Ts, in
 #pragma unroll
             for (int r = m + 1; r < 16; ++r) acc[r] = fmaf(Ab[r * kLDA + m], x[m], acc[r]);
         }
-        float *Tb = Ts + (16 * a) * kLDA + 16 * a;
+        __syncwarp();   // the block's 16 columns are one half warp: all reads done
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tb[r * kLDA + c] = x[r];
+        for (int r = 0; r < 16; ++r) Ab[r * kLDA + c] = x[r];
     }
     named_bar(kBarPrep, kPrepThreads);
 }
@@ -347,9 +346,10 @@ __device__ __forceinline__ void store_strip(float *M, int r0, int c0, const floa
     Mr[8 * kLDA + 1] = sgn * d[3];
 }
 
-__device__ __forceinline__ void solve_off_diag(const float *As, float *Ts, int pt)
+__device__ __forceinline__ void solve_off_diag(float *Ts, int pt)
 {
     const int pw = pt >> 5, lane = pt & 31, g = lane >> 2, q = lane & 3;
+    const float *As = Ts;
     // step 2: T_ab, (a,b) in {(1,0), (3,2)}; warp = (block, 8-column strip)
     if (pw < 4) {
         const int a = (pw >> 1) ? 3 : 1, b = a - 1, nt = pw & 1;
@@ -357,7 +357,8 @@ __device__ __forceinline__ void solve_off_diag(const float *As, float *Ts, int p
         mma_strip(y, As, 16 * a, Ts, 16 * b + 8 * nt, 16 * b + 8 * nt, 2 - nt, g, q);   // A_ab D_b
         // Y strip (16 x 8) parked in the scratch block: rows 0..15, cols 32 + 8 pw
         store_strip(Ts, 0, 32 + 8 * pw, y, 1.f, g, q);
-        __syncwarp();
+        // both strips of A_ab are read before either warp overwrites it with T_ab
+        named_bar(kBarSolve, 128);
         float e[4] = {0.f, 0.f, 0.f, 0.f};
         // -D_a Y : D_a = T[16a.., 16a..], Y rows are the k index
         for (int s = 0; s < 2; ++s) {
@@ -604,7 +605,6 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
     Bars &B = *x.bars;
     const int pw = pt >> 5, lane = pt & 31, qd = pw & 3, hf = pw >> 2;
     float *As = reinterpret_cast<float *>(x.smem + kOffA);
-    float *Ts = reinterpret_cast<float *>(x.smem + kOffT);
     const uint32_t tm_lane = (uint32_t)(qd * 32) << 16;
     const float *beta_h = p.beta + (size_t)x.bh * x.T;
     const float *decay_h = p.decay + (size_t)x.bh * x.T;
@@ -699,8 +699,6 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
             // ---- masks: P (rows of QK^T) and A (rows of KK^T, scan order)
             wait_bar(&B.d1_full, i & 1, x.abort_flag, p.err, 3);
             if (i >= 2) wait_bar(&B.p_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 4);
-            // A shares space with T1/T2 of chunk i-1: their products must be done
-            if (i >= 1) wait_bar(&B.wu_full, (i - 1) & 1, x.abort_flag, p.err, 6);
             PROF_MARK(10);
             tc_fence_after();
             if (!fact) {
@@ -755,22 +753,25 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
             named_bar(kBarPrep, kPrepThreads);
             continue;
         }
-        solve_diag_blocks(As, Ts, pt);
+        solve_diag_blocks(As, pt);
         PROF_MARK(13);
-        solve_off_diag(As, Ts, pt);
+        solve_off_diag(As, pt);
         PROF_MARK(17);
         if (dbg)
             for (int e = pt; e < 64 * 64; e += kPrepThreads) {
                 const int rr = e >> 6, cc = e & 63;
-                p.debug[kDbgT + e] = (cc <= rr) ? Ts[rr * kLDA + cc] : 0.f;
+                p.debug[kDbgT + e] = (cc <= rr) ? As[rr * kLDA + cc] : 0.f;
             }
 
-        // ---- T1 = T diag(b gamma), T2 = T diag(b), physical order, into A's space
+        // ---- T1 = T diag(b gamma), T2 = T diag(b), physical order; the
+        // products of chunk i-1 must be done with the previous T1, T2
+        if (i >= 1) wait_bar(&B.wu_full, (i - 1) & 1, x.abort_flag, p.err, 6);
+        tc_fence_after();
         {
             const int second = pt >> 7, r = (pt >> 1) & 63, h2 = pt & 1;
             const int lr = DIR ? 63 - r : r;
             // scan-order columns of physical half h2
-            const float4 *Trow = reinterpret_cast<const float4 *>(Ts + lr * kLDA + (DIR ? 32 * (1 - h2) : 32 * h2));
+            const float4 *Trow = reinterpret_cast<const float4 *>(As + lr * kLDA + (DIR ? 32 * (1 - h2) : 32 * h2));
             const float *sc = gt + (second ? gBet : gBG) * 64 + 32 * h2;
             float xv[32];
 #pragma unroll
@@ -1086,8 +1087,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tmem_alloc(&B.tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    float *Ts = reinterpret_cast<float *>(smem + kOffT);
-    for (int i = tid; i < 64 * kLDA; i += kThreads) Ts[i] = 0.f;
+    float *As0 = reinterpret_cast<float *>(smem + kOffA);
+    for (int i = tid; i < 64 * kLDA; i += kThreads) As0[i] = 0.f;
     if (tid < 32) reinterpret_cast<long long *>(smem + kOffProf)[tid] = 0;
 #ifdef GDN_PROFILE
     const unsigned long long prof_start = globaltimer();
