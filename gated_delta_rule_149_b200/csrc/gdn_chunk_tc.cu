@@ -67,11 +67,11 @@ using namespace ptx;
 constexpr int kC = 64;           // chunk length
 constexpr int kDK = 128;         // key dim served by this kernel
 constexpr int kDVS = 64;         // dv columns per CTA
-constexpr int kThreads = 608;    // 8 chain + 8 prep + TMA + 2 MMA-issue warps
+constexpr int kThreads = 640;    // 8 chain + 8 prep + TMA + 2 MMA-issue + combine warps
 constexpr int kChainThreads = 256, kPrepThreads = 256;
 constexpr int kNS = 3;           // input stages
 constexpr int kLDA = 68;         // fp32 row stride of the solve buffers
-constexpr int kBarPrep = 1, kBarChain = 2, kBarGates = 3, kBarSolve = 4;   // named barriers (prep, chain, gate warps)
+constexpr int kBarPrep = 1, kBarChain = 2, kBarGates = 3;   // named barriers (prep, chain, gate warps)
 
 // TMEM columns (fp32 accumulators)
 constexpr uint32_t kColD1 = 0;     // [Q;K] K^T   (M=128)
@@ -150,12 +150,36 @@ struct TcParams {
 #define PROF_FLUSH() \
     do {             \
     } while (0)
+#define PROF_SETC(c) \
+    do {             \
+    } while (0)
+#elif defined(GDN_TRACE)
+// Event trace for tracing builds (-DGDN_TRACE): the leader thread of each role
+// in CTA (0,0,0) stores clock64() at each mark for the chunks of a short window
+// (role-local chunk index), to read the critical path off the timestamps.
+constexpr int kTrace0 = 200, kTraceN = 4, kTraceBase = 4096;
+#define PROF_DECL(lead)                                                                     \
+    const bool prof_on = p.prof != nullptr && (lead) && blockIdx.x == 0 && blockIdx.y == 0 && \
+                         blockIdx.z == 0;                                                   \
+    int prof_c = 0;
+#define PROF_SETC(c) prof_c = (c)
+#define PROF_MARK(slot)                                                                    \
+    do {                                                                                   \
+        if (prof_on && prof_c >= kTrace0 && prof_c < kTrace0 + kTraceN)                    \
+            p.prof[kTraceBase + (prof_c - kTrace0) * 32 + (slot)] = (long long)clock64(); \
+    } while (0)
+#define PROF_FLUSH() \
+    do {             \
+    } while (0)
 #else
 #define PROF_DECL(lead)
 #define PROF_MARK(slot) \
     do {                \
     } while (0)
 #define PROF_FLUSH() \
+    do {             \
+    } while (0)
+#define PROF_SETC(c) \
     do {             \
     } while (0)
 #endif
@@ -183,6 +207,8 @@ struct Bars {
     int abort_flag;
     int s_old;
     float s_wsum;
+    int stored_upto;   // last output tile the chain warps stored as first writer
+    int ready_upto;    // last output tile whose other-direction partial is visible
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
 
@@ -219,6 +245,67 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     return wait_bar_slow(bar, parity, abort_flag, err, code);
 }
 
+__device__ __forceinline__ void st_release_cta(int *addr, int v)
+{
+    asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32(addr)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_cta(const int *addr)
+{
+    int v;
+    asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(addr)) : "memory");
+    return v;
+}
+
+// Bounded wait until a shared-memory word written by another warp of the CTA
+// reaches `target`; false on timeout (error recorded, abort raised) or abort.
+__device__ __noinline__ bool wait_smem_slow(const int *addr, int target, volatile int *abort_flag, int *err,
+                                            int code)
+{
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t it = 0; it < (1u << 30); ++it) {
+        if (ld_acquire_cta(addr) >= target) return true;
+        if (*abort_flag) return false;
+        if ((it & 255) == 255 && globaltimer() - t0 > kWaitLimitNs) break;
+    }
+    atomicOr(err, code);
+    *abort_flag = 1;
+    return false;
+}
+
+__device__ __forceinline__ bool wait_smem_at_least(const int *addr, int target, volatile int *abort_flag,
+                                                   int *err, int code)
+{
+    if (ld_acquire_cta(addr) >= target) return true;
+    return wait_smem_slow(addr, target, abort_flag, err, code);
+}
+
+// Bounded wait (one thread) until a device-wide counter reaches `target`,
+// with acquire semantics at GPU scope; false on timeout or abort.
+__device__ __noinline__ bool spin_global_at_least(const int *cnt, int target, volatile int *abort_flag)
+{
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t it = 0; it < (1u << 30); ++it) {
+        int seen;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(cnt) : "memory");
+        if (seen >= target) return true;
+        if (*abort_flag) return false;
+        if ((it & 63) == 63) {
+            if (globaltimer() - t0 > kWaitLimitNs) return false;
+            __nanosleep(64);
+        }
+    }
+    return false;
+}
+
+// o[0..8) += x (eight bf16 values packed in four words), added in L2
+__device__ __forceinline__ void red_add_bf16x8(__nv_bfloat16 *addr, uint32_t a, uint32_t b, uint32_t c,
+                                               uint32_t d)
+{
+    asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};" ::"l"(addr), "r"(a), "r"(b),
+                 "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void named_bar(int id, int count)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -243,20 +330,22 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d)
+// Shared-memory tiles are written with plain stores through pointers derived
+// from the dynamic shared array, so that the compiler can schedule them freely
+// (the fences and barriers that publish them carry the ordering).
+__device__ __forceinline__ void st_tile_v4(uint8_t *tile, uint32_t off, uint32_t a, uint32_t b, uint32_t c,
+                                           uint32_t d)
 {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-                 "r"(d) : "memory");
+    *reinterpret_cast<uint4 *>(tile + off) = make_uint4(a, b, c, d);
 }
 
 // Writes 32 fp32 values as half (64 bytes, 16-byte chunks 4h..4h+3) of a
 // 128-byte bf16 row of a 128B-swizzled tile.
-__device__ __forceinline__ void store_half_row_bf16(uint32_t tile, uint32_t row, int h, const float *x)
+__device__ __forceinline__ void store_half_row_bf16(uint8_t *tile, uint32_t row, int h, const float *x)
 {
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-        st_shared_v4(tile + sw128_off(row, 32 * h + 8 * q), pack_bf16(x[8 * q + 0], x[8 * q + 1]),
+        st_tile_v4(tile, sw128_off(row, 32 * h + 8 * q), pack_bf16(x[8 * q + 0], x[8 * q + 1]),
                      pack_bf16(x[8 * q + 2], x[8 * q + 3]), pack_bf16(x[8 * q + 4], x[8 * q + 5]),
                      pack_bf16(x[8 * q + 6], x[8 * q + 7]));
 }
@@ -283,19 +372,30 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// T = (I + A)^-1 for a strictly lower-triangular 64 x 64 fp32 A (scan order),
-// in place (T overwrites A; each block of A is read before it is replaced),
-// by the 256 prep threads, in four barrier-separated steps:
-//   1. the four 16 x 16 diagonal blocks D_a by forward substitution (one
-//      column per thread, right-looking so one FMA per step is serial);
-//   2. the two 16 x 16 blocks below them inside each 32 x 32 half,
-//      T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2 (tf32 mma.sync);
-//   3. Y = A[32:64, 0:32] T[0:32, 0:32]                  (tf32 mma.sync)
-//   4. T[32:64, 0:32] = -T[32:64, 32:64] Y               (tf32 mma.sync)
-// Products skip the k-steps that the triangular factors make zero.  The
-// upper-right 32 x 32 block (zero in A) is scratch for the intermediate
-// products, so callers mask it out when they read T.
-__device__ __forceinline__ void solve_diag_blocks(float *As, int pt)
+// T = (I + A)^-1 for a strictly lower-triangular 64 x 64 fp32 A (scan order)
+// in 16 x 16 blocks, written straight into the bf16 operands
+// T1 = T diag(b gamma) and T2 = T diag(b) (physical order, 128B-swizzled):
+//   1. the diagonal blocks D_a = (I + A_aa)^-1 by forward substitution, one
+//      column per thread (right-looking, so one FMA per step is serial); D_a
+//      replaces A_aa in place;
+//   2. the blocks below them by block-forward substitution,
+//      T_ab = -D_a sum_{b <= k < a} A_ak T_kb, each prep warp walking one
+//      8-column strip of T down the block rows with tf32 mma.sync, its
+//      earlier blocks kept in registers (no barrier between the steps),
+//      while the two remaining warps write the diagonal blocks' T1, T2.
+// The upper triangle of T1/T2 is never written: it is zeroed once.
+
+// bf16 pair (scan-order row lr, columns lj and lj + 1) into a physical-order
+// tile (dir 1: rows and columns reversed)
+__device__ __forceinline__ void st_tpair(uint8_t *tile, int dir, int lr, int lj, float v0, float v1)
+{
+    const int pr = dir ? 63 - lr : lr;
+    const int pc = dir ? 62 - lj : lj;   // the pair's lower physical column (even)
+    *reinterpret_cast<uint32_t *>(tile + sw128_off(pr, pc)) = dir ? pack_bf16(v1, v0) : pack_bf16(v0, v1);
+}
+
+__device__ __forceinline__ void solve_diag_blocks(float *As, const float *gt, uint8_t *sT1, uint8_t *sT2,
+                                               float *dbgT, int dir, int pt)
 {
     if (pt < 64) {
         const int a = pt >> 4, c = pt & 15;
@@ -312,87 +412,127 @@ __device__ __forceinline__ void solve_diag_blocks(float *As, int pt)
         __syncwarp();   // the block's 16 columns are one half warp: all reads done
 #pragma unroll
         for (int r = 0; r < 16; ++r) Ab[r * kLDA + c] = x[r];
+        if (dbgT)
+            for (int r = 0; r < 16; ++r) dbgT[(16 * a + r) * 64 + 16 * a + c] = x[r];
     }
     named_bar(kBarPrep, kPrepThreads);
 }
 
-// D(16x8) += A[rows r0.., cols k0..k0+8*nk) * B[rows k0.., cols c0..c0+8), fp32 smem, tf32 MMA
-__device__ __forceinline__ void mma_strip(float (&d)[4], const float *Am, int r0, const float *Bm,
-                                          int c0, int k0, int nk, int g, int q)
+// T1, T2 of the four diagonal blocks, from D_a in place in A (64 threads: each
+// writes 16 column pairs of one block row band; a compact loop, run by warps
+// that have no off-diagonal strip).
+__device__ __forceinline__ void store_diag_t12(const float *As, const float *gt, uint8_t *sT1, uint8_t *sT2,
+                                               int dir, int t)
 {
-    for (int s = 0; s < nk; ++s) {
-        const int kk = k0 + 8 * s;
-        uint32_t af[4], bf[2];
-        const float *Ar = Am + (r0 + g) * kLDA + kk + q;
-        af[0] = to_tf32(Ar[0]);
-        af[1] = to_tf32(Ar[8 * kLDA]);
-        af[2] = to_tf32(Ar[4]);
-        af[3] = to_tf32(Ar[8 * kLDA + 4]);
-        const float *Br = Bm + (kk + q) * kLDA + c0 + g;
-        bf[0] = to_tf32(Br[0]);
-        bf[1] = to_tf32(Br[4 * kLDA]);
-        mma_tf32(d, af, bf);
+    const int a = t >> 4, cp = (t & 7) * 2, rh = (t >> 3) & 1;   // block, column pair, row half
+    const int lj = 16 * a + cp;
+    const int pc0 = dir ? 63 - lj : lj, pc1 = dir ? 62 - lj : lj + 1;
+    const float sg0 = gt[gBG * 64 + pc0], sg1 = gt[gBG * 64 + pc1];
+    const float sb0 = gt[gBet * 64 + pc0], sb1 = gt[gBet * 64 + pc1];
+#pragma unroll 1
+    for (int r = 8 * rh; r < 8 * rh + 8; ++r) {
+        const int lr = 16 * a + r;
+        const float2 v = *reinterpret_cast<const float2 *>(As + lr * kLDA + lj);
+        st_tpair(sT1, dir, lr, lj, v.x * sg0, v.y * sg1);
+        st_tpair(sT2, dir, lr, lj, v.x * sb0, v.y * sb1);
     }
 }
 
-// writes a 16 x 8 accumulator strip (times sgn) at rows r0.., cols c0.. of M
-__device__ __forceinline__ void store_strip(float *M, int r0, int c0, const float (&d)[4], float sgn,
-                                            int g, int q)
+// tf32 A fragment (rows r0.., columns k0..) of an fp32 [64][kLDA] matrix
+__device__ __forceinline__ void ld_afrag(uint32_t (&a)[4], const float *M, int r0, int k0, int g, int q)
 {
-    float *Mr = M + (r0 + g) * kLDA + c0 + 2 * q;
-    Mr[0] = sgn * d[0];
-    Mr[1] = sgn * d[1];
-    Mr[8 * kLDA] = sgn * d[2];
-    Mr[8 * kLDA + 1] = sgn * d[3];
+    const float *p = M + (r0 + g) * kLDA + k0 + q;
+    a[0] = to_tf32(p[0]);
+    a[1] = to_tf32(p[8 * kLDA]);
+    a[2] = to_tf32(p[4]);
+    a[3] = to_tf32(p[8 * kLDA + 4]);
 }
 
-__device__ __forceinline__ void solve_off_diag(float *Ts, int pt)
+// A 16 x 8 accumulator tile (C layout) rearranged, through shuffles, into the
+// B operand of a following m16n8k8 product (two k-steps of 8 rows), as tf32
+__device__ __forceinline__ void c_to_b(const float (&c)[4], uint32_t (&b)[2][2], int g, int q)
 {
-    const int pw = pt >> 5, lane = pt & 31, g = lane >> 2, q = lane & 3;
-    const float *As = Ts;
-    // step 2: T_ab, (a,b) in {(1,0), (3,2)}; warp = (block, 8-column strip)
-    if (pw < 4) {
-        const int a = (pw >> 1) ? 3 : 1, b = a - 1, nt = pw & 1;
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_strip(y, As, 16 * a, Ts, 16 * b + 8 * nt, 16 * b + 8 * nt, 2 - nt, g, q);   // A_ab D_b
-        // Y strip (16 x 8) parked in the scratch block: rows 0..15, cols 32 + 8 pw
-        store_strip(Ts, 0, 32 + 8 * pw, y, 1.f, g, q);
-        // both strips of A_ab are read before either warp overwrites it with T_ab
-        named_bar(kBarSolve, 128);
-        float e[4] = {0.f, 0.f, 0.f, 0.f};
-        // -D_a Y : D_a = T[16a.., 16a..], Y rows are the k index
-        for (int s = 0; s < 2; ++s) {
-            const int kk = 8 * s;
-            uint32_t af[4], bf[2];
-            const float *Dr = Ts + (16 * a + g) * kLDA + 16 * a + kk + q;
-            af[0] = to_tf32(Dr[0]);
-            af[1] = to_tf32(Dr[8 * kLDA]);
-            af[2] = to_tf32(Dr[4]);
-            af[3] = to_tf32(Dr[8 * kLDA + 4]);
-            const float *Yr = Ts + (kk + q) * kLDA + 32 + 8 * pw + g;
-            bf[0] = to_tf32(Yr[0]);
-            bf[1] = to_tf32(Yr[4 * kLDA]);
-            mma_tf32(e, af, bf);
+    const int src0 = q * 4 + (g >> 1), src1 = (q + 4) * 4 + (g >> 1);
+    const bool odd = (g & 1) != 0;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const float lo0 = __shfl_sync(0xffffffffu, c[2 * ks], src0);
+        const float hi0 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src0);
+        const float lo1 = __shfl_sync(0xffffffffu, c[2 * ks], src1);
+        const float hi1 = __shfl_sync(0xffffffffu, c[2 * ks + 1], src1);
+        b[ks][0] = to_tf32(odd ? hi0 : lo0);
+        b[ks][1] = to_tf32(odd ? hi1 : lo1);
+    }
+}
+
+// Prep warp pw: the strip of columns [16 jb + 8 hs, +8) of T below its
+// diagonal block jb = pw / 2; the two warps of block column 3 (no block below
+// it) write the diagonal blocks' T1, T2 instead.
+__device__ __forceinline__ void solve_off_diag(const float *As, const float *gt, uint8_t *sT1, uint8_t *sT2,
+                                            float *dbgT, int dir, int pt)
+{
+    const int pw = pt >> 5, lane = pt & 31, g = lane >> 2, q = lane & 3, hs = pw & 1, jb = pw >> 1;
+    if (jb == 3) {   // no strip below block column 3: write the diagonal blocks' T1, T2
+        store_diag_t12(As, gt, sT1, sT2, dir, pt - 192);
+        return;
+    }
+    const int c0 = 16 * jb + 8 * hs;
+    uint32_t tb[3][2][2];   // B fragments of the strip's blocks in block rows jb, jb+1, jb+2
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        tb[0][ks][0] = to_tf32(As[(16 * jb + 8 * ks + q) * kLDA + c0 + g]);
+        tb[0][ks][1] = to_tf32(As[(16 * jb + 8 * ks + q + 4) * kLDA + c0 + g]);
+    }
+    const int lj = c0 + 2 * q;
+    const int pc0 = dir ? 63 - lj : lj, pc1 = dir ? 62 - lj : lj + 1;
+    const float sg0 = gt[gBG * 64 + pc0], sg1 = gt[gBG * 64 + pc1];
+    const float sb0 = gt[gBet * 64 + pc0], sb1 = gt[gBet * 64 + pc1];
+#pragma unroll
+    for (int io = 1; io < 4; ++io) {
+        const int ib = jb + io;   // block row
+        if (ib > 3) break;
+        // S = sum_k A_{ib,k} T_{k,jb}, two accumulators to halve the chain
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ko = 0; ko < 3; ++ko) {
+            if (ko >= io) break;
+            const int kb = jb + ko;
+            uint32_t a[4];
+            if (ko != 0 || hs == 0) {   // D_jb is zero above the strip's diagonal
+                ld_afrag(a, As, 16 * ib, 16 * kb, g, q);
+                mma_tf32(s0, a, tb[ko][0]);
+            }
+            ld_afrag(a, As, 16 * ib, 16 * kb + 8, g, q);
+            mma_tf32(s1, a, tb[ko][1]);
         }
-        store_strip(Ts, 16 * a, 16 * b + 8 * nt, e, -1.f, g, q);
+        float sv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) sv[u] = s0[u] + s1[u];
+        uint32_t sbf[2][2];
+        c_to_b(sv, sbf, g, q);
+        // T_{ib,jb} = -D_ib S
+        float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t a[4];
+            ld_afrag(a, As, 16 * ib, 16 * ib + 8 * ks, g, q);
+            mma_tf32(t, a, sbf[ks]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) t[u] = -t[u];
+        const int lr = 16 * ib + g;
+        st_tpair(sT1, dir, lr, lj, t[0] * sg0, t[1] * sg1);
+        st_tpair(sT1, dir, lr + 8, lj, t[2] * sg0, t[3] * sg1);
+        st_tpair(sT2, dir, lr, lj, t[0] * sb0, t[1] * sb1);
+        st_tpair(sT2, dir, lr + 8, lj, t[2] * sb0, t[3] * sb1);
+        if (dbgT) {
+            dbgT[lr * 64 + lj] = t[0];
+            dbgT[lr * 64 + lj + 1] = t[1];
+            dbgT[(lr + 8) * 64 + lj] = t[2];
+            dbgT[(lr + 8) * 64 + lj + 1] = t[3];
+        }
+        if (io < 3) c_to_b(t, tb[io], g, q);
     }
-    named_bar(kBarPrep, kPrepThreads);
-    // step 3: Y = A[32:64, 0:32] T[0:32, 0:32] -> scratch rows 0..31, cols 32..63
-    {
-        const int mt = pw >> 2, nt = pw & 3;
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_strip(y, As, 32 + 16 * mt, Ts, 8 * nt, 8 * nt, 4 - nt, g, q);
-        store_strip(Ts, 16 * mt, 32 + 8 * nt, y, 1.f, g, q);
-    }
-    named_bar(kBarPrep, kPrepThreads);
-    // step 4: T[32:64, 0:32] = -T[32:64, 32:64] Y
-    {
-        const int mt = pw >> 2, nt = pw & 3;
-        float e[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_strip(e, Ts + 32, 32 + 16 * mt, Ts + 32, 8 * nt, 0, 2 * mt + 2, g, q);
-        store_strip(Ts, 32 + 16 * mt, 8 * nt, e, -1.f, g, q);
-    }
-    named_bar(kBarPrep, kPrepThreads);
 }
 
 struct Ctx {
@@ -419,6 +559,7 @@ __device__ __forceinline__ void tma_role(const Ctx &x, const CUtensorMap *tmQ, c
     PROF_DECL(true);
     for (int i = 0; i < x.NC; ++i) {
         const int s = i % kNS;
+        PROF_SETC(i);
         PROF_MARK(1);
         if (i >= kNS && !wait_bar(&B.stage_empty[s], ((i / kNS) + 1) & 1, x.abort_flag, p.err, 1)) break;
         PROF_MARK(0);
@@ -430,6 +571,7 @@ __device__ __forceinline__ void tma_role(const Ctx &x, const CUtensorMap *tmQ, c
             tma_load_3d(st + kb * 16384 + 8192, tmK, &B.stage_full[s], kb * 64, c * kC, x.bh);
         }
         tma_load_3d(st + 32768, tmV, &B.stage_full[s], x.slice * kDVS, c * kC, x.bh);
+        PROF_MARK(18);
         issued = i + 1;
     }
     PROF_FLUSH();
@@ -443,6 +585,8 @@ __device__ __forceinline__ void tma_role(const Ctx &x, const CUtensorMap *tmQ, c
 }
 
 // ------------------------------------------------------------------ MMA warps
+// (Issue loops are not unrolled: the issuing threads are not the limit, and
+// small loop bodies leave more of the instruction cache to the epilogues.)
 // Two issuing threads, each waiting (suspended) on its next products' inputs in
 // a fixed order: one for the state-independent products of the prep pipeline,
 // one for the serial-chain products.  tcgen05.commit tracks the MMAs of the
@@ -457,14 +601,15 @@ __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
     PROF_DECL(true);
     // [Q;K] K^T of chunk j (needs its stage loaded and D1 read out for chunk j-1)
     auto issue_m1 = [&](int j) -> bool {
+        PROF_SETC(j);
         if (!wait_bar(&B.stage_full[j % kNS], (j / kNS) & 1, x.abort_flag, p.err, 11)) return false;
         if (j > 0 && !wait_bar(&B.d1_empty, (j - 1) & 1, x.abort_flag, p.err, 12)) return false;
         PROF_MARK(2);
         const uint32_t sQK = stage_addr(x, j);
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
+#pragma unroll 1
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tm + kColD1, sw128_desc(sQK + kb * 16384 + ks * 32, 16, 1024),
                          sw128_desc(sQK + kb * 16384 + 8192 + ks * 32, 16, 1024), kIdM1, (kb | ks) != 0);
@@ -480,22 +625,24 @@ __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
         if (j < x.NC && !issue_m1(j)) break;
         if (j == 0) continue;
         const int i = j - 1, b = i & 1;
+        PROF_SETC(i);
         if (!wait_bar(&B.tp_full, i & 1, x.abort_flag, p.err, 13)) break;
+        PROF_MARK(12);
         if (i >= 2 && !wait_bar(&B.du_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 14)) break;
         if (i >= 1 && !wait_bar(&B.dw_empty, (i - 1) & 1, x.abort_flag, p.err, 19)) break;
-        PROF_MARK(2);
+        PROF_MARK(7);
         const uint32_t sQK = stage_addr(x, i), sV = sQK + 32768;
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
             mma_bf16(tm + kColW, sw128_desc(sQK + 8192 + ks * 2048, 16384, 1024),
                      sw128_desc(sT1 + ks * 32, 16, 1024), kIdW, ks != 0);
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
             mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sT2 + ks * 32, 16, 1024),
                      sw128_desc(sV + ks * 2048, 8192, 1024), kIdUt, ks != 0);
         mma_commit(&B.wu_full);
-        PROF_MARK(6);
+        PROF_MARK(5);
     }
     PROF_FLUSH();
     // every issued MMA completes before the CTA releases its TMEM
@@ -515,33 +662,34 @@ __device__ __forceinline__ void mma_chain_role(const Ctx &x, const TcParams &p)
     for (int i = 0; i < x.NC; ++i) {
         const int b = i & 1;
         const uint32_t sQK = stage_addr(x, i);
+        PROF_SETC(i);
         PROF_MARK(28);
         if (!wait_bar(&B.wmn_full, i & 1, x.abort_flag, p.err, 15)) break;
         if (!wait_bar(&B.h_full, i & 1, x.abort_flag, p.err, 16)) break;
         if (i >= 2 && !wait_bar(&B.do_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 17)) break;
-        PROF_MARK(26);
+        PROF_MARK(29);
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 8; ++ks)
             mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sW + ks * 2048, 8192, 1024),
                      sw128_desc(sH + ks * 2048, 8192, 1024), kIdUc, 1);
         mma_commit(&B.chain_full);
-#pragma unroll
+#pragma unroll 1
         for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
+#pragma unroll 1
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tm + kColO0 + 64 * b, sw128_desc(sQK + kb * 16384 + ks * 32, 16, 1024),
                          sw128_desc(sH + (kb * 4 + ks) * 2048, 8192, 1024), kIdOq, (kb | ks) != 0);
         PROF_MARK(4);
         if (!wait_bar(&B.u_full, i & 1, x.abort_flag, p.err, 18)) break;
-        PROF_MARK(27);
+        PROF_MARK(30);
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
             mma_bf16(tm + kColS, sw128_desc(sQK + 8192 + ks * 2048, 16384, 1024),
                      sw128_desc(sUb + ks * 2048, 8192, 1024), kIdS, ks != 0);
         mma_commit(&B.s_full);
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
             mma_bf16(tm + kColO0 + 64 * b, sw128_desc(sP + b * 8192 + ks * 32, 16, 1024),
                      sw128_desc(sU + ks * 2048, 8192, 1024), kIdPU, 1);
@@ -564,7 +712,7 @@ __device__ __forceinline__ void mma_chain_role(const Ctx &x, const TcParams &p)
 // range: some half-chunk decays by more than 2^-120).  Rare, so it is kept out
 // of line; it reads its TMEM half row itself.
 template <int DIR>
-__device__ __noinline__ void m1_epi_direct(uint32_t taddr, const float *gt, float *As, uint32_t sP,
+__device__ __noinline__ void m1_epi_direct(uint32_t taddr, const float *gt, float *As, uint8_t *sP,
                                            int qd, int lane, int hf)
 {
     float xv[32];
@@ -633,6 +781,11 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
     auto compute_gates = [&](int j) {
         const int gj = j % kNG;
         float *gt = gates_buf(x, gj);
+#ifdef GDN_TRACE
+        const bool trg = p.prof && gpt == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 &&
+                         j >= kTrace0 && j < kTrace0 + kTraceN;
+        if (trg) p.prof[kTraceBase + (j - kTrace0) * 32 + 8] = (long long)clock64();
+#endif
         if (j >= kNG) wait_bar(&B.g_empty[gj], ((j / kNG) + 1) & 1, x.abort_flag, p.err, 2);
         float v = fmaxf(log2f(ra), -120.f);   // decay below 2^-120 acts as 2^-120
         const float bcur = rb;
@@ -680,6 +833,9 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
         }
         named_bar(kBarGates, 64);
         if (gpt == 0) mbar_arrive(&B.g_full[gj]);
+#ifdef GDN_TRACE
+        if (trg) p.prof[kTraceBase + (j - kTrace0) * 32 + 9] = (long long)clock64();
+#endif
     };
     load_raw(0);
     PROF_DECL(pt == 0);
@@ -694,6 +850,7 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
                          blockIdx.z == 0;
         if (i >= 0) {
             const bool fact = x.bars->gscal[gi][1] != 0.f;
+            PROF_SETC(i);
             PROF_MARK(16);
 
             // ---- masks: P (rows of QK^T) and A (rows of KK^T, scan order)
@@ -702,7 +859,7 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
             PROF_MARK(10);
             tc_fence_after();
             if (!fact) {
-                m1_epi_direct<DIR>(x.tmem + tm_lane + kColD1 + 32 * hf, gt, As, x.sbase + kOffP + b * 8192, qd,
+                m1_epi_direct<DIR>(x.tmem + tm_lane + kColD1 + 32 * hf, gt, As, x.smem + kOffP + b * 8192, qd,
                                    lane, hf);
             } else {
                 float xv[32];
@@ -722,7 +879,7 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
                         const bool keep = DIR ? (j >= r) : (j <= r);
                         xv[e] = keep ? rf * cf[e] * xv[e] : 0.f;
                     }
-                    store_half_row_bf16(x.sbase + kOffP + b * 8192, r, hf, xv);
+                    store_half_row_bf16(x.smem + kOffP + b * 8192, r, hf, xv);
                 } else {
                     // A row r, written in scan order: row lr, columns lj
                     const float rf = gt[gBet * 64 + r] * gt[(useB ? gRB : gRA) * 64 + r];
@@ -753,40 +910,14 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
             named_bar(kBarPrep, kPrepThreads);
             continue;
         }
-        solve_diag_blocks(As, pt);
-        PROF_MARK(13);
-        solve_off_diag(As, pt);
-        PROF_MARK(17);
-        if (dbg)
-            for (int e = pt; e < 64 * 64; e += kPrepThreads) {
-                const int rr = e >> 6, cc = e & 63;
-                p.debug[kDbgT + e] = (cc <= rr) ? As[rr * kLDA + cc] : 0.f;
-            }
-
-        // ---- T1 = T diag(b gamma), T2 = T diag(b), physical order; the
-        // products of chunk i-1 must be done with the previous T1, T2
+        // the products of chunk i-1 must be done with the previous T1, T2
         if (i >= 1) wait_bar(&B.wu_full, (i - 1) & 1, x.abort_flag, p.err, 6);
         tc_fence_after();
-        {
-            const int second = pt >> 7, r = (pt >> 1) & 63, h2 = pt & 1;
-            const int lr = DIR ? 63 - r : r;
-            // scan-order columns of physical half h2
-            const float4 *Trow = reinterpret_cast<const float4 *>(As + lr * kLDA + (DIR ? 32 * (1 - h2) : 32 * h2));
-            const float *sc = gt + (second ? gBet : gBG) * 64 + 32 * h2;
-            float xv[32];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float4 t4 = Trow[m];
-                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = DIR ? 31 - (4 * m + u) : 4 * m + u;
-                    const int lj = DIR ? 63 - (32 * h2 + e) : 32 * h2 + e;
-                    xv[e] = (lj <= lr) ? tv[u] * sc[e] : 0.f;    // upper triangle: zero
-                }
-            }
-            store_half_row_bf16(x.sbase + (second ? kOffT2 : kOffT1), r, h2, xv);
-        }
+        float *dbgT = dbg ? p.debug + kDbgT : nullptr;
+        solve_diag_blocks(As, gt, x.smem + kOffT1, x.smem + kOffT2, dbgT, DIR, pt);
+        PROF_MARK(13);
+        solve_off_diag(As, gt, x.smem + kOffT1, x.smem + kOffT2, dbgT, DIR, pt);
+        PROF_MARK(17);
         fence_proxy_async_smem();
         PROF_MARK(14);
         if (named_bar_any(kBarPrep, kPrepThreads, *x.abort_flag)) return;
@@ -799,10 +930,11 @@ __device__ __forceinline__ void prep_role(const Ctx &x, const TcParams &p, int p
 // ------------------------------------------------------------------ chain warps
 // 8 warps (256 threads).  Thread (warp cw, lane) owns state row
 // d = 32 * (cw & 3) + lane, columns [32 * (cw >> 2), +32) of the slice.
-// Per chunk i, in this order (so that the serial-chain products of chunk i can
-// start while the output tile of chunk i-1 is written):
-//   W and gamma*Q of chunk i  ->  output tile of chunk i-1  ->  U of chunk i
-//   ->  state update of chunk i.
+// Per chunk i, in this order, so that only the U and state epilogues sit on
+// the serial chain:
+//   U of chunk i  ->  W and gamma*Q of chunk i+1 (while K^T Ubar runs, when
+//   its inputs are ready; else before U of chunk i+1)  ->  state update of
+//   chunk i  ->  output tile of chunk i (while W H of chunk i+1 runs).
 template <int DIR>
 __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int ct)
 {
@@ -811,6 +943,8 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
     const uint32_t tm_lane = (uint32_t)(cq * 32) << 16;
     const int d = cq * 32 + lane;
     const int r = cq * 16 + lane;   // M=64 accumulators: lanes 0-15 of quarter cq hold rows 16 cq ..
+    const bool dbg0 = kDbgOn && p.debug != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+    int w_done = -1;   // last chunk whose W epilogue is done
 
     float h[32];
     {
@@ -822,12 +956,61 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
             const float4 v4 = s0 ? *reinterpret_cast<const float4 *>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
             h[e] = v4.x; h[e + 1] = v4.y; h[e + 2] = v4.z; h[e + 3] = v4.w;
         }
-        store_half_row_bf16(x.sbase + kOffH, d, chf, h);
+        store_half_row_bf16(x.smem + kOffH, d, chf, h);
     }
     fence_proxy_async_smem();
     named_bar(kBarChain, kChainThreads);
     if (ct == 0) mbar_arrive(&B.h_full);
     PROF_DECL(ct == 0);
+
+    // W (MN-major, row d = key index) and gamma-scaled Q of chunk j
+    auto w_epi = [&](int j) -> bool {
+        const int gj = j % kNG;
+        PROF_SETC(j);
+        wait_bar(&B.g_full[gj], (j / kNG) & 1, x.abort_flag, p.err, 7);
+        wait_bar(&B.wu_full, j & 1, x.abort_flag, p.err, 5);
+        PROF_MARK(26);
+        tc_fence_after();
+        {
+            float xv[32];
+            tmem_ld32(x.tmem + tm_lane + kColW + 32 * chf, xv);
+            tmem_wait_ld();
+            if (dbg0 && j == 0) {
+                dbg_half(p.debug + kDbgW, d, chf, xv);
+                float yv[32];
+                tmem_ld32(x.tmem + tm_lane + kColU0 + 32 * chf, yv);
+                tmem_wait_ld();
+                dbg_half(p.debug + kDbgUt, d, chf, yv);
+            }
+            store_half_row_bf16(x.smem + kOffW, d, chf, xv);
+        }
+        {
+            // gamma-scale Q in place (Q is no longer needed unscaled); bf16x2
+            // products: gamma is rounded to bf16 first, one more bf16 rounding
+            const int rq = ct >> 2, kb = (ct >> 1) & 1, part = ct & 1;
+            const __nv_bfloat162 g2 = __float2bfloat162_rn(gates_buf(x, gj)[gGam * 64 + rq]);
+            uint8_t *rowbase = x.smem + kOffStage + (uint32_t)(j % kNS) * kStageBytes + kb * 16384;
+            uint4 w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) w[q] = *reinterpret_cast<const uint4 *>(rowbase + sw128_off(rq, 8 * (4 * part + q)));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 *v = reinterpret_cast<__nv_bfloat162 *>(&w[q]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) v[u] = __hmul2(v[u], g2);
+                *reinterpret_cast<uint4 *>(rowbase + sw128_off(rq, 8 * (4 * part + q))) = w[q];
+            }
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        PROF_MARK(27);
+        if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return false;
+        if (ct == 0) {
+            mbar_arrive(&B.wmn_full);
+            mbar_arrive(&B.dw_empty);
+        }
+        return true;
+    };
 
     // output tile of chunk j: O = (gamma Q) H_prev + P U, from TMEM to o
     // (bidirectional: combined with the other direction's partial)
@@ -839,182 +1022,128 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
         float xv[32];
         tmem_ld32(x.tmem + tm_lane + kColO0 + 64 * bj + 32 * chf, xv);
         tmem_wait_ld();
-        if (kDbgOn && p.debug != nullptr && j == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-            dbg_half(p.debug + kDbgO, d, chf, xv);
+        if (dbg0 && j == 0) dbg_half(p.debug + kDbgO, d, chf, xv);
         const int t = c * kC + r;
         const bool mine = lane < 16 && t < x.T;
         __nv_bfloat16 *orow = p.o + ((size_t)x.bh * x.T + (mine ? t : 0)) * x.dv + x.slice * kDVS + 32 * chf;
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) w[e] = pack_bf16(xv[2 * e], xv[2 * e + 1]);
-        auto store_own = [&]() {
-            if (mine)
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        };
-        auto add_other = [&]() {
-            if (mine && !*x.abort_flag)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 o4 = __ldcg(reinterpret_cast<const uint4 *>(orow + 8 * q));
-                    const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
-                    uint32_t sw[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow[u]));
-                        sw[u] = pack_bf16(f.x + xv[8 * q + 2 * u], f.y + xv[8 * q + 2 * u + 1]);
-                    }
-                    *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-                }
-        };
-        // bounded wait (thread ct == 0) until the counter reaches `target`
-        auto wait_count = [&](int *cnt, int target) {
-            if (ct == 0) {
-                const unsigned long long t0 = globaltimer();
-                int seen = 0;
-                for (uint32_t it = 0; it < (1u << 30); ++it) {
-                    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(cnt) : "memory");
-                    if (seen >= target) break;
-                    if ((it & 255) == 255 && globaltimer() - t0 > kWaitLimitNs) break;
-                }
-                if (seen < target) {
-                    atomicOr(p.err, 32);
-                    *x.abort_flag = 1;
-                }
-            }
-        };
-        // causal: this CTA writes the tile.  Bidirectional: the direction
-        // that reaches the tile first writes its partial and counts it; the
-        // second waits for that count and adds its own partial.
-        bool first = true;
-        int *cnt = nullptr, target = 1;
+        // causal: this CTA writes the tile.  Bidirectional: the direction that
+        // reaches the tile first writes its partial, the second adds its own.
+        bool first = true, add = false;
         if (p.counters != nullptr) {
-            cnt = p.counters + ((size_t)x.bh * x.NC + c) * p.n_slices + x.slice;
+            int *cnt = p.counters + ((size_t)x.bh * x.NC + c) * p.n_slices + x.slice;
             if (p.predict) {
                 // every CTA is resident: the forward scan reaches the first
-                // half of the chunks first, the reverse scan the second half
+                // half of the chunks first, the reverse scan the second half.
+                // The combine warp counts and checks the partials; here the
+                // second writer only waits (in shared memory) for its word.
                 first = DIR == ((2 * c < x.NC) ? 0 : 1);
+                if (!first) add = wait_smem_at_least(&B.ready_upto, j, x.abort_flag, p.err, 33);
             } else {
                 // arrival order decided at run time by a claim on the counter
-                // (0 -> 1 -> 2), the partial's arrival brings it to 3
+                // (0 -> 1 -> 2); the partial's arrival brings it to 3
                 if (ct == 0) x.bars->s_old = atomicAdd(cnt, 1);
                 named_bar(kBarChain, kChainThreads);
                 first = x.bars->s_old == 0;
-                target = 3;
+                if (first) {
+                    if (mine)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            *reinterpret_cast<uint4 *>(orow + 8 * q) =
+                                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                    named_bar(kBarChain, kChainThreads);
+                    if (ct == 0) {
+                        __threadfence();
+                        atomicAdd(cnt, 1);
+                    }
+                } else {
+                    if (ct == 0 && !spin_global_at_least(cnt, 3, x.abort_flag)) {
+                        atomicOr(p.err, 32);
+                        *x.abort_flag = 1;
+                    }
+                    named_bar(kBarChain, kChainThreads);
+                    add = !*x.abort_flag;
+                }
+                first = false;   // stored above, or added below
             }
         }
-        if (first) {
-            store_own();
-            if (cnt != nullptr) {
-                named_bar(kBarChain, kChainThreads);
-                if (ct == 0) {
-                    __threadfence();
-                    atomicAdd(cnt, 1);
-                }
+        if (mine) {
+            if (first) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            } else if (add) {
+                // bf16 add in L2: the partials are rounded to bf16 on each side
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    red_add_bf16x8(orow + 8 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
             }
-        } else {
-            wait_count(cnt, target);
-            named_bar(kBarChain, kChainThreads);
-            add_other();
         }
         tc_fence_before();
         PROF_MARK(25);
         if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return false;
-        if (ct == 0) mbar_arrive(&B.do_empty[bj]);
+        if (ct == 0) {
+            mbar_arrive(&B.do_empty[bj]);
+            // predicted first writer: the tile is stored; the combine warp
+            // makes it visible to the other direction and counts it
+            if (p.counters != nullptr && p.predict && first) st_release_cta(&B.stored_upto, j);
+        }
         return true;
     };
 
 #pragma unroll 1
-    for (int i = 0; i <= x.NC; ++i) {
-        const int b = i & 1, c = chunk_of<DIR>(x, i), gi = i % kNG;
+    for (int i = 0; i < x.NC; ++i) {
+        const int b = i & 1, gi = i % kNG;
         const float *gt = gates_buf(x, gi);
-        const bool dbg = kDbgOn && p.debug != nullptr && i == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
-                         blockIdx.z == 0;
-        if (i < x.NC) {
-            // ---- W (MN-major, row d = key index) and gamma-scaled Q of chunk i
-            wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 7);
-            wait_bar(&B.wu_full, i & 1, x.abort_flag, p.err, 5);
-            PROF_MARK(26);
+        const bool dbg = dbg0 && i == 0;
+        PROF_SETC(i);
+        PROF_MARK(19);
+
+        // s = 0: the W epilogue of chunk i unless it ran early, then U of i;
+        // s = 1: the W epilogue of chunk i+1 if its inputs are ready now
+#pragma unroll 1
+        for (int s = 0; s < 2; ++s) {
+            const int j = i + s;
+            bool run_w = j < x.NC && w_done < j;
+            if (s == 1 && run_w) {
+                const bool ready = mbar_test_wait(&B.g_full[j % kNG], (j / kNG) & 1) &&
+                                   mbar_test_wait(&B.wu_full, j & 1);
+                run_w = !named_bar_any(kBarChain, kChainThreads, !ready);
+            }
+            if (run_w) {
+                if (!w_epi(j)) return;
+                w_done = j;
+                PROF_SETC(i);
+            }
+            if (s == 1) break;
+
+            // ---- U and Ubar rows of chunk i
+            wait_bar(&B.chain_full, i & 1, x.abort_flag, p.err, 8);
+            PROF_MARK(20);
             tc_fence_after();
             {
                 float xv[32];
-                tmem_ld32(x.tmem + tm_lane + kColW + 32 * chf, xv);
+                tmem_ld32(x.tmem + tm_lane + kColU0 + 64 * b + 32 * chf, xv);
                 tmem_wait_ld();
-                if (dbg) {
-                    dbg_half(p.debug + kDbgW, d, chf, xv);
-                    float yv[32];
-                    tmem_ld32(x.tmem + tm_lane + kColU0 + 64 * b + 32 * chf, yv);
-                    tmem_wait_ld();
-                    dbg_half(p.debug + kDbgUt, d, chf, yv);
-                }
-                store_half_row_bf16(x.sbase + kOffW, d, chf, xv);
-            }
-            {
-                // gamma-scale Q in place (Q is no longer needed unscaled); bf16x2
-                // products: gamma is rounded to bf16 first, one more bf16 rounding
-                const int rq = ct >> 2, kb = (ct >> 1) & 1, part = ct & 1;
-                const __nv_bfloat162 g2 = __float2bfloat162_rn(gt[gGam * 64 + rq]);
-                const uint32_t rowbase = stage_addr(x, i) + kb * 16384;
-                uint32_t w[4][4];
-    #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(w[q][0]), "=r"(w[q][1]), "=r"(w[q][2]), "=r"(w[q][3])
-                                 : "r"(rowbase + sw128_off(rq, 8 * (4 * part + q))));
-    #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-    #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        __nv_bfloat162 v = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&w[q][u]), g2);
-                        w[q][u] = *reinterpret_cast<uint32_t *>(&v);
-                    }
-                    st_shared_v4(rowbase + sw128_off(rq, 8 * (4 * part + q)), w[q][0], w[q][1], w[q][2], w[q][3]);
+                if (dbg) dbg_half(p.debug + kDbgU, d, chf, xv);
+                if (lane < 16) {
+                    store_half_row_bf16(x.smem + kOffU, r, chf, xv);
+                    const float eb = gt[gEb * 64 + r];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) xv[e] *= eb;
+                    store_half_row_bf16(x.smem + kOffUb, r, chf, xv);
                 }
             }
             tc_fence_before();
             fence_proxy_async_smem();
-            PROF_MARK(27);
+            PROF_MARK(21);
             if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return;
             if (ct == 0) {
-                mbar_arrive(&B.wmn_full);
-                mbar_arrive(&B.dw_empty);
+                mbar_arrive(&B.u_full);
+                mbar_arrive(&B.du_empty[b]);
             }
-        }
-
-        // ---- output tile of the previous chunk (overlaps this chunk's products)
-        if (i > 0 && !out_tile(i - 1)) return;
-        if (i == x.NC) break;
-
-        // ---- U and Ubar rows of chunk i
-        wait_bar(&B.chain_full, i & 1, x.abort_flag, p.err, 8);
-        PROF_MARK(20);
-        tc_fence_after();
-        {
-            float xv[32];
-            tmem_ld32(x.tmem + tm_lane + kColU0 + 64 * b + 32 * chf, xv);
-            tmem_wait_ld();
-            if (dbg) dbg_half(p.debug + kDbgU, d, chf, xv);
-            if (lane < 16) {
-                store_half_row_bf16(x.sbase + kOffU, r, chf, xv);
-                const float eb = gt[gEb * 64 + r];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) xv[e] *= eb;
-                store_half_row_bf16(x.sbase + kOffUb, r, chf, xv);
-                // bidirectional, second direction for this tile: pull the other
-                // direction's partial into L2 ahead of the output step
-                const int t = c * kC + r;
-                if (p.counters != nullptr && p.predict && t < x.T && DIR != ((2 * c < x.NC) ? 0 : 1))
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + ((size_t)x.bh * x.T + t) * x.dv + x.slice * kDVS + 32 * chf));
-            }
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        PROF_MARK(21);
-        if (named_bar_any(kBarChain, kChainThreads, *x.abort_flag)) return;
-        if (ct == 0) {
-            mbar_arrive(&B.u_full);
-            mbar_arrive(&B.du_empty[b]);
         }
 
         // ---- state update (fp32 registers) and its bf16 copy
@@ -1029,7 +1158,7 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
             const float ge = exp2f(x.bars->gscal[gi][0]);
 #pragma unroll
             for (int e = 0; e < 32; ++e) h[e] = fmaf(ge, h[e], xv[e]);
-            store_half_row_bf16(x.sbase + kOffH, d, chf, h);
+            store_half_row_bf16(x.smem + kOffH, d, chf, h);
         }
         tc_fence_before();
         fence_proxy_async_smem();
@@ -1039,6 +1168,9 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
             mbar_arrive(&B.h_full);
             mbar_arrive(&B.g_empty[gi]);
         }
+
+        // ---- output tile of chunk i (overlaps the next chunk's W H)
+        if (!out_tile(i)) return;
     }
     PROF_FLUSH();
 
@@ -1047,6 +1179,36 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4 *>(so + e) = make_float4(h[e], h[e + 1], h[e + 2], h[e + 3]);
+    }
+}
+
+// ------------------------------------------------------------------ combine warp
+// Bidirectional launches whose CTAs are all resident (the first writer of each
+// output tile is known in advance): one thread takes the grid-wide handshake
+// of each tile off the chain warps.  For a tile this CTA writes first it waits
+// until the chain warps have stored it, then makes the stores visible device-
+// wide and bumps the tile's counter; for a tile it writes second it waits for
+// the other direction's count and then releases the chain warps to add.
+template <int DIR>
+__device__ __forceinline__ void combine_role(const Ctx &x, const TcParams &p)
+{
+    if (p.counters == nullptr || !p.predict) return;
+    Bars &B = *x.bars;
+    for (int i = 0; i < x.NC; ++i) {
+        const int c = chunk_of<DIR>(x, i);
+        int *cnt = p.counters + ((size_t)x.bh * x.NC + c) * p.n_slices + x.slice;
+        if (DIR == ((2 * c < x.NC) ? 0 : 1)) {
+            if (!wait_smem_at_least(&B.stored_upto, i, x.abort_flag, p.err, 34)) return;
+            __threadfence();
+            atomicAdd(cnt, 1);
+        } else {
+            if (!spin_global_at_least(cnt, 1, x.abort_flag)) {
+                if (!*x.abort_flag) atomicOr(p.err, 32);
+                *x.abort_flag = 1;
+                return;
+            }
+            st_release_cta(&B.ready_upto, i);
+        }
     }
 }
 
@@ -1078,6 +1240,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int nbar = (int)(offsetof(Bars, gscal) / sizeof(uint64_t));
         for (int k = 0; k < nbar; ++k) mbar_init(&all[k], 1);
         B.abort_flag = 0;
+        B.stored_upto = -1;
+        B.ready_upto = -1;
         fence_mbar_init();
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
@@ -1089,6 +1253,9 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     float *As0 = reinterpret_cast<float *>(smem + kOffA);
     for (int i = tid; i < 64 * kLDA; i += kThreads) As0[i] = 0.f;
+    // T1, T2: the upper triangle stays zero for the whole scan
+    uint32_t *T12 = reinterpret_cast<uint32_t *>(smem + kOffT1);
+    for (int i = tid; i < 16384 / 4; i += kThreads) T12[i] = 0u;
     if (tid < 32) reinterpret_cast<long long *>(smem + kOffProf)[tid] = 0;
 #ifdef GDN_PROFILE
     const unsigned long long prof_start = globaltimer();
@@ -1111,8 +1278,13 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
     } else if (warp == 17) {
         if (lane == 0) mma_prep_role(x, p);
-    } else {
+    } else if (warp == 18) {
         if (lane == 0) mma_chain_role(x, p);
+    } else {
+        if (lane == 0) {
+            if (x.dir) combine_role<1>(x, p);
+            else combine_role<0>(x, p);
+        }
     }
 
     tc_fence_before();

@@ -96,6 +96,15 @@ def test_bf16_fast_decay(oracle_mod, kernel):
     check(oracle_mod, inp, True, recurrent=(kernel == "recurrent"))
 
 
+@pytest.mark.parametrize("dv", [64, 128])
+def test_bf16_bidi_more_ctas_than_sms(oracle_mod, dv):
+    """160 CTAs (more than the 148 SMs): the order in which the two scans reach
+    an output tile is decided at run time instead of in advance."""
+    heads = 160 // (2 * (dv // 64))
+    inp = make_custom(1, heads, 333, 128, dv, dtype="bf16", seed=11 + dv, bidi=True)
+    check(oracle_mod, inp, True, recurrent=False)
+
+
 @pytest.mark.parametrize("kernel", BF16_KERNELS)
 def test_bf16_no_decay_unit_gates(oracle_mod, kernel):
     """a = 1, b = 1: the pure delta rule, the hardest case for carried error."""
