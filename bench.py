@@ -27,6 +27,7 @@ there is no upstream code to run).
 import argparse
 import ctypes
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -71,11 +72,16 @@ def load_peaks():
 
 
 def kernel_source_sha():
+    """Hash of the kernel sources' code (comments and whitespace removed), so
+    that a recorded traffic figure stays tied to the code it was taken on."""
     h = hashlib.sha256()
     for name in ("gdn_chunk_tc.cu", "gdn_recurrent.cu", "sm100_ptx.cuh", "gdn_internal.h"):
         p = os.path.join(ROOT, "gated_delta_rule_149_b200", "csrc", name)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            src = open(p).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            src = re.sub(r"//[^\n]*", "", src)
+            h.update("".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

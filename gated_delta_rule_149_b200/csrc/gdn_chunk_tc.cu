@@ -23,16 +23,18 @@
 // more than 2^-240 (a factor could leave the normal range) it is formed
 // directly, so nothing overflows however strong the decay.
 //
-// One CTA per (64-wide dv slice, direction, batch*head), 19 warps:
+// One CTA per (64-wide dv slice, direction, batch*head), 20 warps:
 //   warps 0-7   chain: fp32 state in registers (each thread owns 32 columns
-//                      of one row of the dk x 64 slice); U, state and output
-//                      epilogues;
+//                      of one row of the dk x 64 slice); W and gamma*Q
+//                      operands, U, state and output epilogues;
 //   warps 8-15  prep:  gates, masks, the triangular solve (16x16 diagonal
-//                      blocks by substitution, the rest with tf32 mma.sync),
-//                      T1 = T diag(b gamma), T2 = T diag(b), gamma*Q, W;
+//                      blocks by substitution, the blocks below by strip-wise
+//                      block substitution with tf32 mma.sync), written straight
+//                      into T1 = T diag(b gamma) and T2 = T diag(b);
 //   warp 16     TMA:   q, k and the v slice of each chunk, three stages ahead;
 //   warp 17     MMA:   issues the state-independent products ([Q;K]K^T, W, U~);
-//   warp 18     MMA:   issues the serial-chain products (W H, Q H, K^T Ubar, P U).
+//   warp 18     MMA:   issues the serial-chain products (W H, Q H, K^T Ubar, P U);
+//   warp 19     combine: the grid-wide handshake of the bidirectional tiles.
 // Tensor-core products (bf16 operands, fp32 accumulation in TMEM):
 //     [Q;K] K^T        M=128 N=64  K=dk     -> QK^T, KK^T
 //     W^T = K^T T1^T   M=128 N=64  K=64
@@ -41,8 +43,8 @@
 //     O   = (gamma Q) H, O += P U           M=64 N=64
 //     D_S = K^T Ubar   M=128 N=64  K=64     (Ubar = diag(2^(G_end-G)) U)
 // Bidirectional: both scans run in the same launch; for each (head, chunk,
-// slice) output tile the first finisher writes its partial and the second
-// adds its own and writes the sum (an arrival counter decides who is who).
+// slice) output tile the first writer stores its partial and the second adds
+// its own in L2 once an arrival counter shows the first is visible.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
