@@ -274,7 +274,8 @@ def run_reference(args, world, rank):
 
 def run_gpu(args, world, rank, local):
     import torch
-    from gated_delta_rule_149_b200 import gdn, gdn_forward, gdn_forward_host, gdn_device_status
+    from gated_delta_rule_149_b200 import (gdn, gdn_forward, gdn_forward_host, gdn_forward_segmented,
+                                           gdn_device_status)
     from gated_delta_rule_149_b200.inputs import WORKLOADS, make_inputs
 
     wl = WORKLOADS[args.workload]
@@ -291,9 +292,17 @@ def run_gpu(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     lib = gdn.load_library()
 
+    segmented = args.segments > 0
+    if segmented and (wl.bidi or recurrent):
+        raise SystemExit("--segments runs causal bf16 workloads only")
+
     def step():
-        gdn_forward(q, k, v, beta, decay, s0, bidi=wl.bidi, recurrent=recurrent, o=o,
-                    state_out=s_out, stream=stream)
+        if segmented:
+            gdn_forward_segmented(q, k, v, beta, decay, s0, n_segments=args.segments, o=o,
+                                  state_out=s_out, stream=stream)
+        else:
+            gdn_forward(q, k, v, beta, decay, s0, bidi=wl.bidi, recurrent=recurrent, o=o,
+                        state_out=s_out, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -352,8 +361,16 @@ def run_gpu(args, world, rank, local):
     hso = torch.empty(s_out.shape, dtype=torch.float32).pin_memory()
 
     def e2e_step():
-        gdn_forward_host(hq, hk, hv, hb, ha, hs0, bidi=wl.bidi, recurrent=recurrent, o=ho,
-                         state_out=hso, stream=stream)
+        if segmented:   # the same call on device copies of pinned host buffers
+            for h, dst in ((hq, q), (hk, k), (hv, v), (hb, beta), (ha, decay), (hs0, s0)):
+                if h is not None:
+                    dst.copy_(h, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hso.copy_(s_out, non_blocking=True)
+        else:
+            gdn_forward_host(hq, hk, hv, hb, ha, hs0, bidi=wl.bidi, recurrent=recurrent, o=ho,
+                             state_out=hso, stream=stream)
 
     e2e_steps = max(1, min(args.steps, 5))
     e2e_step()
@@ -374,7 +391,8 @@ def run_gpu(args, world, rank, local):
             "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk,
                        "dv": wl.dv, "mode": "bidi" if wl.bidi else "causal",
-                       "kernel": "recurrent" if recurrent else "chunk_tc",
+                       "kernel": ("recurrent" if recurrent else
+                                  f"chunk_tc, segment-parallel x{args.segments}" if segmented else "chunk_tc"),
                        "token_heads_per_gpu": wl.token_heads,
                        "l2": ("no flush: inputs of %.2f GB per step exceed the 126 MB L2" % (bytes_ / 1e9)
                               if flush_buf is None else
@@ -404,6 +422,8 @@ def main():
     ap.add_argument("--recurrent", action="store_true",
                     help="time the token-by-token SIMT kernel instead of the chunkwise one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="causal workloads: run the segment-parallel scan with this many segments")
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="seconds of CPU work per oracle sample (default 15; 8 for --impl reference)")
     args = ap.parse_args()

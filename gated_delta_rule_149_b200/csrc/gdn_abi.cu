@@ -263,6 +263,38 @@ int gdn_forward_noalloc(const void *q, const void *k, const void *v, const float
     }
 }
 
+int gdn_forward_segmented(const void *q, const void *k, const void *v, const float *beta,
+                          const float *decay, const float *state_in, float *state_out, void *o,
+                          int B, int H, int T, int dk, int dv, int n_segments, int mode,
+                          void *stream)
+{
+    try {
+        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                              mode, "T");
+        if (rc != GDN_OK) return rc;
+        if (n_segments < 1) return fail(GDN_ERR_INVALID_ARG, "n_segments must be >= 1 (got %d)", n_segments);
+        if (mode & (GDN_BIDI | GDN_FP32 | GDN_RECURRENT))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_segmented is causal and runs the bf16 chunkwise kernel only "
+                        "(no GDN_BIDI / GDN_FP32 / GDN_RECURRENT)");
+        gdn::FwdArgs a = make_args(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                                   mode);
+        if (!gdn::chunk_tc_supported(a))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_segmented needs dk = 128 and dv in {64, 128} (got dk=%d, dv=%d)",
+                        dk, dv);
+        int seg_chunks = 0;
+        const int S = gdn::segment_count(T, n_segments, &seg_chunks);
+        if ((long long)B * H * S > 65535)
+            return fail(GDN_ERR_UNSUPPORTED, "B*H*segments = %lld exceeds 65535", (long long)B * H * S);
+        cudaError_t err = gdn::launch_segmented(a, n_segments, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return fail(GDN_ERR_CUDA, "launch failed: %s", cudaGetErrorString(err));
+        return ok();
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in gdn_forward_segmented");
+    }
+}
+
 int gdn_device_status(void *stream)
 {
     int err = 0;

@@ -128,6 +128,7 @@ struct TcParams {
     float *debug;        // optional: first-chunk intermediates of CTA (0,0,0)
     long long *prof;     // optional (profiling builds): per-phase cycle counts of CTA (0,0,0)
     int BH, T, dv, n_chunks, n_slices;
+    int n_seg, seg0, seg_chunks;   // segments of each head in this launch (1, 0, n_chunks: whole)
     int predict;         // bidi: all CTAs resident, first writer of each tile known in advance
 };
 
@@ -544,11 +545,13 @@ struct Ctx {
     volatile int *abort_flag;
     uint32_t tmem;
     int slice, dir, bh, NC, T, dv;
+    int row;   // state row (head, segment): blockIdx.z
+    int c0;    // first (global) chunk of this CTA's segment
 };
 
 __device__ __forceinline__ uint32_t stage_addr(const Ctx &x, int i) { return x.sbase + kOffStage + (uint32_t)(i % kNS) * kStageBytes; }
 template <int DIR>
-__device__ __forceinline__ int chunk_of(const Ctx &x, int i) { return DIR ? (x.NC - 1 - i) : i; }
+__device__ __forceinline__ int chunk_of(const Ctx &x, int i) { return x.c0 + (DIR ? (x.NC - 1 - i) : i); }
 __device__ __forceinline__ float *gates_buf(const Ctx &x, int g) { return reinterpret_cast<float *>(x.smem + kOffGates) + g * kGateFloats; }
 
 // ------------------------------------------------------------------ TMA warp
@@ -951,7 +954,7 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
     float h[32];
     {
         const float *s0 = (DIR == 0 && p.state_in)
-                              ? p.state_in + ((size_t)x.bh * kDK + d) * x.dv + x.slice * kDVS + 32 * chf
+                              ? p.state_in + ((size_t)x.row * kDK + d) * x.dv + x.slice * kDVS + 32 * chf
                               : nullptr;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -1177,7 +1180,7 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
     PROF_FLUSH();
 
     if (p.state_out) {
-        float *so = p.state_out + (((size_t)DIR * p.BH + x.bh) * kDK + d) * x.dv + x.slice * kDVS + 32 * chf;
+        float *so = p.state_out + (((size_t)DIR * gridDim.z + x.row) * kDK + d) * x.dv + x.slice * kDVS + 32 * chf;
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4 *>(so + e) = make_float4(h[e], h[e + 1], h[e + 2], h[e + 3]);
@@ -1231,9 +1234,11 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     x.abort_flag = &x.bars->abort_flag;
     x.slice = blockIdx.x;
     x.dir = blockIdx.y;
-    x.bh = blockIdx.z;
+    x.row = blockIdx.z;
+    x.bh = blockIdx.z / p.n_seg;
+    x.c0 = (p.seg0 + blockIdx.z % p.n_seg) * p.seg_chunks;
     x.T = p.T;
-    x.NC = p.n_chunks;
+    x.NC = min(p.seg_chunks, p.n_chunks - x.c0);   // >= 1: the host launches no empty segment
     x.dv = p.dv;
     Bars &B = *x.bars;
 
@@ -1339,6 +1344,22 @@ bool make_map(CUtensorMap *m, const void *base, int inner, int T, int BH)
     return r == CUDA_SUCCESS;
 }
 
+// The kernel's dynamic shared-memory size, set once per device.
+cudaError_t set_smem_attribute()
+{
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+    err = cudaFuncSetAttribute(gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSmemAlloc);
+    if (err == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+    return err;
+}
+
 // Whether every CTA of the grid is resident at once (one CTA per SM, as the
 // shared-memory footprint forces), so that each bidirectional output tile's
 // first writer can be fixed in advance.
@@ -1375,16 +1396,22 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
     p.BH = BH; p.T = a.T; p.dv = a.dv;
     p.n_chunks = (a.T + kC - 1) / kC;
     p.n_slices = a.dv / kDVS;
+    p.n_seg = a.n_seg;
+    p.seg0 = a.seg0;
+    p.seg_chunks = a.seg_chunks > 0 ? a.seg_chunks : p.n_chunks;
     p.counters = nullptr;
     p.debug = g_debug_dump;
     p.prof = g_prof_buf;
     cudaError_t err = device_error_word(&p.err);
     if (err != cudaSuccess) return err;
+    if (a.bidi && (a.n_seg != 1 || p.seg_chunks != p.n_chunks)) return cudaErrorInvalidValue;
+    if (a.n_seg < 1 || (size_t)BH * a.n_seg > 65535 ||
+        (a.seg0 + a.n_seg - 1) * (size_t)p.seg_chunks >= (size_t)p.n_chunks)
+        return cudaErrorInvalidValue;   // every launched segment holds at least one chunk
     err = all_resident(BH * (a.bidi ? 2 : 1) * p.n_slices, &p.predict);
     if (err != cudaSuccess) return err;
 
-    err = cudaFuncSetAttribute(gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kSmemAlloc);
+    err = set_smem_attribute();
     if (err != cudaSuccess) return err;
     const size_t n_cnt = (size_t)BH * p.n_chunks * p.n_slices;
     if (a.bidi) {
@@ -1393,7 +1420,7 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
         err = cudaMemsetAsync(p.counters, 0, n_cnt * sizeof(int), stream);
     }
     if (err == cudaSuccess) {
-        dim3 grid(p.n_slices, a.bidi ? 2 : 1, BH);
+        dim3 grid(p.n_slices, a.bidi ? 2 : 1, BH * a.n_seg);
         gdn_chunk_tc_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, p);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
@@ -1442,6 +1469,9 @@ cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream)
     p.BH = BH; p.T = a.T; p.dv = a.dv;
     p.n_chunks = (a.T + kC - 1) / kC;
     p.n_slices = a.dv / kDVS;
+    p.n_seg = 1;
+    p.seg0 = 0;
+    p.seg_chunks = p.n_chunks;
     p.counters = nullptr;
     p.debug = nullptr;
     p.prof = nullptr;
@@ -1449,8 +1479,7 @@ cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream)
     if (err != cudaSuccess) return err;
     err = all_resident(BH * (a.bidi ? 2 : 1) * p.n_slices, &p.predict);
     if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kSmemAlloc);
+    err = set_smem_attribute();
     if (err != cudaSuccess) return err;
 
     if (a.bidi) {

@@ -16,6 +16,12 @@ struct FwdArgs {
     int B, H, T, dk, dv;
     bool bidi;
     bool fp32;                // q/k/v/o dtype: fp32 (else bf16)
+    // Segments (chunkwise kernel, causal only): the launch runs n_seg
+    // consecutive segments seg0 .. seg0 + n_seg - 1 of seg_chunks 64-token
+    // chunks of every head (the last one may be shorter); state_in/state_out
+    // then hold one [dk][dv] state per (head, segment), head-major.
+    // seg_chunks = 0: one segment, the whole sequence.
+    int seg0 = 0, n_seg = 1, seg_chunks = 0;
 };
 
 // Token-by-token fp32 SIMT kernel (any dtype; dk, dv multiples of 32, <= 128).
@@ -29,6 +35,13 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream);
 // counters come from a fixed static device array of noalloc_capacity() ints.
 size_t noalloc_capacity();
 cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream);
+
+// Segment-parallel causal scan (chunkwise kernel): splits each head's sequence
+// into about n_segments whole-chunk segments, runs them in parallel and threads
+// the state through them (three kernel passes and a combine).  segment_count
+// returns the number of segments used and their length in chunks.
+int segment_count(int T, int n_segments, int *seg_chunks);
+cudaError_t launch_segmented(const FwdArgs &a, int n_segments, cudaStream_t stream);
 
 // Device-side error word (set by bounded waits that gave up).
 cudaError_t device_error_word(int **ptr);

@@ -143,6 +143,34 @@ int gdn_forward_noalloc(const void *q, const void *k, const void *v,
                         int B, int H, int T, int dk, int dv, int mode, void *stream);
 
 /*
+ * gdn_forward_segmented -- causal gdn_forward with each head's sequence split
+ * along time into segments that run in parallel (the segment-parallel scan
+ * for streaming calls with few heads: flashdreams SANA-WM page, chunk-causal
+ * streaming, where the per-chunk latency is what matters, and LongSANA's
+ * causal KV cache).
+ *
+ * Same arguments, layouts and results as gdn_forward with mode GDN_CAUSAL
+ * (bf16 inputs, dk = 128, dv in {64, 128}), up to rounding: the state is
+ * affine in its initial value, so each segment's transition
+ * P = prod a_t (I - b_t k_t k_t^T) and its zero-start final state L are
+ * computed in parallel, the states entering the segments follow from
+ * E_{p+1} = P_p E_p + L_p (fp32), and the segments are rerun from them.
+ * `n_segments` is the requested number of segments (>= 1); segments are whole
+ * 64-token chunks (the last may be shorter), and with fewer than three the
+ * call is a plain gdn_forward.  Costs about three times the arithmetic of one
+ * scan for a chain about 3/n_segments as long; worth it when B*H*2*(dv/64)
+ * CTAs leave most of the GPU idle.  Workspace (stream-ordered): about
+ * 4 B*H*n_segments*dk*dv*4 + 2 B*H*n_segments*dk*dk*4 + 4 B*H*T*dk bytes.
+ * Errors: as gdn_forward; GDN_BIDI, GDN_FP32 or GDN_RECURRENT return
+ * GDN_ERR_UNSUPPORTED, n_segments < 1 returns GDN_ERR_INVALID_ARG.
+ */
+int gdn_forward_segmented(const void *q, const void *k, const void *v,
+                          const float *beta, const float *decay,
+                          const float *state_in, float *state_out, void *o,
+                          int B, int H, int T, int dk, int dv, int n_segments, int mode,
+                          void *stream);
+
+/*
  * gdn_device_status -- synchronises `stream` and reports (and clears) the
  * library's device-side error word: GDN_OK, or GDN_ERR_DEVICE_TIMEOUT if a
  * bounded wait inside a kernel gave up since the last call, or GDN_ERR_CUDA.

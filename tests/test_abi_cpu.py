@@ -27,7 +27,7 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_forward_noalloc",
-              "gdn_device_status", "gdn_kernel_launches",
+              "gdn_forward_segmented", "gdn_device_status", "gdn_kernel_launches",
               "gdn_last_error", "gdn_version"):
         assert n in names
 
@@ -112,3 +112,19 @@ def test_noalloc_rejects_before_launch(lib):
     assert f(mode=1 | 4) == -2                          # recurrent kernel
     assert f(dk=64) == -2
     assert f(T=0) == -1
+
+
+def test_segmented_rejects_before_launch(lib):
+    """The segment-parallel entry point is causal, bf16 chunkwise only, and
+    needs at least one segment; each refusal happens before any CUDA call."""
+    f = lambda T=640, dk=128, dv=128, nseg=4, mode=0: lib.gdn_forward_segmented(
+        P, P, P, P, P, None, None, P, 1, 1, T, dk, dv, nseg, mode, None)
+    assert f(nseg=0) == -1 and b"n_segments" in lib.gdn_last_error()
+    assert f(mode=1) == -2                               # bidirectional
+    assert f(mode=2) == -2                               # fp32
+    assert f(mode=4) == -2                               # recurrent kernel
+    assert f(dk=64) == -2
+    assert f(dv=96) == -2
+    assert f(T=0) == -1
+    assert lib.gdn_forward_segmented(P, P, P, P, P, None, None, P, 1, 64, 64 * 4000, 128, 128, 2000, 0,
+                                     None) == -2         # B*H*segments > 65535

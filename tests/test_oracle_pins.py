@@ -15,6 +15,7 @@ by closed forms and brute force instead:
   exact rational evaluation of the definition;
 * bidirectional = forward + re-reversed forward on the reversed sequence;
 * a rollout split at arbitrary points = one scan (bitwise);
+* the final state is affine in the initial one (the segment transition);
 * the contraction bound ||H_t|| <= a_t ||H_{t-1}|| + b_t ||v_t|| for unit keys.
 Each pin is chosen so that a dropped term, a wrong sign or index, or a
 transposed state would fail at least one of them.
@@ -246,6 +247,29 @@ def test_split_scan_equals_single_scan_bitwise(oracle_mod, cuts):
         pieces.append(o)
     assert np.array_equal(np.concatenate(pieces, axis=2), o_full)
     assert np.array_equal(state, s_full)
+
+
+def test_state_is_affine_in_the_initial_state(oracle_mod):
+    """The segment-parallel scan rests on this: a segment's final state is
+    P X + L for any initial state X, where P = prod_t a_t (I - b_t k_t k_t^T)
+    (later tokens on the left) is the final state of the same segment run with
+    v = 0 from the identity, and L its final state from zero."""
+    T, dk, dv = 60, 6, 5
+    q = RNG.standard_normal((T, dk))
+    k = rand_unit(T, dk)
+    v = RNG.standard_normal((T, dv))
+    a = RNG.uniform(0.5, 1.0, T)
+    b = RNG.uniform(0.0, 1.0, T)
+    _, P = oracle_mod.gdn_forward(batch(q), batch(k), batch(np.zeros((T, dk))), batch(b), batch(a),
+                                  state_in=batch(np.eye(dk)))
+    P_ref = np.eye(dk)
+    for t in range(T):
+        P_ref = a[t] * (np.eye(dk) - b[t] * np.outer(k[t], k[t])) @ P_ref
+    np.testing.assert_allclose(P[0, 0], P_ref, rtol=1e-12, atol=1e-14)
+    _, L = oracle_mod.gdn_forward(batch(q), batch(k), batch(v), batch(b), batch(a))
+    X = RNG.standard_normal((dk, dv))
+    _, F = oracle_mod.gdn_forward(batch(q), batch(k), batch(v), batch(b), batch(a), state_in=batch(X))
+    np.testing.assert_allclose(F[0, 0], P_ref @ X + L[0, 0], rtol=1e-11, atol=1e-13)
 
 
 def test_rollout_entry_equals_single_scan_bitwise(oracle_mod):
