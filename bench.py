@@ -274,8 +274,8 @@ def run_reference(args, world, rank):
 
 def run_gpu(args, world, rank, local):
     import torch
-    from gated_delta_rule_149_b200 import (gdn, gdn_forward, gdn_forward_host, gdn_forward_segmented,
-                                           gdn_device_status)
+    from gated_delta_rule_149_b200 import (gdn, gdn_forward, gdn_forward_blockcausal, gdn_forward_host,
+                                           gdn_forward_segmented, gdn_device_status)
     from gated_delta_rule_149_b200.inputs import WORKLOADS, make_inputs
 
     wl = WORKLOADS[args.workload]
@@ -292,12 +292,15 @@ def run_gpu(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     lib = gdn.load_library()
 
-    segmented = args.segments > 0
+    segmented = args.segments > 0 or args.block > 0
     if segmented and (wl.bidi or recurrent):
-        raise SystemExit("--segments runs causal bf16 workloads only")
+        raise SystemExit("--segments / --block run causal bf16 workloads only")
 
     def step():
-        if segmented:
+        if args.block > 0:
+            gdn_forward_blockcausal(q, k, v, beta, decay, s0, block=args.block, o=o, state_out=s_out,
+                                    stream=stream)
+        elif args.segments > 0:
             gdn_forward_segmented(q, k, v, beta, decay, s0, n_segments=args.segments, o=o,
                                   state_out=s_out, stream=stream)
         else:
@@ -392,6 +395,7 @@ def run_gpu(args, world, rank, local):
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk,
                        "dv": wl.dv, "mode": "bidi" if wl.bidi else "causal",
                        "kernel": ("recurrent" if recurrent else
+                                  f"chunk_tc, frame-block read-out, blocks of {args.block}" if args.block > 0 else
                                   f"chunk_tc, segment-parallel x{args.segments}" if segmented else "chunk_tc"),
                        "token_heads_per_gpu": wl.token_heads,
                        "l2": ("no flush: inputs of %.2f GB per step exceed the 126 MB L2" % (bytes_ / 1e9)
@@ -422,6 +426,8 @@ def main():
     ap.add_argument("--recurrent", action="store_true",
                     help="time the token-by-token SIMT kernel instead of the chunkwise one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", type=int, default=0,
+                    help="causal workloads: frame-block read-out with blocks of this many tokens")
     ap.add_argument("--segments", type=int, default=0,
                     help="causal workloads: run the segment-parallel scan with this many segments")
     ap.add_argument("--ref-seconds", type=float, default=None,

@@ -295,6 +295,37 @@ int gdn_forward_segmented(const void *q, const void *k, const void *v, const flo
     }
 }
 
+int gdn_forward_blockcausal(const void *q, const void *k, const void *v, const float *beta,
+                            const float *decay, const float *state_in, float *state_out, void *o,
+                            int B, int H, int T, int dk, int dv, int block, int mode, void *stream)
+{
+    try {
+        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                              mode, "T");
+        if (rc != GDN_OK) return rc;
+        if (block < 1 || T % block != 0)
+            return fail(GDN_ERR_INVALID_ARG, "block must be >= 1 and divide T (got block=%d, T=%d)", block, T);
+        if (mode & (GDN_BIDI | GDN_FP32 | GDN_RECURRENT))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_blockcausal is causal and runs the bf16 chunkwise kernel only "
+                        "(no GDN_BIDI / GDN_FP32 / GDN_RECURRENT)");
+        gdn::FwdArgs a = make_args(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                                   mode);
+        if (!gdn::chunk_tc_supported(a))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_blockcausal needs dk = 128 and dv in {64, 128} (got dk=%d, dv=%d)",
+                        dk, dv);
+        if ((long long)B * H * (T / block) > 65535)
+            return fail(GDN_ERR_UNSUPPORTED, "B*H*T/block = %lld exceeds 65535",
+                        (long long)B * H * (T / block));
+        cudaError_t err = gdn::launch_blockcausal(a, block, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return fail(GDN_ERR_CUDA, "launch failed: %s", cudaGetErrorString(err));
+        return ok();
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in gdn_forward_blockcausal");
+    }
+}
+
 int gdn_device_status(void *stream)
 {
     int err = 0;

@@ -43,6 +43,11 @@ cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream);
 int segment_count(int T, int n_segments, int *seg_chunks);
 cudaError_t launch_segmented(const FwdArgs &a, int n_segments, cudaStream_t stream);
 
+// Frame-block read-out (chunkwise kernel, causal): every token of block f of
+// `block` tokens is read out with the state after the whole block.  T must be
+// a multiple of block.
+cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream);
+
 // Device-side error word (set by bounded waits that gave up).
 cudaError_t device_error_word(int **ptr);
 

@@ -42,13 +42,21 @@ __global__ void identity_fill_kernel(float *out, size_t n_mats)
     }
 }
 
-// E_1 = L_0;  E_{p+1} = P_p E_p + L_p  (p = 1 .. S-2), for one head (blockIdx.x)
-// and 16 state columns (blockIdx.y).  L: [BH][S-1][dk][dv], P: [BH][S-2][dk][dk],
-// E: [BH][S-1][dk][dv] (row p-1 holds E_p).  128 threads, thread r owns row r
+__global__ void fill_kernel(float *out, size_t n, float value)
+{
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x)
+        out[e] = value;
+}
+
+// Threads the state through consecutive pieces of one head (blockIdx.x), 16
+// state columns (blockIdx.y) at a time:  E[0] = L[0],  E[j] = P[p0 + j - 1] E[j-1]
+// + L[j]  for j = 1 .. steps.  L and E hold nrows [dk][dv] states per head, P
+// holds prows [dk][dk] transitions per head.  128 threads, thread r owns row r
 // of the 16-column block; the previous E block sits in shared memory and is
 // read 4 columns at a time.
 __global__ void __launch_bounds__(128) segment_combine_kernel(const float *L, const float *P, float *E,
-                                                              int S, int dv)
+                                                              int nrows, int prows, int p0, int steps,
+                                                              int dv)
 {
     __shared__ __align__(16) float Es[kDKs][16];
     const int bh = blockIdx.x, r = threadIdx.x;
@@ -56,8 +64,8 @@ __global__ void __launch_bounds__(128) segment_combine_kernel(const float *L, co
     const size_t sz = (size_t)kDKs * dv;
     float acc[16];
     {
-        const float *L0 = L + (size_t)bh * (S - 1) * sz + (size_t)r * dv + cg;
-        float *E1 = E + (size_t)bh * (S - 1) * sz + (size_t)r * dv + cg;
+        const float *L0 = L + (size_t)bh * nrows * sz + (size_t)r * dv + cg;
+        float *E1 = E + (size_t)bh * nrows * sz + (size_t)r * dv + cg;
 #pragma unroll
         for (int c = 0; c < 16; c += 4) {
             const float4 v = *reinterpret_cast<const float4 *>(L0 + c);
@@ -65,13 +73,13 @@ __global__ void __launch_bounds__(128) segment_combine_kernel(const float *L, co
             *reinterpret_cast<float4 *>(E1 + c) = v;
         }
     }
-    for (int pp = 1; pp <= S - 2; ++pp) {
+    for (int pp = 1; pp <= steps; ++pp) {
 #pragma unroll
         for (int c = 0; c < 16; c += 4)
             *reinterpret_cast<float4 *>(&Es[r][c]) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
         __syncthreads();
-        const float *Lp = L + ((size_t)bh * (S - 1) + pp) * sz + (size_t)r * dv + cg;
-        const float *Pr = P + ((size_t)bh * (S - 2) + (pp - 1)) * kDKs * kDKs + (size_t)r * kDKs;
+        const float *Lp = L + ((size_t)bh * nrows + pp) * sz + (size_t)r * dv + cg;
+        const float *Pr = P + ((size_t)bh * prows + p0 + pp - 1) * kDKs * kDKs + (size_t)r * kDKs;
 #pragma unroll
         for (int c = 0; c < 16; c += 4) {
             const float4 v = *reinterpret_cast<const float4 *>(Lp + c);
@@ -92,7 +100,7 @@ __global__ void __launch_bounds__(128) segment_combine_kernel(const float *L, co
                     acc[c + 3] = fmaf(pv[u], e.w, acc[c + 3]);
                 }
         }
-        float *Ep = E + ((size_t)bh * (S - 1) + pp) * sz + (size_t)r * dv + cg;
+        float *Ep = E + ((size_t)bh * nrows + pp) * sz + (size_t)r * dv + cg;
 #pragma unroll
         for (int c = 0; c < 16; c += 4)
             *reinterpret_cast<float4 *>(Ep + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
@@ -216,7 +224,8 @@ cudaError_t launch_segmented(const FwdArgs &a, int n_segments, cudaStream_t stre
     }
     // combine: the state entering each segment
     if (err == cudaSuccess) {
-        segment_combine_kernel<<<dim3((unsigned)BH, a.dv / 16), 128, 0, stream>>>(Lst, Pst, Est, S, a.dv);
+        segment_combine_kernel<<<dim3((unsigned)BH, a.dv / 16), 128, 0, stream>>>(Lst, Pst, Est, S - 1, S - 2, 0,
+                                                                                   S - 2, a.dv);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }
@@ -232,6 +241,118 @@ cudaError_t launch_segmented(const FwdArgs &a, int n_segments, cudaStream_t stre
     }
     if (err == cudaSuccess && a.state_out)
         err = cudaMemcpy2DAsync(a.state_out, sz * 4, Fst + (size_t)(S - 2) * sz, (S - 1) * sz * 4, sz * 4, BH,
+                                cudaMemcpyDeviceToDevice, stream);
+    const cudaError_t e2 = cudaFreeAsync(ws, stream);
+    return err != cudaSuccess ? err : e2;
+}
+
+
+// ------------------------------------------------------------ frame-block read-out
+//
+// Every token of block f (tokens [f*Tb, (f+1)*Tb) of a head) is read out with
+// the state after the whole block, o_t = H_{(f+1)Tb-1}^T q_t (the frame-block
+// causal form of a linear-attention KV cache carried across video frames: a
+// token sees its whole frame and every earlier one).  A head-major [B,H,T,d]
+// tensor with T = F*Tb is also a [B*H*F, Tb, d] tensor, so every pass below is
+// one chunkwise launch over B*H*F independent blocks:
+//   1. the blocks from zero (block 0 of each head from the given state): L_f;
+//   2. at the same time, on a second stream: the blocks' transitions P_f
+//      (v = 0 from the identity);
+//   3. combine: E_0 = L_0, E_f = P_f E_{f-1} + L_f, the state after block f;
+//   4. read-out: every block from E_f with identity tokens (b = 0, a = 1), so
+//      the state stays E_f and the kernel's output is o_t = E_f^T q_t.
+cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream)
+{
+    const int F = a.T / block;
+    const size_t BH = (size_t)a.B * a.H, BHF = BH * F, sz = (size_t)a.dk * a.dv, pz = (size_t)a.dk * a.dk;
+    const size_t ntok = BH * (size_t)a.T;
+    const size_t b_st = align_up(BHF * sz * 4), b_p = align_up(BHF * pz * 4);
+    const size_t b_vz = align_up(ntok * a.dk * 2), b_g = align_up(ntok * 4);
+    uint8_t *ws = nullptr;
+    cudaError_t err = cudaMallocAsync(reinterpret_cast<void **>(&ws), 3 * b_st + 2 * b_p + 2 * b_vz + 2 * b_g, stream);
+    if (err != cudaSuccess) return err;
+    float *Sin = reinterpret_cast<float *>(ws);
+    float *Lst = reinterpret_cast<float *>(ws + b_st);
+    float *Est = reinterpret_cast<float *>(ws + 2 * b_st);
+    float *Pin = reinterpret_cast<float *>(ws + 3 * b_st);
+    float *Pst = reinterpret_cast<float *>(ws + 3 * b_st + b_p);
+    void *Vz = ws + 3 * b_st + 2 * b_p;
+    void *Ow = ws + 3 * b_st + 2 * b_p + b_vz;
+    float *Zb = reinterpret_cast<float *>(ws + 3 * b_st + 2 * b_p + 2 * b_vz);
+    float *On = reinterpret_cast<float *>(ws + 3 * b_st + 2 * b_p + 2 * b_vz + b_g);
+
+    FwdArgs blocks = a;   // the [B*H*F, Tb] view
+    blocks.B = (int)BHF;
+    blocks.H = 1;
+    blocks.T = block;
+
+    int dev = 0;
+    err = cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStream *side = nullptr;
+    if (err == cudaSuccess) err = side_stream(dev, &side);
+
+    // pass 2 (second stream): transitions of every block
+    if (err == cudaSuccess) err = cudaEventRecord(side->fork, stream);
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(side->s, side->fork, 0);
+    if (err == cudaSuccess) err = cudaMemsetAsync(Vz, 0, ntok * a.dk * 2, side->s);
+    if (err == cudaSuccess) {
+        identity_fill_kernel<<<148, 256, 0, side->s>>>(Pin, BHF);
+        err = cudaGetLastError();
+        if (err == cudaSuccess) count_launches(1);
+    }
+    if (err == cudaSuccess) {
+        FwdArgs a2 = blocks;
+        a2.v = Vz;
+        a2.dv = a.dk;
+        a2.o = Ow;
+        a2.state_in = Pin;
+        a2.state_out = Pst;
+        err = launch_chunk_tc(a2, side->s);
+    }
+    const bool forked = err == cudaSuccess;
+    if (forked) err = cudaEventRecord(side->join, side->s);
+
+    // pass 1 (caller's stream): every block from zero, block 0 from the given
+    // state; its outputs land in o and are overwritten by the read-out
+    if (err == cudaSuccess) err = cudaMemsetAsync(Sin, 0, BHF * sz * 4, stream);
+    if (err == cudaSuccess && a.state_in)
+        err = cudaMemcpy2DAsync(Sin, F * sz * 4, a.state_in, sz * 4, sz * 4, BH, cudaMemcpyDeviceToDevice,
+                                stream);
+    if (err == cudaSuccess) {
+        FwdArgs a1 = blocks;
+        a1.state_in = Sin;
+        a1.state_out = Lst;
+        err = launch_chunk_tc(a1, stream);
+    }
+    if (forked) {
+        const cudaError_t ej = cudaStreamWaitEvent(stream, side->join, 0);
+        if (err == cudaSuccess) err = ej;
+    }
+    // combine: the state after every block
+    if (err == cudaSuccess) {
+        segment_combine_kernel<<<dim3((unsigned)BH, a.dv / 16), 128, 0, stream>>>(Lst, Pst, Est, F, F, 1, F - 1,
+                                                                                   a.dv);
+        err = cudaGetLastError();
+        if (err == cudaSuccess) count_launches(1);
+    }
+    // read-out with identity tokens
+    if (err == cudaSuccess) err = cudaMemsetAsync(Zb, 0, ntok * 4, stream);
+    if (err == cudaSuccess) {
+        fill_kernel<<<148, 256, 0, stream>>>(On, ntok, 1.f);
+        err = cudaGetLastError();
+        if (err == cudaSuccess) count_launches(1);
+    }
+    if (err == cudaSuccess) {
+        FwdArgs a3 = blocks;
+        a3.beta = Zb;
+        a3.decay = On;
+        a3.state_in = Est;
+        a3.state_out = nullptr;
+        err = launch_chunk_tc(a3, stream);
+    }
+    if (err == cudaSuccess && a.state_out)
+        err = cudaMemcpy2DAsync(a.state_out, sz * 4, Est + (size_t)(F - 1) * sz, F * sz * 4, sz * 4, BH,
                                 cudaMemcpyDeviceToDevice, stream);
     const cudaError_t e2 = cudaFreeAsync(ws, stream);
     return err != cudaSuccess ? err : e2;

@@ -51,6 +51,8 @@ def load_library():
         lib.gdn_forward_noalloc.restype = i
         lib.gdn_forward_segmented.argtypes = [vp] * 8 + [i] * 7 + [vp]
         lib.gdn_forward_segmented.restype = i
+        lib.gdn_forward_blockcausal.argtypes = [vp] * 8 + [i] * 7 + [vp]
+        lib.gdn_forward_blockcausal.restype = i
         lib.gdn_rollout.argtypes = [vp] * 9 + [i] * 7 + [vp]
         lib.gdn_rollout.restype = i
         lib.gdn_device_status.argtypes = [vp]
@@ -164,6 +166,37 @@ def gdn_forward_segmented(q, k, v, beta, decay, state_in=None, *, n_segments=4, 
     _check(lib.gdn_forward_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(state_in),
                                      _ptr(state_out), _ptr(o), B, H, T, dk, dv, int(n_segments),
                                      _mode(q, False, False), _stream_handle(stream, dev)))
+    return o, state_out
+
+
+def gdn_forward_blockcausal(q, k, v, beta, decay, state_in=None, *, block, o=None,
+                            state_out=None, want_state=True, stream=None):
+    """Frame-block causal read-out: every token of block f (frames of `block`
+    tokens, T a multiple of it) is read out with the state after the whole
+    block.  Arguments and layouts as gdn_forward (bf16, dk = 128, dv in
+    {64, 128}); returns o and the final state."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_forward_blockcausal runs on CUDA tensors only")
+    for t, name, shape, dt in ((k, "k", (B, H, T, dk), q.dtype), (v, "v", (B, H, T, dv), q.dtype),
+                               (beta, "beta", (B, H, T), torch.float32),
+                               (decay, "decay", (B, H, T), torch.float32), (q, "q", (B, H, T, dk), q.dtype)):
+        _expect(t, name, shape, dt, dev)
+    if state_in is not None:
+        _expect(state_in, "state_in", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=dev)
+    _expect(o, "o", (B, H, T, dv), q.dtype, dev)
+    if state_out is None and want_state:
+        state_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _expect(state_out, "state_out", (B, H, dk, dv), torch.float32, dev)
+    lib = load_library()
+    _check(lib.gdn_forward_blockcausal(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(state_in),
+                                       _ptr(state_out), _ptr(o), B, H, T, dk, dv, int(block),
+                                       _mode(q, False, False), _stream_handle(stream, dev)))
     return o, state_out
 
 

@@ -171,6 +171,31 @@ int gdn_forward_segmented(const void *q, const void *k, const void *v,
                           void *stream);
 
 /*
+ * gdn_forward_blockcausal -- the frame-block causal read-out: every token of a
+ * frame sees its whole frame and every earlier one (the LongSANA page, "PR
+ * feature": a causal linear-attention KV cache carried across video frames).
+ * The state runs token by token exactly as in gdn_forward; token t of block f
+ * (tokens [f*block, (f+1)*block) of a head) is read out with the state after
+ * the whole block:  o_t = H_{(f+1)*block-1}^T q_t.  state_out is the final
+ * state, as in gdn_forward.
+ *
+ * Arguments and layouts as gdn_forward (bf16 inputs, dk = 128, dv in {64, 128},
+ * mode GDN_CAUSAL); `block` is the frame length in tokens and T must be a
+ * multiple of it.  The blocks' zero-start states and transitions are computed
+ * in parallel (B*H*T/block independent blocks), the state after every block
+ * follows from an fp32 combine, and a read-out pass forms o.  Workspace
+ * (stream-ordered): about B*H*(T/block)*(3*dk*dv + 2*dk*dk)*4 + B*H*T*(4*dk + 8)
+ * bytes.  Errors: as gdn_forward; block < 1 or T not a multiple of block
+ * return GDN_ERR_INVALID_ARG; GDN_BIDI, GDN_FP32 or GDN_RECURRENT, or
+ * B*H*T/block > 65535, return GDN_ERR_UNSUPPORTED.
+ */
+int gdn_forward_blockcausal(const void *q, const void *k, const void *v,
+                            const float *beta, const float *decay,
+                            const float *state_in, float *state_out, void *o,
+                            int B, int H, int T, int dk, int dv, int block, int mode,
+                            void *stream);
+
+/*
  * gdn_device_status -- synchronises `stream` and reports (and clears) the
  * library's device-side error word: GDN_OK, or GDN_ERR_DEVICE_TIMEOUT if a
  * bounded wait inside a kernel gave up since the last call, or GDN_ERR_CUDA.

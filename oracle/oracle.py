@@ -82,3 +82,31 @@ def gdn_rollout(q, k, v, beta, decay, state_in=None, n_threads=None):
     if rc != 0:
         raise RuntimeError(f"oracle_gdn_rollout failed ({rc})")
     return o, s_out, cs
+
+
+def gdn_forward_blockcausal(q, k, v, beta, decay, block, state_in=None, n_threads=None):
+    """Frame-block causal read-out (test infrastructure only).
+
+    Reading (the LongSANA page, "PR feature": a causal linear-attention KV
+    cache carried across video chunks; here every token of a frame sees its
+    whole frame and every earlier frame): the state runs token by token as in
+    gdn_forward, and every token t of block f (tokens [f*block, (f+1)*block))
+    is read out with the state after the whole block:
+        o_t = H_{(f+1)*block - 1}^T q_t.
+    q,k [B,H,T,dk], v [B,H,T,dv], gates [B,H,T]; T a multiple of block.
+    Returns (o [B,H,T,dv], final state [B,H,dk,dv]).  The state after each
+    block comes from the token-by-token scan, run block by block with the
+    state carried (bitwise the single scan); the read-out is a matrix product.
+    """
+    q, k, v, beta, decay = map(_f64, (q, k, v, beta, decay))
+    B, H, T, dk = q.shape
+    assert block >= 1 and T % block == 0
+    state = None if state_in is None else _f64(state_in)
+    o = np.zeros(v.shape, dtype=np.float64)
+    for f in range(T // block):
+        sl = slice(f * block, (f + 1) * block)
+        cut = lambda x: np.ascontiguousarray(x[:, :, sl])
+        _, state = gdn_forward(cut(q), cut(k), cut(v), cut(beta), cut(decay), state_in=state,
+                               n_threads=n_threads)
+        o[:, :, sl] = np.einsum("bhtk,bhkv->bhtv", q[:, :, sl], state)
+    return o, state

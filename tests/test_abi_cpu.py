@@ -27,7 +27,8 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_forward_noalloc",
-              "gdn_forward_segmented", "gdn_device_status", "gdn_kernel_launches",
+              "gdn_forward_segmented", "gdn_forward_blockcausal", "gdn_device_status",
+              "gdn_kernel_launches",
               "gdn_last_error", "gdn_version"):
         assert n in names
 
@@ -128,3 +129,16 @@ def test_segmented_rejects_before_launch(lib):
     assert f(T=0) == -1
     assert lib.gdn_forward_segmented(P, P, P, P, P, None, None, P, 1, 64, 64 * 4000, 128, 128, 2000, 0,
                                      None) == -2         # B*H*segments > 65535
+
+
+def test_blockcausal_rejects_before_launch(lib):
+    """The frame-block entry point needs a block that divides T, runs causal
+    bf16 chunkwise only, and refuses each bad case before any CUDA call."""
+    f = lambda T=640, dk=128, dv=128, block=64, mode=0: lib.gdn_forward_blockcausal(
+        P, P, P, P, P, None, None, P, 1, 1, T, dk, dv, block, mode, None)
+    assert f(block=0) == -1 and b"block" in lib.gdn_last_error()
+    assert f(block=100) == -1                            # 640 is not a multiple of 100
+    assert f(mode=1) == -2                               # bidirectional
+    assert f(mode=2) == -2                               # fp32
+    assert f(dk=64) == -2
+    assert f(T=70000, block=1) == -2                     # 70000 blocks > 65535

@@ -16,6 +16,8 @@ by closed forms and brute force instead:
 * bidirectional = forward + re-reversed forward on the reversed sequence;
 * a rollout split at arbitrary points = one scan (bitwise);
 * the final state is affine in the initial one (the segment transition);
+* the frame-block read-out: blocks of one token = the causal scan; one block
+  with orthonormal keys = its closed form; tiny cases by brute force;
 * the contraction bound ||H_t|| <= a_t ||H_{t-1}|| + b_t ||v_t|| for unit keys.
 Each pin is chosen so that a dropped term, a wrong sign or index, or a
 transposed state would fail at least one of them.
@@ -270,6 +272,59 @@ def test_state_is_affine_in_the_initial_state(oracle_mod):
     X = RNG.standard_normal((dk, dv))
     _, F = oracle_mod.gdn_forward(batch(q), batch(k), batch(v), batch(b), batch(a), state_in=batch(X))
     np.testing.assert_allclose(F[0, 0], P_ref @ X + L[0, 0], rtol=1e-11, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------
+# Frame-block causal read-out
+# ----------------------------------------------------------------------------
+
+def test_blockcausal_block_one_is_the_causal_scan(oracle_mod):
+    """Blocks of one token: every token is read out with its own state."""
+    q, k, v, b, a = _rand_case(2, 2, 40, 6, 5)
+    H0 = RNG.standard_normal((2, 2, 6, 5))
+    o, s = oracle_mod.gdn_forward(q, k, v, b, a, state_in=H0)
+    ob, sb = oracle_mod.gdn_forward_blockcausal(q, k, v, b, a, 1, state_in=H0)
+    np.testing.assert_allclose(ob, o, rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(sb, s)
+
+
+def test_blockcausal_one_block_orthonormal_keys_closed_form(oracle_mod):
+    """One block over the whole sequence with orthonormal keys: the erase term
+    vanishes, the final state is the decayed sum of b_s k_s v_s^T, and every
+    token reads it out."""
+    T, dk, dv = 12, 16, 5
+    k = orthonormal_rows(T, dk)
+    q = RNG.standard_normal((T, dk))
+    v = RNG.standard_normal((T, dv))
+    a = RNG.uniform(0.3, 1.0, T)
+    b = RNG.uniform(0.1, 1.0, T)
+    Hf = sum(np.prod(a[s_ + 1:]) * b[s_] * np.outer(k[s_], v[s_]) for s_ in range(T))
+    o, s = oracle_mod.gdn_forward_blockcausal(batch(q), batch(k), batch(v), batch(b), batch(a), T)
+    np.testing.assert_allclose(s[0, 0], Hf, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(o[0, 0], q @ Hf, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("T,block", [(6, 2), (6, 3), (8, 4)])
+def test_blockcausal_product_expansion(oracle_mod, T, block):
+    """Brute force: every state from the explicit dk x dk product expansion,
+    each token read out with the state at the end of its block."""
+    dk, dv = 3, 2
+    q = RNG.standard_normal((T, dk))
+    k = RNG.standard_normal((T, dk))
+    v = RNG.standard_normal((T, dv))
+    a = RNG.uniform(0.2, 1.0, T)
+    b = RNG.uniform(0.0, 1.0, T)
+    H0 = RNG.standard_normal((dk, dv))
+    states = []
+    H = H0
+    for t in range(T):
+        H = a[t] * (np.eye(dk) - b[t] * np.outer(k[t], k[t])) @ H + b[t] * np.outer(k[t], v[t])
+        states.append(H)
+    ref = np.array([q[t] @ states[(t // block + 1) * block - 1] for t in range(T)])
+    o, s = oracle_mod.gdn_forward_blockcausal(batch(q), batch(k), batch(v), batch(b), batch(a), block,
+                                              state_in=batch(H0))
+    np.testing.assert_allclose(o[0, 0], ref, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(s[0, 0], states[-1], rtol=1e-11, atol=1e-12)
 
 
 def test_rollout_entry_equals_single_scan_bitwise(oracle_mod):
