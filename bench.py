@@ -275,7 +275,7 @@ def run_reference(args, world, rank):
 def run_gpu(args, world, rank, local):
     import torch
     from gated_delta_rule_149_b200 import (gdn, gdn_forward, gdn_forward_blockcausal, gdn_forward_host,
-                                           gdn_forward_segmented, gdn_device_status)
+                                           gdn_forward_normalized, gdn_forward_segmented, gdn_device_status)
     from gated_delta_rule_149_b200.inputs import WORKLOADS, make_inputs
 
     wl = WORKLOADS[args.workload]
@@ -292,12 +292,16 @@ def run_gpu(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     lib = gdn.load_library()
 
-    segmented = args.segments > 0 or args.block > 0
-    if segmented and (wl.bidi or recurrent):
+    segmented = args.segments > 0 or args.block > 0 or args.normalized
+    if (args.segments > 0 or args.block > 0) and (wl.bidi or recurrent):
         raise SystemExit("--segments / --block run causal bf16 workloads only")
+    if args.normalized and recurrent:
+        raise SystemExit("--normalized runs bf16 workloads only")
 
     def step():
-        if args.block > 0:
+        if args.normalized:
+            gdn_forward_normalized(q, k, v, beta, decay, s0, eps=1e-6, bidi=wl.bidi, o=o, stream=stream)
+        elif args.block > 0:
             gdn_forward_blockcausal(q, k, v, beta, decay, s0, block=args.block, o=o, state_out=s_out,
                                     stream=stream)
         elif args.segments > 0:
@@ -395,6 +399,7 @@ def run_gpu(args, world, rank, local):
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk,
                        "dv": wl.dv, "mode": "bidi" if wl.bidi else "causal",
                        "kernel": ("recurrent" if recurrent else
+                                  "chunk_tc, normalised read-out (z state, second pass)" if args.normalized else
                                   f"chunk_tc, frame-block read-out, blocks of {args.block}" if args.block > 0 else
                                   f"chunk_tc, segment-parallel x{args.segments}" if segmented else "chunk_tc"),
                        "token_heads_per_gpu": wl.token_heads,
@@ -426,6 +431,8 @@ def main():
     ap.add_argument("--recurrent", action="store_true",
                     help="time the token-by-token SIMT kernel instead of the chunkwise one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--normalized", action="store_true",
+                    help="normalised read-out with a z state (eps 1e-6)")
     ap.add_argument("--block", type=int, default=0,
                     help="causal workloads: frame-block read-out with blocks of this many tokens")
     ap.add_argument("--segments", type=int, default=0,

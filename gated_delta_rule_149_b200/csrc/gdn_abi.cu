@@ -326,6 +326,36 @@ int gdn_forward_blockcausal(const void *q, const void *k, const void *v, const f
     }
 }
 
+int gdn_forward_normalized(const void *q, const void *k, const void *v, const float *beta,
+                           const float *decay, const float *state_in, const float *state_z_in,
+                           float *state_out, float *state_z_out, void *o, int B, int H, int T, int dk,
+                           int dv, float eps, int mode, void *stream)
+{
+    try {
+        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                              mode, "T");
+        if (rc != GDN_OK) return rc;
+        if ((reinterpret_cast<uintptr_t>(state_z_in) | reinterpret_cast<uintptr_t>(state_z_out)) & 15)
+            return fail(GDN_ERR_MISALIGNED, "state_z_in / state_z_out is not 16-byte aligned");
+        if (mode & (GDN_FP32 | GDN_RECURRENT))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_normalized runs the bf16 chunkwise kernel only (no GDN_FP32 / "
+                        "GDN_RECURRENT)");
+        gdn::FwdArgs a = make_args(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                                   mode);
+        if (!gdn::chunk_tc_supported(a))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_normalized needs dk = 128 and dv in {64, 128} (got dk=%d, dv=%d)",
+                        dk, dv);
+        cudaError_t err = gdn::launch_normalized(a, state_z_in, state_z_out, eps,
+                                                 static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return fail(GDN_ERR_CUDA, "launch failed: %s", cudaGetErrorString(err));
+        return ok();
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in gdn_forward_normalized");
+    }
+}
+
 int gdn_device_status(void *stream)
 {
     int err = 0;

@@ -48,6 +48,12 @@ cudaError_t launch_segmented(const FwdArgs &a, int n_segments, cudaStream_t stre
 // a multiple of block.
 cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream);
 
+// Normalised read-out o = (S q) / (z.q + eps), z the same recurrence driven by a
+// value of 1; state_z_in [B,H,dk] or nullptr, state_z_out [B,H,dk] (bidi
+// [2,B,H,dk]) or nullptr.
+cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *state_z_out, float eps,
+                              cudaStream_t stream);
+
 // Device-side error word (set by bounded waits that gave up).
 cudaError_t device_error_word(int **ptr);
 

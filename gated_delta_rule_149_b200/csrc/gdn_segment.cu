@@ -359,3 +359,120 @@ cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream)
 }
 
 }  // namespace gdn
+
+// ------------------------------------------------------------ normalised read-out
+//
+// o_t = (S_t q_t) / (z_t . q_t + eps), with z the same gated delta recurrence
+// driven by a constant value of 1 (bidirectional: numerators and denominators
+// summed over the two directions, then divided).  The numerator is the plain
+// call; the denominator is a second call with a 64-wide value of ones (every
+// column is the same z), on a second stream for causal calls; a last kernel
+// divides.
+
+namespace gdn {
+namespace {
+
+__global__ void fill_bf16_kernel(__nv_bfloat16 *out, size_t n, float value)
+{
+    const __nv_bfloat16 v = __float2bfloat16(value);
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x)
+        out[e] = v;
+}
+
+// every column of the [rows][64] output is z_in[row]
+__global__ void broadcast_cols_kernel(float *out, const float *z, size_t rows)
+{
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < rows * 64; e += (size_t)gridDim.x * blockDim.x)
+        out[e] = z[e / 64];
+}
+
+// o[row][c] /= (den[row][0] + eps), 8 bf16 values per thread step
+__global__ void divide_rows_kernel(__nv_bfloat16 *o, const __nv_bfloat16 *den, size_t rows, int dv, float eps)
+{
+    const int per = dv / 8;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < rows * per; e += (size_t)gridDim.x * blockDim.x) {
+        const size_t row = e / per;
+        const float inv = 1.f / (__bfloat162float(den[row * 64]) + eps);
+        uint4 w = *reinterpret_cast<const uint4 *>(o + e * 8);
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&w);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float2 f = __bfloat1622float2(h[u]);
+            h[u] = __floats2bfloat162_rn(f.x * inv, f.y * inv);
+        }
+        *reinterpret_cast<uint4 *>(o + e * 8) = w;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *state_z_out, float eps,
+                              cudaStream_t stream)
+{
+    const size_t BH = (size_t)a.B * a.H, ntok = BH * (size_t)a.T, ndir = a.bidi ? 2 : 1;
+    const size_t b_ones = align_up(ntok * 64 * 2), b_den = b_ones;
+    const size_t b_zin = align_up(BH * a.dk * 64 * 4), b_zout = align_up(ndir * BH * a.dk * 64 * 4);
+    uint8_t *ws = nullptr;
+    cudaError_t err = cudaMallocAsync(reinterpret_cast<void **>(&ws), b_ones + b_den + b_zin + b_zout, stream);
+    if (err != cudaSuccess) return err;
+    auto *ones = reinterpret_cast<__nv_bfloat16 *>(ws);
+    auto *den = reinterpret_cast<__nv_bfloat16 *>(ws + b_ones);
+    float *zin = reinterpret_cast<float *>(ws + b_ones + b_den);
+    float *zout = reinterpret_cast<float *>(ws + b_ones + b_den + b_zin);
+
+    // causal: the denominator pass runs beside the numerator pass on a second
+    // stream.  Bidirectional: after it, on the caller's stream (a bidirectional
+    // launch counts on having every one of its CTAs resident at once).
+    int dev = 0;
+    err = cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStream *side = nullptr;
+    if (err == cudaSuccess && !a.bidi) err = side_stream(dev, &side);
+    cudaStream_t ds = a.bidi ? stream : (side ? side->s : stream);
+    bool forked = false;
+    if (err == cudaSuccess && !a.bidi) {
+        err = cudaEventRecord(side->fork, stream);
+        if (err == cudaSuccess) err = cudaStreamWaitEvent(side->s, side->fork, 0);
+    }
+    if (err == cudaSuccess && a.bidi) err = launch_chunk_tc(a, stream);   // numerator first
+    if (err == cudaSuccess) {
+        fill_bf16_kernel<<<148, 256, 0, ds>>>(ones, ntok * 64, 1.f);
+        err = cudaGetLastError();
+        if (err == cudaSuccess) count_launches(1);
+    }
+    if (err == cudaSuccess && state_z_in) {
+        broadcast_cols_kernel<<<148, 256, 0, ds>>>(zin, state_z_in, BH * a.dk);
+        err = cudaGetLastError();
+        if (err == cudaSuccess) count_launches(1);
+    }
+    if (err == cudaSuccess) {
+        FwdArgs az = a;
+        az.v = ones;
+        az.dv = 64;
+        az.o = den;
+        az.state_in = state_z_in ? zin : nullptr;
+        az.state_out = state_z_out ? zout : nullptr;
+        err = launch_chunk_tc(az, ds);
+    }
+    if (!a.bidi && side) {
+        forked = err == cudaSuccess;
+        if (forked) err = cudaEventRecord(side->join, side->s);
+        if (err == cudaSuccess) err = launch_chunk_tc(a, stream);            // numerator
+        if (forked) {
+            const cudaError_t ej = cudaStreamWaitEvent(stream, side->join, 0);
+            if (err == cudaSuccess) err = ej;
+        }
+    }
+    if (err == cudaSuccess) {
+        divide_rows_kernel<<<592, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(a.o), den, ntok, a.dv, eps);
+        err = cudaGetLastError();
+        if (err == cudaSuccess) count_launches(1);
+    }
+    // z out: column 0 of every [dk][64] state
+    if (err == cudaSuccess && state_z_out)
+        err = cudaMemcpy2DAsync(state_z_out, 4, zout, 64 * 4, 4, ndir * BH * a.dk, cudaMemcpyDeviceToDevice, stream);
+    const cudaError_t e2 = cudaFreeAsync(ws, stream);
+    return err != cudaSuccess ? err : e2;
+}
+
+}  // namespace gdn

@@ -53,6 +53,8 @@ def load_library():
         lib.gdn_forward_segmented.restype = i
         lib.gdn_forward_blockcausal.argtypes = [vp] * 8 + [i] * 7 + [vp]
         lib.gdn_forward_blockcausal.restype = i
+        lib.gdn_forward_normalized.argtypes = [vp] * 10 + [i] * 5 + [ctypes.c_float, i, vp]
+        lib.gdn_forward_normalized.restype = i
         lib.gdn_rollout.argtypes = [vp] * 9 + [i] * 7 + [vp]
         lib.gdn_rollout.restype = i
         lib.gdn_device_status.argtypes = [vp]
@@ -198,6 +200,38 @@ def gdn_forward_blockcausal(q, k, v, beta, decay, state_in=None, *, block, o=Non
                                        _ptr(state_out), _ptr(o), B, H, T, dk, dv, int(block),
                                        _mode(q, False, False), _stream_handle(stream, dev)))
     return o, state_out
+
+
+def gdn_forward_normalized(q, k, v, beta, decay, state_in=None, state_z_in=None, *, eps=1e-6,
+                           bidi=False, o=None, stream=None):
+    """Normalised read-out o = (S q) / (z.q + eps), z the same recurrence driven
+    by a value of 1.  Arguments as gdn_forward (bf16, dk = 128, dv in
+    {64, 128}) plus state_z_in [B,H,dk] fp32 or None.  Returns o, the kv state
+    and the z state ([B,H,dk], bidi [2,B,H,dk])."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_forward_normalized runs on CUDA tensors only")
+    for t, name, shape, dt in ((k, "k", (B, H, T, dk), q.dtype), (v, "v", (B, H, T, dv), q.dtype),
+                               (beta, "beta", (B, H, T), torch.float32),
+                               (decay, "decay", (B, H, T), torch.float32), (q, "q", (B, H, T, dk), q.dtype)):
+        _expect(t, name, shape, dt, dev)
+    if state_in is not None:
+        _expect(state_in, "state_in", (B, H, dk, dv), torch.float32, dev)
+    if state_z_in is not None:
+        _expect(state_z_in, "state_z_in", (B, H, dk), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=dev)
+    _expect(o, "o", (B, H, T, dv), q.dtype, dev)
+    lead = (2,) if bidi else ()
+    s_kv = torch.empty(lead + (B, H, dk, dv), dtype=torch.float32, device=dev)
+    s_z = torch.empty(lead + (B, H, dk), dtype=torch.float32, device=dev)
+    lib = load_library()
+    _check(lib.gdn_forward_normalized(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(state_in),
+                                      _ptr(state_z_in), _ptr(s_kv), _ptr(s_z), _ptr(o), B, H, T, dk, dv,
+                                      ctypes.c_float(eps), _mode(q, bidi, False), _stream_handle(stream, dev)))
+    return o, s_kv, s_z
 
 
 def gdn_rollout(q, k, v, beta, decay, state_in=None, *, recurrent=False, chunk_states=False,

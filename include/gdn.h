@@ -196,6 +196,32 @@ int gdn_forward_blockcausal(const void *q, const void *k, const void *v,
                             void *stream);
 
 /*
+ * gdn_forward_normalized -- the normalised read-out with a z state next to the
+ * kv state (the librediffusion PR #21 review names state_kv and state_z of its
+ * bidirectional kernel; the pages give no formula, so this is a reading).  z
+ * runs the same gated delta recurrence driven by a constant value of 1,
+ *     z_t = a_t (I - b_t k_t k_t^T) z_{t-1} + b_t k_t,
+ * and o_t = (S_t q_t) / (z_t . q_t + eps).  GDN_BIDI sums the numerators and
+ * the denominators of the two scan directions, then divides.
+ *
+ * Arguments as gdn_forward (bf16 inputs, dk = 128, dv in {64, 128}), plus
+ * state_z_in [B,H,dk] fp32 (NULL: zero; forward scan only), state_z_out
+ * [B,H,dk] (GDN_BIDI: [2,B,H,dk]) or NULL, and eps.  The denominators come from
+ * a second chunkwise pass over a 64-wide value of ones (beside the first on a
+ * second stream for causal calls, after it for bidirectional ones); both
+ * passes write bf16, so numerator and denominator are each rounded to bf16
+ * before the division.  Workspace (stream-ordered): about B*H*T*256 +
+ * B*H*dk*768 bytes.  Errors: as gdn_forward; GDN_FP32 or GDN_RECURRENT return
+ * GDN_ERR_UNSUPPORTED; a misaligned state_z pointer GDN_ERR_MISALIGNED.
+ */
+int gdn_forward_normalized(const void *q, const void *k, const void *v,
+                           const float *beta, const float *decay,
+                           const float *state_in, const float *state_z_in,
+                           float *state_out, float *state_z_out, void *o,
+                           int B, int H, int T, int dk, int dv, float eps, int mode,
+                           void *stream);
+
+/*
  * gdn_device_status -- synchronises `stream` and reports (and clears) the
  * library's device-side error word: GDN_OK, or GDN_ERR_DEVICE_TIMEOUT if a
  * bounded wait inside a kernel gave up since the last call, or GDN_ERR_CUDA.

@@ -3,4 +3,6 @@
 Imported by tests/, __graft_entry__.smoke() and bench.py's CPU-baseline leg;
 never by the product package.
 """
-from .oracle import gdn_forward, gdn_forward_blockcausal, gdn_rollout, load  # noqa: F401
+from .oracle import (  # noqa: F401
+    gdn_forward, gdn_forward_blockcausal, gdn_forward_normalized, gdn_rollout, load,
+)

@@ -110,3 +110,26 @@ def gdn_forward_blockcausal(q, k, v, beta, decay, block, state_in=None, n_thread
                                n_threads=n_threads)
         o[:, :, sl] = np.einsum("bhtk,bhkv->bhtv", q[:, :, sl], state)
     return o, state
+
+
+def gdn_forward_normalized(q, k, v, beta, decay, state_in=None, state_z_in=None, eps=1e-6,
+                           bidi=False, n_threads=None):
+    """Normalised read-out with a z state (test infrastructure only).
+
+    Reading (the librediffusion PR #21 review names a state_z next to
+    state_kv in its bidirectional kernel, with no formula): z is the same
+    gated delta recurrence driven by a constant value of 1,
+        z_t = a_t (I - b_t k_t k_t^T) z_{t-1} + b_t k_t,
+    and o_t = (S_t q_t) / (z_t . q_t + eps).  Bidirectional: numerators and
+    denominators are each summed over the two scan directions (as gdn_forward
+    sums o), then divided.  z runs token by token through the same oracle scan
+    with a one-column value of ones.
+    Returns (o [B,H,T,dv], state_kv, state_z [B,H,dk] (bidi: [2,B,H,dk])).
+    """
+    q, k, v, beta, decay = map(_f64, (q, k, v, beta, decay))
+    B, H, T, dk = q.shape
+    num, s_kv = gdn_forward(q, k, v, beta, decay, state_in=state_in, bidi=bidi, n_threads=n_threads)
+    ones = np.ones((B, H, T, 1))
+    z_in = None if state_z_in is None else _f64(state_z_in)[..., None]
+    den, s_z = gdn_forward(q, k, ones, beta, decay, state_in=z_in, bidi=bidi, n_threads=n_threads)
+    return num / (den + eps), s_kv, s_z[..., 0]

@@ -27,7 +27,8 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_forward_noalloc",
-              "gdn_forward_segmented", "gdn_forward_blockcausal", "gdn_device_status",
+              "gdn_forward_segmented", "gdn_forward_blockcausal", "gdn_forward_normalized",
+              "gdn_device_status",
               "gdn_kernel_launches",
               "gdn_last_error", "gdn_version"):
         assert n in names
@@ -142,3 +143,15 @@ def test_blockcausal_rejects_before_launch(lib):
     assert f(mode=2) == -2                               # fp32
     assert f(dk=64) == -2
     assert f(T=70000, block=1) == -2                     # 70000 blocks > 65535
+
+
+def test_normalized_rejects_before_launch(lib):
+    """The normalised read-out runs the bf16 chunkwise kernel only and checks
+    its z-state pointers, before any CUDA call."""
+    f = lambda dk=128, dv=128, mode=0, zin=None, zout=None: lib.gdn_forward_normalized(
+        P, P, P, P, P, None, zin, None, zout, P, 1, 1, 640, dk, dv, ctypes.c_float(1e-6), mode, None)
+    assert f(mode=2) == -2                               # fp32
+    assert f(mode=4) == -2                               # recurrent kernel
+    assert f(dk=64) == -2
+    assert f(zin=PM) == -3 and b"state_z" in lib.gdn_last_error()
+    assert f(zout=PM) == -3

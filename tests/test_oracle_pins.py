@@ -18,6 +18,8 @@ by closed forms and brute force instead:
 * the final state is affine in the initial one (the segment transition);
 * the frame-block read-out: blocks of one token = the causal scan; one block
   with orthonormal keys = its closed form; tiny cases by brute force;
+* the normalised read-out: its closed form with orthonormal keys, z against its
+  written-out recurrence, linearity in v, the bidirectional sums;
 * the contraction bound ||H_t|| <= a_t ||H_{t-1}|| + b_t ||v_t|| for unit keys.
 Each pin is chosen so that a dropped term, a wrong sign or index, or a
 transposed state would fail at least one of them.
@@ -325,6 +327,62 @@ def test_blockcausal_product_expansion(oracle_mod, T, block):
                                               state_in=batch(H0))
     np.testing.assert_allclose(o[0, 0], ref, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(s[0, 0], states[-1], rtol=1e-11, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Normalised read-out (z state)
+# ----------------------------------------------------------------------------
+
+def test_normalized_orthonormal_keys_closed_form(oracle_mod):
+    """Orthonormal keys: both states are decayed sums (no erase), so
+    o_t = sum_s w_ts (k_s.q_t) v_s / (sum_s w_ts (k_s.q_t) + eps) with
+    w_ts = b_s prod_{r=s+1..t} a_r, by a double sum."""
+    T, dk, dv, eps = 10, 16, 4, 1e-3
+    k = orthonormal_rows(T, dk)
+    q = np.abs(RNG.standard_normal((T, dk)))
+    v = RNG.standard_normal((T, dv))
+    a = RNG.uniform(0.3, 1.0, T)
+    b = RNG.uniform(0.1, 1.0, T)
+    o, s_kv, s_z = oracle_mod.gdn_forward_normalized(batch(q), batch(k), batch(v), batch(b), batch(a), eps=eps)
+    ref = np.zeros((T, dv))
+    for t in range(T):
+        w = [b[s_] * np.prod(a[s_ + 1:t + 1]) * (k[s_] @ q[t]) for s_ in range(t + 1)]
+        ref[t] = sum(w[s_] * v[s_] for s_ in range(t + 1)) / (sum(w) + eps)
+    np.testing.assert_allclose(o[0, 0], ref, rtol=1e-11, atol=1e-12)
+    z_ref = sum(b[s_] * np.prod(a[s_ + 1:]) * k[s_] for s_ in range(T))
+    np.testing.assert_allclose(s_z[0, 0], z_ref, rtol=1e-12, atol=1e-13)
+
+
+def test_normalized_z_is_the_recurrence_with_unit_values(oracle_mod):
+    """z against its recurrence written out with the dk x dk factor, from a
+    given initial z; and a value scale passes straight through the read-out."""
+    T, dk, dv = 9, 5, 3
+    q = RNG.standard_normal((T, dk))
+    k = rand_unit(T, dk)
+    v = RNG.standard_normal((T, dv))
+    a = RNG.uniform(0.2, 1.0, T)
+    b = RNG.uniform(0.0, 1.0, T)
+    z0 = RNG.standard_normal(dk)
+    z = z0.copy()
+    for t in range(T):
+        z = a[t] * (np.eye(dk) - b[t] * np.outer(k[t], k[t])) @ z + b[t] * k[t]
+    o, _, s_z = oracle_mod.gdn_forward_normalized(batch(q), batch(k), batch(v), batch(b), batch(a),
+                                                   state_z_in=z0[None, None], eps=0.5)
+    np.testing.assert_allclose(s_z[0, 0], z, rtol=1e-12, atol=1e-13)
+    o3, _, _ = oracle_mod.gdn_forward_normalized(batch(q), batch(k), batch(3 * v), batch(b), batch(a),
+                                                 state_z_in=z0[None, None], eps=0.5)
+    np.testing.assert_allclose(o3, 3 * o, rtol=1e-12, atol=1e-13)
+
+
+def test_normalized_bidi_sums_numerators_and_denominators(oracle_mod):
+    q, k, v, b, a = _rand_case(1, 2, 30, 6, 4)
+    q = np.abs(q)
+    eps = 1e-2
+    o, s_kv, s_z = oracle_mod.gdn_forward_normalized(q, k, v, b, a, eps=eps, bidi=True)
+    num, _ = oracle_mod.gdn_forward(q, k, v, b, a, bidi=True)
+    den, _ = oracle_mod.gdn_forward(q, k, np.ones(v.shape[:3] + (1,)), b, a, bidi=True)
+    np.testing.assert_array_equal(o, num / (den + eps))
+    assert s_z.shape == (2, 1, 2, 6)
 
 
 def test_rollout_entry_equals_single_scan_bitwise(oracle_mod):
