@@ -76,6 +76,15 @@ enum gdn_status {
  *   bf16 (chunkwise tensor-core kernel): dk = 128, dv in {64, 128}.
  *   fp32, or any dtype with GDN_RECURRENT: dk, dv multiples of 32, <= 128.
  * T >= 1 of any value (a ragged last chunk is handled).  B*H <= 65535.
+ *
+ * Bidirectional bf16 calls whose CTAs (B*H*2*dv/64) fit on the GPU's SMs fix
+ * the order in which the two directions write each output tile in advance and
+ * wait for one another inside the kernel: they count on every CTA being
+ * resident at once.  If other work on other streams keeps SMs busy meanwhile,
+ * a wait can run out (4 s) and the call reports GDN_ERR_DEVICE_TIMEOUT through
+ * gdn_device_status (no hang, no silent result); run such calls without
+ * concurrent kernels.  Larger grids decide the order at run time and have no
+ * such requirement.
  */
 int gdn_forward(const void *q, const void *k, const void *v,
                 const float *beta, const float *decay,
