@@ -72,10 +72,11 @@ def load_peaks():
 
 
 def kernel_source_sha():
-    """Hash of the kernel sources' code (comments and whitespace removed), so
-    that a recorded traffic figure stays tied to the code it was taken on."""
+    """Hash of the chunkwise kernel's device code (its source and the PTX
+    wrappers it includes; comments and whitespace removed), so that a recorded
+    traffic figure stays tied to the kernel it was taken on."""
     h = hashlib.sha256()
-    for name in ("gdn_chunk_tc.cu", "gdn_recurrent.cu", "sm100_ptx.cuh", "gdn_internal.h"):
+    for name in ("gdn_chunk_tc.cu", "sm100_ptx.cuh"):
         p = os.path.join(ROOT, "gated_delta_rule_149_b200", "csrc", name)
         if os.path.exists(p):
             src = open(p).read()
