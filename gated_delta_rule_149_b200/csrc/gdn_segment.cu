@@ -1,3 +1,7 @@
+// Forms of the recurrence built from passes of the chunkwise kernel plus small
+// kernels of their own: the segment-parallel causal scan, the frame-block
+// read-out and the normalised read-out (sections below).
+//
 // Segment-parallel causal scan: a few long scans (few heads, many chunks) are
 // split along time so that more SMs work at once.
 //
