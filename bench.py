@@ -177,13 +177,23 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The maximum of a per-rank scalar over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(token_heads_per_rank, total_ms, steps, world):
+    """Weak scaling over replicas: every rank runs its own full workload, the
+    job's step time is the slowest rank's, and the job processes world times
+    one rank's tokens*heads per step.  Returns (ms_per_step, value)."""
+    ms_per_step = max_over_ranks(total_ms, world) / steps
+    return ms_per_step, world * token_heads_per_rank / (ms_per_step * 1e-3)
 
 
 # --------------------------------------------------------------------------
@@ -344,9 +354,7 @@ def run_gpu(args, world, rank, local):
     per_call = [a.elapsed_time(b) for a, b in ev]
     # with flushes between steps, the steps' own events give the step time
     total_ms = t_all0.elapsed_time(t_all1) if flush_buf is None else sum(per_call)
-    total_ms = max_over_ranks(total_ms, world)
-    ms_per_step = total_ms / args.steps
-    value = world * wl.token_heads / (ms_per_step * 1e-3)
+    ms_per_step, value = replica_throughput(wl.token_heads, total_ms, args.steps, world)
 
     # roofline of the main kernel (the call is one main kernel plus a tiny memset)
     hbm_peak, tc_peak, peak_kind = load_peaks()
