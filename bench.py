@@ -285,8 +285,10 @@ def run_reference(args, world, rank):
 
 def run_gpu(args, world, rank, local):
     import torch
-    from gated_delta_rule_149_b200 import (gdn, gdn_forward, gdn_forward_blockcausal, gdn_forward_host,
-                                           gdn_forward_normalized, gdn_forward_segmented, gdn_device_status)
+    from gated_delta_rule_149_b200 import (gdn, gdn_forward, gdn_forward_blockcausal, gdn_forward_fp8,
+                                           gdn_forward_host, gdn_forward_normalized, gdn_forward_segmented,
+                                           gdn_device_status)
+    from gated_delta_rule_149_b200.inputs import quantize_e4m3
     from gated_delta_rule_149_b200.inputs import WORKLOADS, make_inputs
 
     wl = WORKLOADS[args.workload]
@@ -303,14 +305,22 @@ def run_gpu(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     lib = gdn.load_library()
 
-    segmented = args.segments > 0 or args.block > 0 or args.normalized
+    segmented = args.segments > 0 or args.block > 0 or args.normalized or args.fp8
+    if args.fp8:
+        if recurrent:
+            raise SystemExit("--fp8 runs bf16-output workloads only")
+        (q8, sq), (k8, sk), (v8, sv) = (quantize_e4m3(x) for x in (inp.q, inp.k, inp.v))
+        q8, k8, v8, sq, sk, sv = (t.to(dev) for t in (q8, k8, v8, sq, sk, sv))
     if (args.segments > 0 or args.block > 0) and (wl.bidi or recurrent):
         raise SystemExit("--segments / --block run causal bf16 workloads only")
     if args.normalized and recurrent:
         raise SystemExit("--normalized runs bf16 workloads only")
 
     def step():
-        if args.normalized:
+        if args.fp8:
+            gdn_forward_fp8(q8, k8, v8, sq, sk, sv, beta, decay, s0, bidi=wl.bidi, o=o, state_out=s_out,
+                            stream=stream)
+        elif args.normalized:
             gdn_forward_normalized(q, k, v, beta, decay, s0, eps=1e-6, bidi=wl.bidi, o=o, stream=stream)
         elif args.block > 0:
             gdn_forward_blockcausal(q, k, v, beta, decay, s0, block=args.block, o=o, state_out=s_out,
@@ -371,14 +381,20 @@ def run_gpu(args, world, rank, local):
 
     # end to end through the host-buffer entry point
     pin = lambda t: t.pin_memory()
-    hq, hk, hv, hb, ha = map(pin, (inp.q, inp.k, inp.v, inp.beta, inp.decay))
+    if args.fp8:   # the host buffers of an fp8 call are its codes and scales
+        hq, hk, hv, hsq, hsk, hsv = (pin(t.cpu()) for t in (q8, k8, v8, sq, sk, sv))
+    else:
+        hq, hk, hv = map(pin, (inp.q, inp.k, inp.v))
+    hb, ha = map(pin, (inp.beta, inp.decay))
     hs0 = None if inp.state0 is None else pin(inp.state0)
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hso = torch.empty(s_out.shape, dtype=torch.float32).pin_memory()
 
     def e2e_step():
         if segmented:   # the same call on device copies of pinned host buffers
-            for h, dst in ((hq, q), (hk, k), (hv, v), (hb, beta), (ha, decay), (hs0, s0)):
+            pairs = ((hq, q8), (hk, k8), (hv, v8), (hsq, sq), (hsk, sk), (hsv, sv)) if args.fp8 else \
+                ((hq, q), (hk, k), (hv, v))
+            for h, dst in pairs + ((hb, beta), (ha, decay), (hs0, s0)):
                 if h is not None:
                     dst.copy_(h, non_blocking=True)
             step()
@@ -408,6 +424,7 @@ def run_gpu(args, world, rank, local):
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk,
                        "dv": wl.dv, "mode": "bidi" if wl.bidi else "causal",
                        "kernel": ("recurrent" if recurrent else
+                                  "chunk_tc, fp8 E4M3 inputs (dequantising pre-pass)" if args.fp8 else
                                   "chunk_tc, normalised read-out (z state, second pass)" if args.normalized else
                                   f"chunk_tc, frame-block read-out, blocks of {args.block}" if args.block > 0 else
                                   f"chunk_tc, segment-parallel x{args.segments}" if segmented else "chunk_tc"),
@@ -418,7 +435,8 @@ def run_gpu(args, world, rank, local):
                               "in the 126 MB L2); step time from the steps' own events" % (bytes_ / 1e9)),
                        "parallelism": f"replicas x{world} (independent scans, no collective)"},
             "e2e": {"value": world * wl.token_heads / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": nbytes(hq, hk, hv, hb, ha, hs0),
+                    "h2d_bytes_per_step": nbytes(hq, hk, hv, hb, ha, hs0,
+                                                 *((hsq, hsk, hsv) if args.fp8 else ())),
                     "d2h_bytes_per_step": nbytes(ho, hso)},
             "gpu_launches": int(launches),
             "roofline": roofline,
@@ -440,6 +458,8 @@ def main():
     ap.add_argument("--recurrent", action="store_true",
                     help="time the token-by-token SIMT kernel instead of the chunkwise one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="fp8 (E4M3) q, k, v with per-head scales (dequantising pre-pass)")
     ap.add_argument("--normalized", action="store_true",
                     help="normalised read-out with a z state (eps 1e-6)")
     ap.add_argument("--block", type=int, default=0,

@@ -356,6 +356,33 @@ int gdn_forward_normalized(const void *q, const void *k, const void *v, const fl
     }
 }
 
+int gdn_forward_fp8(const void *q8, const void *k8, const void *v8, const float *q_scale,
+                    const float *k_scale, const float *v_scale, const float *beta, const float *decay,
+                    const float *state_in, float *state_out, void *o, int B, int H, int T, int dk, int dv,
+                    int mode, void *stream)
+{
+    try {
+        int rc = check_common(q8, k8, v8, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                              mode, "T");
+        if (rc != GDN_OK) return rc;
+        if (!q_scale || !k_scale || !v_scale)
+            return fail(GDN_ERR_INVALID_ARG, "q_scale, k_scale and v_scale must be non-NULL");
+        if (mode & (GDN_FP32 | GDN_RECURRENT))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_fp8 takes E4M3 inputs and writes bf16 o (no GDN_FP32 / GDN_RECURRENT)");
+        gdn::FwdArgs a = make_args(q8, k8, v8, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                                   mode);
+        if (!gdn::chunk_tc_supported(a))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_forward_fp8 needs dk = 128 and dv in {64, 128} (got dk=%d, dv=%d)", dk, dv);
+        cudaError_t err = gdn::launch_fp8(a, q_scale, k_scale, v_scale, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return fail(GDN_ERR_CUDA, "launch failed: %s", cudaGetErrorString(err));
+        return ok();
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in gdn_forward_fp8");
+    }
+}
+
 int gdn_device_status(void *stream)
 {
     int err = 0;

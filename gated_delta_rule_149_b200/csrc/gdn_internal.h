@@ -54,6 +54,11 @@ cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream)
 cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *state_z_out, float eps,
                               cudaStream_t stream);
 
+// fp8 (E4M3) q, k, v with per-(batch, head) fp32 scales: dequantised to bf16
+// workspace copies, then the chunkwise kernel (a.q, a.k, a.v are the fp8 codes).
+cudaError_t launch_fp8(const FwdArgs &a, const float *q_scale, const float *k_scale, const float *v_scale,
+                       cudaStream_t stream);
+
 // Device-side error word (set by bounded waits that gave up).
 cudaError_t device_error_word(int **ptr);
 

@@ -55,6 +55,8 @@ def load_library():
         lib.gdn_forward_blockcausal.restype = i
         lib.gdn_forward_normalized.argtypes = [vp] * 10 + [i] * 5 + [ctypes.c_float, i, vp]
         lib.gdn_forward_normalized.restype = i
+        lib.gdn_forward_fp8.argtypes = [vp] * 11 + [i] * 6 + [vp]
+        lib.gdn_forward_fp8.restype = i
         lib.gdn_rollout.argtypes = [vp] * 9 + [i] * 7 + [vp]
         lib.gdn_rollout.restype = i
         lib.gdn_device_status.argtypes = [vp]
@@ -232,6 +234,38 @@ def gdn_forward_normalized(q, k, v, beta, decay, state_in=None, state_z_in=None,
                                       _ptr(state_z_in), _ptr(s_kv), _ptr(s_z), _ptr(o), B, H, T, dk, dv,
                                       ctypes.c_float(eps), _mode(q, bidi, False), _stream_handle(stream, dev)))
     return o, s_kv, s_z
+
+
+def gdn_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, beta, decay, state_in=None, *, bidi=False,
+                    o=None, state_out=None, want_state=True, stream=None):
+    """gdn_forward on fp8 (E4M3) q, k, v given as uint8 codes [B,H,T,d] with
+    fp32 scales [B,H] (x = scale * decode(x8)); o is bf16."""
+    B, H, T, dk = q8.shape
+    dv = v8.shape[-1]
+    dev = q8.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_forward_fp8 runs on CUDA tensors only")
+    for t, name, shape, dt in ((q8, "q8", (B, H, T, dk), torch.uint8), (k8, "k8", (B, H, T, dk), torch.uint8),
+                               (v8, "v8", (B, H, T, dv), torch.uint8),
+                               (q_scale, "q_scale", (B, H), torch.float32), (k_scale, "k_scale", (B, H), torch.float32),
+                               (v_scale, "v_scale", (B, H), torch.float32),
+                               (beta, "beta", (B, H, T), torch.float32), (decay, "decay", (B, H, T), torch.float32)):
+        _expect(t, name, shape, dt, dev)
+    if state_in is not None:
+        _expect(state_in, "state_in", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=torch.bfloat16, device=dev)
+    _expect(o, "o", (B, H, T, dv), torch.bfloat16, dev)
+    s_shape = ((2,) if bidi else ()) + (B, H, dk, dv)
+    if state_out is None and want_state:
+        state_out = torch.empty(s_shape, dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _expect(state_out, "state_out", s_shape, torch.float32, dev)
+    lib = load_library()
+    _check(lib.gdn_forward_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+                               _ptr(beta), _ptr(decay), _ptr(state_in), _ptr(state_out), _ptr(o),
+                               B, H, T, dk, dv, GDN_BIDI if bidi else 0, _stream_handle(stream, dev)))
+    return o, state_out
 
 
 def gdn_rollout(q, k, v, beta, decay, state_in=None, *, recurrent=False, chunk_states=False,

@@ -149,3 +149,14 @@ def make_custom(B, H, T, dk, dv, dtype="bf16", seed=0, bidi=False, decay_shift=2
                   tokens_per_frame=tokens_per_frame, decay_shift=decay_shift,
                   state0=state0, seed=seed)
     return make_inputs(wl)
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-(batch, head) scaled fp8 E4M3 codes of a [B,H,T,d] tensor: scale =
+    max|x| / 448 over the head (1 for an all-zero head), codes = the nearest
+    E4M3 value of x / scale.  Returns (uint8 codes, fp32 scales [B,H])."""
+    xf = x.to(torch.float32)
+    amax = xf.abs().amax(dim=(2, 3))
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    codes = (xf / scale[:, :, None, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.contiguous()

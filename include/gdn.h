@@ -231,6 +231,27 @@ int gdn_forward_normalized(const void *q, const void *k, const void *v,
                            void *stream);
 
 /*
+ * gdn_forward_fp8 -- gdn_forward with fp8 (E4M3) q, k, v and one fp32 scale
+ * per (batch, head) for each (the flashdreams SANA-WM page, "Developer
+ * Details": FP8 inference on sm_90 and newer): the inputs are
+ * x = x_scale[b][h] * decode(x8), o is bf16.
+ *   q8, k8 [B,H,T,dk], v8 [B,H,T,dv]: E4M3 codes (one byte each);
+ *   q_scale, k_scale, v_scale [B,H] fp32;
+ *   beta, decay, state_in, state_out, o and mode as gdn_forward (o bf16;
+ *   GDN_CAUSAL or GDN_BIDI).
+ * dk = 128, dv in {64, 128}.  This version dequantises into bf16 workspace
+ * copies (stream-ordered, 2*B*H*T*(2*dk + dv) bytes) and runs the bf16
+ * chunkwise kernel on them: fp8 inputs are accepted, their bandwidth is not
+ * yet saved.  Errors: as gdn_forward; a NULL scale returns
+ * GDN_ERR_INVALID_ARG; GDN_FP32 or GDN_RECURRENT, GDN_ERR_UNSUPPORTED.
+ */
+int gdn_forward_fp8(const void *q8, const void *k8, const void *v8,
+                    const float *q_scale, const float *k_scale, const float *v_scale,
+                    const float *beta, const float *decay,
+                    const float *state_in, float *state_out, void *o,
+                    int B, int H, int T, int dk, int dv, int mode, void *stream);
+
+/*
  * gdn_device_status -- synchronises `stream` and reports (and clears) the
  * library's device-side error word: GDN_OK, or GDN_ERR_DEVICE_TIMEOUT if a
  * bounded wait inside a kernel gave up since the last call, or GDN_ERR_CUDA.

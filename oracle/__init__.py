@@ -4,5 +4,6 @@ Imported by tests/, __graft_entry__.smoke() and bench.py's CPU-baseline leg;
 never by the product package.
 """
 from .oracle import (  # noqa: F401
-    gdn_forward, gdn_forward_blockcausal, gdn_forward_normalized, gdn_rollout, load,
+    decode_e4m3, gdn_forward, gdn_forward_blockcausal, gdn_forward_fp8, gdn_forward_normalized, gdn_rollout,
+    load,
 )

@@ -133,3 +133,27 @@ def gdn_forward_normalized(q, k, v, beta, decay, state_in=None, state_z_in=None,
     z_in = None if state_z_in is None else _f64(state_z_in)[..., None]
     den, s_z = gdn_forward(q, k, ones, beta, decay, state_in=z_in, bidi=bidi, n_threads=n_threads)
     return num / (den + eps), s_kv, s_z[..., 0]
+
+
+def decode_e4m3(codes):
+    """fp8 E4M3 bytes -> float64 (test infrastructure only), from the format's
+    definition: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
+    exponent field 0 holds subnormals m/8 * 2^-6; S.1111.111 is NaN (no
+    infinities); the largest finite value is 448."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((e == 0xF) & (m == 7), np.nan, val)
+    return sign * val
+
+
+def gdn_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, beta, decay, state_in=None, bidi=False,
+                    n_threads=None):
+    """fp8 (E4M3) q, k, v with one fp32 scale per (batch, head) (test
+    infrastructure only): the inputs are x = scale * decode(x8), exactly, and
+    the recurrence is gdn_forward on them."""
+    deq = lambda x8, s: decode_e4m3(x8) * np.asarray(s, dtype=np.float64)[:, :, None, None]
+    return gdn_forward(deq(q8, q_scale), deq(k8, k_scale), deq(v8, v_scale), beta, decay,
+                       state_in=state_in, bidi=bidi, n_threads=n_threads)

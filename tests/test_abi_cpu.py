@@ -28,6 +28,7 @@ def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_forward_noalloc",
               "gdn_forward_segmented", "gdn_forward_blockcausal", "gdn_forward_normalized",
+              "gdn_forward_fp8",
               "gdn_device_status",
               "gdn_kernel_launches",
               "gdn_last_error", "gdn_version"):
@@ -155,3 +156,14 @@ def test_normalized_rejects_before_launch(lib):
     assert f(dk=64) == -2
     assert f(zin=PM) == -3 and b"state_z" in lib.gdn_last_error()
     assert f(zout=PM) == -3
+
+
+def test_fp8_rejects_before_launch(lib):
+    """The fp8 entry point needs its three scales and runs bf16-output chunkwise
+    shapes only; each refusal happens before any CUDA call."""
+    f = lambda sq=P, dk=128, dv=128, mode=0: lib.gdn_forward_fp8(
+        P, P, P, sq, P, P, P, P, None, None, P, 1, 1, 640, dk, dv, mode, None)
+    assert f(sq=None) == -1 and b"scale" in lib.gdn_last_error()
+    assert f(mode=2) == -2
+    assert f(mode=4) == -2
+    assert f(dk=64) == -2

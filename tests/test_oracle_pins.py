@@ -20,6 +20,9 @@ by closed forms and brute force instead:
   with orthonormal keys = its closed form; tiny cases by brute force;
 * the normalised read-out: its closed form with orthonormal keys, z against its
   written-out recurrence, linearity in v, the bidirectional sums;
+* fp8 inputs: the E4M3 decoder against the format's fixed codes and torch's
+  float8 type for all 256 codes; the fp8 entry = the forward on exact
+  dequantised inputs;
 * the contraction bound ||H_t|| <= a_t ||H_{t-1}|| + b_t ||v_t|| for unit keys.
 Each pin is chosen so that a dropped term, a wrong sign or index, or a
 transposed state would fail at least one of them.
@@ -383,6 +386,47 @@ def test_normalized_bidi_sums_numerators_and_denominators(oracle_mod):
     den, _ = oracle_mod.gdn_forward(q, k, np.ones(v.shape[:3] + (1,)), b, a, bidi=True)
     np.testing.assert_array_equal(o, num / (den + eps))
     assert s_z.shape == (2, 1, 2, 6)
+
+
+# ----------------------------------------------------------------------------
+# fp8 (E4M3) inputs
+# ----------------------------------------------------------------------------
+
+def test_e4m3_decoder_known_codes(oracle_mod):
+    """Codes fixed by the format: 1.0, -2.0, the largest finite value 448, the
+    smallest subnormal 2^-9, the largest subnormal 7/8 * 2^-6, 0.5, zero, NaN."""
+    codes = [0x38, 0xC0, 0x7E, 0x01, 0x07, 0x30, 0x00, 0x7F, 0xFF]
+    ref = [1.0, -2.0, 448.0, 2.0 ** -9, 7 / 8 * 2.0 ** -6, 0.5, 0.0]
+    got = oracle_mod.decode_e4m3(codes)
+    np.testing.assert_array_equal(got[:7], ref)
+    assert np.isnan(got[7]) and np.isnan(got[8])
+
+
+def test_e4m3_decoder_matches_torch_float8_for_every_code(oracle_mod):
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle_mod.decode_e4m3(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    np.testing.assert_array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+
+
+def test_fp8_forward_is_the_forward_on_dequantised_inputs(oracle_mod):
+    """With power-of-two scales the dequantised values are exact, so the fp8
+    entry equals gdn_forward on them bitwise; a per-head scale of v scales o."""
+    rng = np.random.default_rng(77)
+    B, H, T, dk, dv = 1, 2, 20, 8, 4
+    q8, k8, v8 = (rng.integers(0, 0x7E, (B, H, T, d), dtype=np.uint8) for d in (dk, dk, dv))
+    sq, sk, sv = (np.full((B, H), 2.0 ** -6) for _ in range(3))
+    b = rng.uniform(0, 1, (B, H, T))
+    a = rng.uniform(0.5, 1, (B, H, T))
+    o, s = oracle_mod.gdn_forward_fp8(q8, k8, v8, sq, sk, sv, b, a)
+    dq = lambda x: oracle_mod.decode_e4m3(x) * 2.0 ** -6
+    o_ref, s_ref = oracle_mod.gdn_forward(dq(q8), dq(k8), dq(v8), b, a)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(s, s_ref)
+    o2, _ = oracle_mod.gdn_forward_fp8(q8, k8, v8, sq, sk, 4 * sv, b, a)
+    np.testing.assert_allclose(o2, 4 * o, rtol=1e-12, atol=1e-14)
 
 
 def test_rollout_entry_equals_single_scan_bitwise(oracle_mod):
