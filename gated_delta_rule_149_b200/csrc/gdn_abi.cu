@@ -140,7 +140,7 @@ int gdn_rollout(const void *q, const void *k, const void *v, const float *beta,
 
         float *ws = nullptr;   // ping-pong states when the caller keeps none
         if (n_chunks > 1 && !chunk_states) {
-            cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * BH * st * sizeof(float),
+            cudaError_t e = gdn::ws_alloc(reinterpret_cast<void **>(&ws), 2 * BH * st * sizeof(float),
                                             stream);
             if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "workspace: %s", cudaGetErrorString(e));
         }
@@ -165,7 +165,7 @@ int gdn_rollout(const void *q, const void *k, const void *v, const float *beta,
             if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "state copy: %s", cudaGetErrorString(e));
         }
         if (ws) {
-            cudaError_t e = cudaFreeAsync(ws, stream);
+            cudaError_t e = gdn::ws_free(ws, stream);
             if (rc == GDN_OK && e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "workspace free: %s", cudaGetErrorString(e));
         }
         return rc == GDN_OK ? ok() : rc;
@@ -192,7 +192,7 @@ int gdn_forward_host(const void *q, const void *k, const void *v, const float *b
         const size_t total = 2 * up(nqk) + 2 * up(nv) + 2 * up(ng) + (state_in ? up(nst) : 0) +
                              (state_out ? up(nso) : 0);
         char *base = nullptr;
-        cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&base), total, stream);
+        cudaError_t e = gdn::ws_alloc(reinterpret_cast<void **>(&base), total, stream);
         if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device buffers: %s", cudaGetErrorString(e));
         char *p = base;
         auto take = [&p, &up](size_t n) { char *r = p; p += up(n); return r; };
@@ -218,7 +218,7 @@ int gdn_forward_host(const void *q, const void *k, const void *v, const float *b
                 e = cudaMemcpyAsync(state_out, dso, nso, cudaMemcpyDeviceToHost, stream);
             if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "device->host copy: %s", cudaGetErrorString(e));
         }
-        e = cudaFreeAsync(base, stream);
+        e = gdn::ws_free(base, stream);
         cudaError_t es2 = cudaStreamSynchronize(stream);
         if (rc == GDN_OK && (e != cudaSuccess || es2 != cudaSuccess))
             rc = fail(GDN_ERR_CUDA, "gdn_forward_host: %s",
@@ -389,6 +389,25 @@ int gdn_device_status(void *stream)
     cudaError_t e = gdn::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &err);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device status: %s", cudaGetErrorString(e));
     if (err) return fail(GDN_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (code %d)", err);
+    return ok();
+}
+
+int gdn_workspace_release(int device)
+{
+    cudaError_t e = gdn::ws_release(device);
+    if (e == cudaErrorInvalidDevice) return fail(GDN_ERR_INVALID_ARG, "no device %d", device);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "workspace release: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int gdn_workspace_reserved(int device, unsigned long long *bytes)
+{
+    if (!bytes) return fail(GDN_ERR_INVALID_ARG, "bytes must be non-NULL");
+    uint64_t v = 0;
+    cudaError_t e = gdn::ws_reserved(device, &v);
+    *bytes = v;
+    if (e == cudaErrorInvalidDevice) return fail(GDN_ERR_INVALID_ARG, "no device %d", device);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "workspace size: %s", cudaGetErrorString(e));
     return ok();
 }
 

@@ -1415,7 +1415,7 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
     if (err != cudaSuccess) return err;
     const size_t n_cnt = (size_t)BH * p.n_chunks * p.n_slices;
     if (a.bidi) {
-        err = cudaMallocAsync(reinterpret_cast<void **>(&p.counters), n_cnt * sizeof(int), stream);
+        err = ws_alloc(reinterpret_cast<void **>(&p.counters), n_cnt * sizeof(int), stream);
         if (err != cudaSuccess) return err;
         err = cudaMemsetAsync(p.counters, 0, n_cnt * sizeof(int), stream);
     }
@@ -1426,7 +1426,7 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
         if (err == cudaSuccess) count_launches(1);
     }
     if (p.counters) {
-        cudaError_t e2 = cudaFreeAsync(p.counters, stream);
+        cudaError_t e2 = ws_free(p.counters, stream);
         if (err == cudaSuccess) err = e2;
     }
     return err;

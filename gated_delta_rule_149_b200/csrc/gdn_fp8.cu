@@ -52,7 +52,7 @@ cudaError_t launch_fp8(const FwdArgs &a, const float *q_scale, const float *k_sc
     const size_t BH = (size_t)a.B * a.H, nk = BH * a.T * a.dk, nv = BH * a.T * a.dv;
     const size_t bq = align_up256(nk * 2), bv = align_up256(nv * 2);
     uint8_t *ws = nullptr;
-    cudaError_t err = cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * bq + bv, stream);
+    cudaError_t err = ws_alloc(reinterpret_cast<void **>(&ws), 2 * bq + bv, stream);
     if (err != cudaSuccess) return err;
     auto *q = reinterpret_cast<__nv_bfloat16 *>(ws);
     auto *k = reinterpret_cast<__nv_bfloat16 *>(ws + bq);
@@ -74,7 +74,7 @@ cudaError_t launch_fp8(const FwdArgs &a, const float *q_scale, const float *k_sc
         b.v = v;
         err = launch_chunk_tc(b, stream);
     }
-    const cudaError_t e2 = cudaFreeAsync(ws, stream);
+    const cudaError_t e2 = ws_free(ws, stream);
     return err != cudaSuccess ? err : e2;
 }
 

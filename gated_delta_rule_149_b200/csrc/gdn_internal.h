@@ -59,6 +59,14 @@ cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *
 cudaError_t launch_fp8(const FwdArgs &a, const float *q_scale, const float *k_scale, const float *v_scale,
                        cudaStream_t stream);
 
+// Scratch memory: stream-ordered allocations from the library's own pool on
+// the current device, which keeps its reservation across synchronisations;
+// ws_release trims it to nothing, ws_reserved reads its size.
+cudaError_t ws_alloc(void **ptr, size_t bytes, cudaStream_t stream);
+cudaError_t ws_free(void *ptr, cudaStream_t stream);
+cudaError_t ws_release(int dev);
+cudaError_t ws_reserved(int dev, uint64_t *bytes);
+
 // Device-side error word (set by bounded waits that gave up).
 cudaError_t device_error_word(int **ptr);
 

@@ -148,7 +148,7 @@ cudaError_t launch_typed(const FwdArgs &a, cudaStream_t stream)
     const size_t n_out = (size_t)p.BH * a.T * a.dv;
     cudaError_t err = cudaSuccess;
     if (a.bidi) {
-        err = cudaMallocAsync(reinterpret_cast<void **>(&p.part), 2 * n_out * sizeof(float), stream);
+        err = ws_alloc(reinterpret_cast<void **>(&p.part), 2 * n_out * sizeof(float), stream);
         if (err != cudaSuccess) return err;
     }
     dim3 grid(p.BH, a.bidi ? 2 : 1);
@@ -170,7 +170,7 @@ cudaError_t launch_typed(const FwdArgs &a, cudaStream_t stream)
             err = cudaGetLastError();
             if (err == cudaSuccess) count_launches(1);
         }
-        cudaError_t e2 = cudaFreeAsync(p.part, stream);
+        cudaError_t e2 = ws_free(p.part, stream);
         if (err == cudaSuccess) err = e2;
     }
     return err;

@@ -162,7 +162,7 @@ cudaError_t launch_segmented(const FwdArgs &a, int n_segments, cudaStream_t stre
     const size_t b_pin = align_up(nP * pz * 4), b_pout = b_pin;
     const size_t b_vz = align_up(BH * (size_t)a.T * a.dk * 2), b_ow = b_vz;
     uint8_t *ws = nullptr;
-    cudaError_t err = cudaMallocAsync(reinterpret_cast<void **>(&ws),
+    cudaError_t err = ws_alloc(reinterpret_cast<void **>(&ws),
                                       b_sin + b_l + b_e + b_f + b_pin + b_pout + b_vz + b_ow, stream);
     if (err != cudaSuccess) return err;
     float *Sin = reinterpret_cast<float *>(ws);
@@ -246,7 +246,7 @@ cudaError_t launch_segmented(const FwdArgs &a, int n_segments, cudaStream_t stre
     if (err == cudaSuccess && a.state_out)
         err = cudaMemcpy2DAsync(a.state_out, sz * 4, Fst + (size_t)(S - 2) * sz, (S - 1) * sz * 4, sz * 4, BH,
                                 cudaMemcpyDeviceToDevice, stream);
-    const cudaError_t e2 = cudaFreeAsync(ws, stream);
+    const cudaError_t e2 = ws_free(ws, stream);
     return err != cudaSuccess ? err : e2;
 }
 
@@ -273,7 +273,7 @@ cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream)
     const size_t b_st = align_up(BHF * sz * 4), b_p = align_up(BHF * pz * 4);
     const size_t b_vz = align_up(ntok * a.dk * 2), b_g = align_up(ntok * 4);
     uint8_t *ws = nullptr;
-    cudaError_t err = cudaMallocAsync(reinterpret_cast<void **>(&ws), 3 * b_st + 2 * b_p + 2 * b_vz + 2 * b_g, stream);
+    cudaError_t err = ws_alloc(reinterpret_cast<void **>(&ws), 3 * b_st + 2 * b_p + 2 * b_vz + 2 * b_g, stream);
     if (err != cudaSuccess) return err;
     float *Sin = reinterpret_cast<float *>(ws);
     float *Lst = reinterpret_cast<float *>(ws + b_st);
@@ -358,7 +358,7 @@ cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream)
     if (err == cudaSuccess && a.state_out)
         err = cudaMemcpy2DAsync(a.state_out, sz * 4, Est + (size_t)(F - 1) * sz, F * sz * 4, sz * 4, BH,
                                 cudaMemcpyDeviceToDevice, stream);
-    const cudaError_t e2 = cudaFreeAsync(ws, stream);
+    const cudaError_t e2 = ws_free(ws, stream);
     return err != cudaSuccess ? err : e2;
 }
 
@@ -417,7 +417,7 @@ cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *
     const size_t b_ones = align_up(ntok * 64 * 2), b_den = b_ones;
     const size_t b_zin = align_up(BH * a.dk * 64 * 4), b_zout = align_up(ndir * BH * a.dk * 64 * 4);
     uint8_t *ws = nullptr;
-    cudaError_t err = cudaMallocAsync(reinterpret_cast<void **>(&ws), b_ones + b_den + b_zin + b_zout, stream);
+    cudaError_t err = ws_alloc(reinterpret_cast<void **>(&ws), b_ones + b_den + b_zin + b_zout, stream);
     if (err != cudaSuccess) return err;
     auto *ones = reinterpret_cast<__nv_bfloat16 *>(ws);
     auto *den = reinterpret_cast<__nv_bfloat16 *>(ws + b_ones);
@@ -475,7 +475,7 @@ cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *
     // z out: column 0 of every [dk][64] state
     if (err == cudaSuccess && state_z_out)
         err = cudaMemcpy2DAsync(state_z_out, 4, zout, 64 * 4, 4, ndir * BH * a.dk, cudaMemcpyDeviceToDevice, stream);
-    const cudaError_t e2 = cudaFreeAsync(ws, stream);
+    const cudaError_t e2 = ws_free(ws, stream);
     return err != cudaSuccess ? err : e2;
 }
 

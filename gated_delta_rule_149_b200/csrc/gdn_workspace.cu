@@ -1,0 +1,87 @@
+// Stream-ordered scratch memory of the library's calls.
+//
+// Every call that needs scratch (bidirectional arrival counters, fp8
+// dequantised copies, segment states and transitions, the normaliser pass,
+// rollout state ping-pong, the staging buffers of gdn_forward_host) takes it
+// from one memory pool per device that the library owns.  That pool keeps
+// what it has reserved across synchronisations (unlimited release threshold),
+// so a steady loop of calls maps device memory once.  CUDA's default pool
+// instead hands reserved memory back to the driver at every synchronise, and
+// the next call pays to map it again (a two-step timed loop of fp8 calls over
+// 2x16 heads and 75,600 tokens, 1.9 GB of dequantised copies, measured 221 ms
+// per step on a B200 against 5.5 ms of kernel time).
+// gdn_workspace_release() trims the pool; gdn_workspace_reserved() reads it.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kMaxPoolDev = 64;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxPoolDev] = {};
+
+// The pool of device `dev`, created on first use when `create` is set (else
+// *out stays nullptr until some call has created it).
+cudaError_t pool_of(int dev, bool create, cudaMemPool_t *out)
+{
+    *out = nullptr;
+    if (dev < 0 || dev >= kMaxPoolDev) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    if (!g_pool[dev] && create) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p = nullptr;
+        cudaError_t err = cudaMemPoolCreate(&p, &props);
+        if (err != cudaSuccess) return err;
+        uint64_t keep = UINT64_MAX;
+        err = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (err != cudaSuccess) {
+            cudaMemPoolDestroy(p);
+            return err;
+        }
+        g_pool[dev] = p;
+    }
+    *out = g_pool[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t ws_alloc(void **ptr, size_t bytes, cudaStream_t stream)
+{
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    cudaMemPool_t pool = nullptr;
+    if (err == cudaSuccess) err = pool_of(dev, true, &pool);
+    if (err == cudaSuccess) err = cudaMallocFromPoolAsync(ptr, bytes, pool, stream);
+    return err;
+}
+
+cudaError_t ws_free(void *ptr, cudaStream_t stream) { return cudaFreeAsync(ptr, stream); }
+
+cudaError_t ws_release(int dev)
+{
+    cudaMemPool_t pool = nullptr;
+    cudaError_t err = pool_of(dev, false, &pool);
+    if (err == cudaSuccess && pool) err = cudaMemPoolTrimTo(pool, 0);
+    return err;
+}
+
+cudaError_t ws_reserved(int dev, uint64_t *bytes)
+{
+    *bytes = 0;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t err = pool_of(dev, false, &pool);
+    if (err == cudaSuccess && pool) err = cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReservedMemCurrent, bytes);
+    return err;
+}
+
+}  // namespace gdn

@@ -67,6 +67,10 @@ def load_library():
         lib.gdn_version.restype = i
         lib.gdn_kernel_launches.argtypes = []
         lib.gdn_kernel_launches.restype = ctypes.c_longlong
+        lib.gdn_workspace_release.argtypes = [i]
+        lib.gdn_workspace_release.restype = i
+        lib.gdn_workspace_reserved.argtypes = [i, ctypes.POINTER(ctypes.c_ulonglong)]
+        lib.gdn_workspace_reserved.restype = i
         _lib = lib
     return _lib
 
@@ -323,3 +327,25 @@ def gdn_device_status(stream=None, device=None):
     """Synchronises the stream and raises GDNError if a bounded device wait gave up."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     _check(load_library().gdn_device_status(_stream_handle(stream, dev)))
+
+
+def _device_index(device):
+    if device is None:
+        return torch.cuda.current_device()
+    if isinstance(device, int):
+        return device
+    d = torch.device(device)
+    return torch.cuda.current_device() if d.index is None else d.index
+
+
+def gdn_workspace_release(device=None):
+    """Returns the library's reserved workspace memory on `device` (default: the
+    current CUDA device) to the driver; synchronise its streams first."""
+    _check(load_library().gdn_workspace_release(_device_index(device)))
+
+
+def gdn_workspace_reserved(device=None):
+    """Bytes of device memory the library's workspace pool on `device` holds."""
+    v = ctypes.c_ulonglong(0)
+    _check(load_library().gdn_workspace_reserved(_device_index(device), ctypes.byref(v)))
+    return v.value

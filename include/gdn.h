@@ -36,8 +36,10 @@
  * caller (except gdn_forward_host, which takes host memory).  Calls enqueue
  * work on `stream` (a cudaStream_t; NULL = the legacy default stream) and
  * return without synchronising.  Temporary workspace is taken stream-ordered
- * (cudaMallocAsync / cudaFreeAsync on `stream`); nothing persists between
- * calls.  state_in == state_out is allowed.  Inputs must not overlap outputs
+ * on `stream` from a memory pool the library keeps per device; the pool holds
+ * on to what it has reserved between calls (so a loop of calls maps device
+ * memory once) until gdn_workspace_release().  No other state persists
+ * between calls.  state_in == state_out is allowed.  Inputs must not overlap outputs
  * otherwise.
  *
  * Errors: every call returns GDN_OK (0) or a negative code below, and records
@@ -263,6 +265,21 @@ const char *gdn_last_error(void);
 
 /* ABI version: major * 10000 + minor * 100 + patch. */
 int gdn_version(void);
+
+/*
+ * gdn_workspace_release -- returns to the driver the device memory that the
+ * library's workspace pool on `device` holds in reserve (all of it once every
+ * call on that device has completed: synchronise first).  Later calls reserve
+ * again as they need.  GDN_OK also when the pool was never used;
+ * GDN_ERR_INVALID_ARG for a device index outside [0, 64); GDN_ERR_CUDA if the
+ * driver refuses.
+ *
+ * gdn_workspace_reserved -- writes to *bytes the device memory that pool now
+ * reserves (0 if never used).  GDN_ERR_INVALID_ARG for a NULL `bytes` or a bad
+ * device index.
+ */
+int gdn_workspace_release(int device);
+int gdn_workspace_reserved(int device, unsigned long long *bytes);
 
 /*
  * gdn_kernel_launches -- number of CUDA kernels this library has launched in

@@ -30,7 +30,7 @@ def test_header_declares_the_abi():
               "gdn_forward_segmented", "gdn_forward_blockcausal", "gdn_forward_normalized",
               "gdn_forward_fp8",
               "gdn_device_status",
-              "gdn_kernel_launches",
+              "gdn_kernel_launches", "gdn_workspace_release", "gdn_workspace_reserved",
               "gdn_last_error", "gdn_version"):
         assert n in names
 
@@ -167,3 +167,16 @@ def test_fp8_rejects_before_launch(lib):
     assert f(mode=2) == -2
     assert f(mode=4) == -2
     assert f(dk=64) == -2
+
+
+def test_workspace_calls_validate_and_start_empty(lib):
+    """Bad device indices and a NULL out-pointer are rejected before any CUDA
+    call; a pool no call has used reports 0 bytes and releases as a no-op."""
+    v = ctypes.c_ulonglong(123)
+    for dev in (-1, 64):
+        assert lib.gdn_workspace_reserved(dev, ctypes.byref(v)) == -1
+        assert lib.gdn_workspace_release(dev) == -1
+    assert lib.gdn_workspace_reserved(0, None) == -1
+    assert lib.gdn_workspace_reserved(0, ctypes.byref(v)) == 0 and v.value == 0
+    assert lib.gdn_workspace_release(0) == 0
+
