@@ -99,17 +99,68 @@ def recorded_traffic(workload, sha):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
+    """SM clock and clock-event (throttle) reasons during the timed region.
+
+    An NVML thread polls every 5 ms (read-only queries) and has taken its first
+    sample before the region starts, so short regions are covered too;
+    nvidia-smi is the fallback where NVML cannot be loaded."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+            "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, device=None):
         self.gpu = gpu_index
+        self.device = device
         self.proc = None
         self.f = None
+        self.thread = None
+        self.samples = []
+        self.max_mhz = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.device if self.device is not None else self.gpu)
+            bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _start_nvml(self):
+        import threading
+        nv, h = self._nvml_handle()
+        self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        self._stop, first = threading.Event(), threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                         int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                except Exception:
+                    break
+                first.set()
+                self._stop.wait(0.005)
+            first.set()
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+        first.wait(2.0)
+        if not self.samples:
+            raise RuntimeError("NVML gave no sample")
 
     def __enter__(self):
+        try:
+            self._start_nvml()
+            return self
+        except Exception:
+            self.thread = None
+            self.samples = []
         try:
             self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
@@ -121,6 +172,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=2.0)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -129,13 +183,18 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        if self.thread is not None:
+            if not self.samples:
+                return None
+            reasons = sorted(n for n in self.NAMES if any(r & self.BITS[n] for _, r in self.samples))
+            return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                    "reasons": reasons, "samples": len(self.samples), "source": "nvml, 5 ms"}
         if self.f is None:
             return None
         self.f.flush()
         rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
         os.unlink(self.f.name)
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             r = [x.strip() for x in r]
             if len(r) < 9:
@@ -145,13 +204,13 @@ class ClockSampler:
                 mx = float(r[2])
             except ValueError:
                 continue
-            for n, val in zip(names, r[5:9]):
+            for n, val in zip(self.NAMES, r[5:9]):
                 if val.lower() in ("active", "1"):
                     reasons.add(n)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi"}
 
 
 def dist_setup():
@@ -346,7 +405,7 @@ def run_gpu(args, world, rank, local):
           for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, dev) as clk:
         t_all0 = torch.cuda.Event(enable_timing=True)
         t_all1 = torch.cuda.Event(enable_timing=True)
         t_all0.record(stream)

@@ -590,19 +590,33 @@ __device__ __forceinline__ void tma_role(const Ctx &x, const CUtensorMap *tmQ, c
 }
 
 // ------------------------------------------------------------------ MMA warps
-// (Issue loops are not unrolled: the issuing threads are not the limit, and
-// small loop bodies leave more of the instruction cache to the epilogues.)
+// An issuing thread shares its SM sub-partition's issue slots with four busy
+// epilogue warps, so every instruction between two MMAs stretches the MMA
+// stream: each product is one unrolled run of MMAs whose operand descriptors
+// are a base descriptor plus an immediate (the 14-bit start-address field,
+// in 16-byte units, holds any shared-memory address, so adding to the
+// descriptor never carries out of it); loop-invariant bases are built once.
 // Two issuing threads, each waiting (suspended) on its next products' inputs in
 // a fixed order: one for the state-independent products of the prep pipeline,
 // one for the serial-chain products.  tcgen05.commit tracks the MMAs of the
 // issuing thread only; the mbarrier protocol orders the two streams.
+
+// N MMAs of one product into d: the operand descriptors advance by A_STEP and
+// B_STEP (16-byte units) per K step; the first MMA overwrites D unless acc.
+template <int N, uint32_t A_STEP, uint32_t B_STEP>
+__device__ __forceinline__ void mma_run(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, bool acc)
+{
+#pragma unroll
+    for (int k = 0; k < N; ++k)
+        mma_bf16(d, a + (uint64_t)(k * A_STEP), b + (uint64_t)(k * B_STEP), idesc, (k > 0 || acc) ? 1u : 0u);
+}
 
 // [Q;K] K^T, then W^T = K^T T1^T and U~ = T2 V, chunk after chunk.
 __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
 {
     Bars &B = *x.bars;
     const uint32_t tm = x.tmem;
-    const uint32_t sT1 = x.sbase + kOffT1, sT2 = x.sbase + kOffT2;
+    const uint64_t dT1 = sw128_desc(x.sbase + kOffT1, 16, 1024), dT2 = sw128_desc(x.sbase + kOffT2, 16, 1024);
     PROF_DECL(true);
     // [Q;K] K^T of chunk j (needs its stage loaded and D1 read out for chunk j-1)
     auto issue_m1 = [&](int j) -> bool {
@@ -611,13 +625,10 @@ __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
         if (j > 0 && !wait_bar(&B.d1_empty, (j - 1) & 1, x.abort_flag, p.err, 12)) return false;
         PROF_MARK(2);
         const uint32_t sQK = stage_addr(x, j);
+        const uint64_t a = sw128_desc(sQK, 16, 1024), b = sw128_desc(sQK + 8192, 16, 1024);
         tc_fence_after();
-#pragma unroll 1
-        for (int kb = 0; kb < 2; ++kb)
-#pragma unroll 1
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + kColD1, sw128_desc(sQK + kb * 16384 + ks * 32, 16, 1024),
-                         sw128_desc(sQK + kb * 16384 + 8192 + ks * 32, 16, 1024), kIdM1, (kb | ks) != 0);
+        mma_run<4, 2, 2>(tm + kColD1, a, b, kIdM1, false);                  // K block 0
+        mma_run<4, 2, 2>(tm + kColD1, a + 1024, b + 1024, kIdM1, true);     // K block 1 (+16 KB)
         mma_commit(&B.d1_full);
         PROF_MARK(6);
         return true;
@@ -636,16 +647,11 @@ __device__ __forceinline__ void mma_prep_role(const Ctx &x, const TcParams &p)
         if (i >= 2 && !wait_bar(&B.du_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 14)) break;
         if (i >= 1 && !wait_bar(&B.dw_empty, (i - 1) & 1, x.abort_flag, p.err, 19)) break;
         PROF_MARK(7);
-        const uint32_t sQK = stage_addr(x, i), sV = sQK + 32768;
+        const uint32_t sQK = stage_addr(x, i);
+        const uint64_t dKmn = sw128_desc(sQK + 8192, 16384, 1024), dVmn = sw128_desc(sQK + 32768, 8192, 1024);
         tc_fence_after();
-#pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tm + kColW, sw128_desc(sQK + 8192 + ks * 2048, 16384, 1024),
-                     sw128_desc(sT1 + ks * 32, 16, 1024), kIdW, ks != 0);
-#pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sT2 + ks * 32, 16, 1024),
-                     sw128_desc(sV + ks * 2048, 8192, 1024), kIdUt, ks != 0);
+        mma_run<4, 128, 2>(tm + kColW, dKmn, dT1, kIdW, false);
+        mma_run<4, 2, 128>(tm + kColU0 + 64 * b, dT2, dVmn, kIdUt, false);
         mma_commit(&B.wu_full);
         PROF_MARK(5);
     }
@@ -661,8 +667,9 @@ __device__ __forceinline__ void mma_chain_role(const Ctx &x, const TcParams &p)
 {
     Bars &B = *x.bars;
     const uint32_t tm = x.tmem;
-    const uint32_t sP = x.sbase + kOffP, sW = x.sbase + kOffW, sU = x.sbase + kOffU;
-    const uint32_t sUb = x.sbase + kOffUb, sH = x.sbase + kOffH;
+    const uint64_t dP = sw128_desc(x.sbase + kOffP, 16, 1024), dW = sw128_desc(x.sbase + kOffW, 8192, 1024);
+    const uint64_t dU = sw128_desc(x.sbase + kOffU, 8192, 1024), dUb = sw128_desc(x.sbase + kOffUb, 8192, 1024);
+    const uint64_t dH = sw128_desc(x.sbase + kOffH, 8192, 1024);
     PROF_DECL(true);
     for (int i = 0; i < x.NC; ++i) {
         const int b = i & 1;
@@ -673,31 +680,19 @@ __device__ __forceinline__ void mma_chain_role(const Ctx &x, const TcParams &p)
         if (!wait_bar(&B.h_full, i & 1, x.abort_flag, p.err, 16)) break;
         if (i >= 2 && !wait_bar(&B.do_empty[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 17)) break;
         PROF_MARK(29);
+        const uint64_t dQ = sw128_desc(sQK, 16, 1024);
         tc_fence_after();
-#pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks)
-            mma_bf16(tm + kColU0 + 64 * b, sw128_desc(sW + ks * 2048, 8192, 1024),
-                     sw128_desc(sH + ks * 2048, 8192, 1024), kIdUc, 1);
+        mma_run<8, 128, 128>(tm + kColU0 + 64 * b, dW, dH, kIdUc, true);
         mma_commit(&B.chain_full);
-#pragma unroll 1
-        for (int kb = 0; kb < 2; ++kb)
-#pragma unroll 1
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + kColO0 + 64 * b, sw128_desc(sQK + kb * 16384 + ks * 32, 16, 1024),
-                         sw128_desc(sH + (kb * 4 + ks) * 2048, 8192, 1024), kIdOq, (kb | ks) != 0);
+        mma_run<4, 2, 128>(tm + kColO0 + 64 * b, dQ, dH, kIdOq, false);               // K block 0
+        mma_run<4, 2, 128>(tm + kColO0 + 64 * b, dQ + 1024, dH + 512, kIdOq, true);   // K block 1
         PROF_MARK(4);
         if (!wait_bar(&B.u_full, i & 1, x.abort_flag, p.err, 18)) break;
         PROF_MARK(30);
         tc_fence_after();
-#pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tm + kColS, sw128_desc(sQK + 8192 + ks * 2048, 16384, 1024),
-                     sw128_desc(sUb + ks * 2048, 8192, 1024), kIdS, ks != 0);
+        mma_run<4, 128, 128>(tm + kColS, sw128_desc(sQK + 8192, 16384, 1024), dUb, kIdS, false);
         mma_commit(&B.s_full);
-#pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tm + kColO0 + 64 * b, sw128_desc(sP + b * 8192 + ks * 32, 16, 1024),
-                     sw128_desc(sU + ks * 2048, 8192, 1024), kIdPU, 1);
+        mma_run<4, 2, 128>(tm + kColO0 + 64 * b, dP + (uint64_t)(b * 512), dU, kIdPU, true);
         mma_commit(&B.o_full[b]);
         mma_commit(&B.p_empty[b]);
         mma_commit(&B.stage_empty[i % kNS]);
