@@ -425,7 +425,8 @@ def run_gpu(args, world, rank, local):
     total_ms = t_all0.elapsed_time(t_all1) if flush_buf is None else sum(per_call)
     ms_per_step, value = replica_throughput(wl.token_heads, total_ms, args.steps, world)
 
-    # roofline of the main kernel (the call is one main kernel plus a tiny memset)
+    # roofline of the main kernel (the plain call is one main kernel plus a tiny
+    # memset; the other forms time their whole call, which "scope" says)
     hbm_peak, tc_peak, peak_kind = load_peaks()
     call_s = statistics.mean(per_call) * 1e-3
     achieved = bytes_ / call_s / 1e9
@@ -434,6 +435,12 @@ def run_gpu(args, world, rank, local):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": traffic,
                 "peak_kind": peak_kind, "algorithmic_bytes": bytes_,
+                "scope": ("the token-by-token kernel (and, bidirectional, the add of its partials)"
+                          if recurrent else
+                          "the chunkwise kernel (the call's one kernel)" if not segmented else
+                          "the whole call: the bf16 kernel's algorithmic bytes over the time of all "
+                          "its launches (%s)" % ("dequantising pre-pass included" if args.fp8 else
+                                                 "every pass and combine included")),
                 "tensor_tflops": algorithmic_flops(wl) / call_s / 1e12,
                 "tensor_frac": algorithmic_flops(wl) / call_s / 1e12 / tc_peak,
                 "kernel_source_sha": sha}
