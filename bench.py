@@ -15,12 +15,16 @@ scans are independent, there is no collective on the data path (weak scaling).
 Also measured, and printed on the same JSON line:
   e2e          the same metric through the library's host-buffer entry point
                (pinned host inputs; host->device copies, the kernels, and the
-               device->host copy of o and the states inside the timed region);
+               device->host copy of o and the states inside the timed region),
+               as a streaming loop runs it: asynchronous calls alternating
+               between two streams, so call i+1's copies in overlap call i's
+               kernels and copies out;
   roofline     the main kernel's algorithmic bytes / its average event-timed
                duration, against the measured HBM copy bandwidth;
   cpu_baseline the fp64 CPU oracle on a bounded sample of the same workload
                (rank 0, N = 1 only);
-  clocks       nvidia-smi samples taken during the timed region.
+  clocks       SM clock and throttle reasons sampled (NVML) during the timed
+               region.
 --impl reference times the CPU oracle alone (the reference arm of this build:
 there is no upstream code to run).
 """
@@ -345,7 +349,7 @@ def run_reference(args, world, rank):
 def run_gpu(args, world, rank, local):
     import torch
     from gated_delta_rule_149_b200 import (gdn, gdn_forward, gdn_forward_blockcausal, gdn_forward_fp8,
-                                           gdn_forward_host, gdn_forward_normalized, gdn_forward_segmented,
+                                           gdn_forward_host_async, gdn_forward_normalized, gdn_forward_segmented,
                                            gdn_device_status)
     from gated_delta_rule_149_b200.inputs import quantize_e4m3
     from gated_delta_rule_149_b200.inputs import WORKLOADS, make_inputs
@@ -453,10 +457,14 @@ def run_gpu(args, world, rank, local):
         hq, hk, hv = map(pin, (inp.q, inp.k, inp.v))
     hb, ha = map(pin, (inp.beta, inp.decay))
     hs0 = None if inp.state0 is None else pin(inp.state0)
-    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    hso = torch.empty(s_out.shape, dtype=torch.float32).pin_memory()
+    # two sets of host outputs and two streams: a streaming loop keeps one call
+    # in flight while the next one's inputs upload
+    e2e_streams = [stream, torch.cuda.Stream(dev)]
+    hos = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
+    hsos = [torch.empty(s_out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
 
-    def e2e_step():
+    def e2e_step(n):
+        ho, hso = hos[n % 2], hsos[n % 2]
         if segmented:   # the same call on device copies of pinned host buffers
             pairs = ((hq, q8), (hk, k8), (hv, v8), (hsq, sq), (hsk, sk), (hsv, sv)) if args.fp8 else \
                 ((hq, q), (hk, k), (hv, v))
@@ -467,19 +475,27 @@ def run_gpu(args, world, rank, local):
             ho.copy_(o, non_blocking=True)
             hso.copy_(s_out, non_blocking=True)
         else:
-            gdn_forward_host(hq, hk, hv, hb, ha, hs0, bidi=wl.bidi, recurrent=recurrent, o=ho,
-                             state_out=hso, stream=stream)
+            gdn_forward_host_async(hq, hk, hv, hb, ha, hs0, bidi=wl.bidi, recurrent=recurrent, o=ho,
+                                   state_out=hso, stream=e2e_streams[n % 2])
 
-    e2e_steps = max(1, min(args.steps, 5))
-    e2e_step()
+    e2e_steps = max(2, min(args.steps, 6))
+    e2e_step(0)
+    e2e_step(1)
+    torch.cuda.synchronize()
+    gdn_device_status(stream)
     barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    e2e_streams[1].wait_event(e0)
+    for n in range(e2e_steps):
+        e2e_step(n)
+    joined = torch.cuda.Event()
+    joined.record(e2e_streams[1])
+    stream.wait_event(joined)
     e1.record(stream)
     torch.cuda.synchronize()
+    gdn_device_status(stream)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     nbytes = lambda *ts: sum(t.numel() * t.element_size() for t in ts if t is not None)
 
@@ -503,7 +519,9 @@ def run_gpu(args, world, rank, local):
             "e2e": {"value": world * wl.token_heads / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": nbytes(hq, hk, hv, hb, ha, hs0,
                                                  *((hsq, hsk, hsv) if args.fp8 else ())),
-                    "d2h_bytes_per_step": nbytes(ho, hso)},
+                    "d2h_bytes_per_step": nbytes(hos[0], hsos[0]),
+                    "calls": ("synchronous, one stream" if segmented else
+                              "gdn_forward_host_async on two alternating streams (2 calls in flight)")},
             "gpu_launches": int(launches),
             "roofline": roofline,
             "clocks": clk.summary()}

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/gdn.h"
 #include "gdn_internal.h"
@@ -94,6 +95,88 @@ int dispatch(const gdn::FwdArgs &a, int mode, cudaStream_t stream)
 
 size_t dtype_size(int mode) { return (mode & GDN_FP32) ? 4 : 2; }
 
+// The kernels of host-buffer calls on one device run one after another
+// whatever their streams: a bidirectional launch whose CTAs all fit on the GPU
+// counts on being resident at once, which two such launches side by side would
+// not be.  Each call's kernels wait for the previous call's (an event per
+// device) and record their own completion.
+constexpr int kMaxOrderDev = 64;
+std::mutex g_order_mu;
+cudaEvent_t g_order_ev[kMaxOrderDev] = {};
+
+int ordered_dispatch(const gdn::FwdArgs &a, int mode, cudaStream_t stream)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess && (dev < 0 || dev >= kMaxOrderDev)) e = cudaErrorInvalidDevice;
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device: %s", cudaGetErrorString(e));
+    std::lock_guard<std::mutex> lock(g_order_mu);
+    if (!g_order_ev[dev]) e = cudaEventCreateWithFlags(&g_order_ev[dev], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, g_order_ev[dev], 0);   // no-op before the first record
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "call order: %s", cudaGetErrorString(e));
+    const int rc = dispatch(a, mode, stream);
+    if (rc != GDN_OK) return rc;
+    e = cudaEventRecord(g_order_ev[dev], stream);
+    return e == cudaSuccess ? GDN_OK : fail(GDN_ERR_CUDA, "call order: %s", cudaGetErrorString(e));
+}
+
+// gdn_forward on host buffers: stage the inputs in pool memory, run, copy the
+// results back; `sync` waits for all of it before returning.
+int host_call(const void *q, const void *k, const void *v, const float *beta, const float *decay,
+              const float *state_in, float *state_out, void *o, int B, int H, int T, int dk, int dv,
+              int mode, void *stream_, bool sync, const char *name)
+{
+    try {
+        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
+                              mode, "T");
+        if (rc != GDN_OK) return rc;
+        cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+        const size_t BH = (size_t)B * H, es = dtype_size(mode);
+        const size_t nqk = BH * T * dk * es, nv = BH * T * dv * es, ng = BH * T * sizeof(float);
+        const size_t nst = BH * (size_t)dk * dv * sizeof(float);
+        const size_t nso = nst * ((mode & GDN_BIDI) ? 2 : 1);
+        // one device block, 256-byte aligned sub-buffers
+        auto up = [](size_t n) { return (n + 255) & ~(size_t)255; };
+        const size_t total = 2 * up(nqk) + 2 * up(nv) + 2 * up(ng) + (state_in ? up(nst) : 0) +
+                             (state_out ? up(nso) : 0);
+        char *base = nullptr;
+        cudaError_t e = gdn::ws_alloc(reinterpret_cast<void **>(&base), total, stream);
+        if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device buffers: %s", cudaGetErrorString(e));
+        char *p = base;
+        auto take = [&p, &up](size_t n) { char *r = p; p += up(n); return r; };
+        char *dq = take(nqk), *dk_ = take(nqk), *dv_ = take(nv), *dout = take(nv);
+        float *db = reinterpret_cast<float *>(take(ng)), *da = reinterpret_cast<float *>(take(ng));
+        float *dsi = state_in ? reinterpret_cast<float *>(take(nst)) : nullptr;
+        float *dso = state_out ? reinterpret_cast<float *>(take(nso)) : nullptr;
+
+        struct Cp { void *dst; const void *src; size_t n; };
+        const Cp h2d[] = {{dq, q, nqk}, {dk_, k, nqk}, {dv_, v, nv}, {db, beta, ng}, {da, decay, ng},
+                          {dsi, state_in, dsi ? nst : 0}};
+        for (const Cp &c : h2d)
+            if (c.n && e == cudaSuccess)
+                e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, stream);
+        if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "host->device copy: %s", cudaGetErrorString(e));
+        if (rc == GDN_OK) {
+            gdn::FwdArgs a = make_args(dq, dk_, dv_, db, da, dsi, dso, dout, B, H, T, dk, dv, mode);
+            rc = ordered_dispatch(a, mode, stream);
+        }
+        if (rc == GDN_OK) {
+            e = cudaMemcpyAsync(o, dout, nv, cudaMemcpyDeviceToHost, stream);
+            if (e == cudaSuccess && dso)
+                e = cudaMemcpyAsync(state_out, dso, nso, cudaMemcpyDeviceToHost, stream);
+            if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "device->host copy: %s", cudaGetErrorString(e));
+        }
+        e = gdn::ws_free(base, stream);
+        cudaError_t es2 = sync ? cudaStreamSynchronize(stream) : cudaSuccess;
+        if (rc == GDN_OK && (e != cudaSuccess || es2 != cudaSuccess))
+            rc = fail(GDN_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e != cudaSuccess ? e : es2));
+        return rc == GDN_OK ? ok() : rc;
+    } catch (...) {
+        return fail(GDN_ERR_CUDA, "internal error in %s", name);
+    }
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -176,57 +259,18 @@ int gdn_rollout(const void *q, const void *k, const void *v, const float *beta,
 
 int gdn_forward_host(const void *q, const void *k, const void *v, const float *beta,
                      const float *decay, const float *state_in, float *state_out, void *o,
-                     int B, int H, int T, int dk, int dv, int mode, void *stream_)
+                     int B, int H, int T, int dk, int dv, int mode, void *stream)
 {
-    try {
-        int rc = check_common(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv,
-                              mode, "T");
-        if (rc != GDN_OK) return rc;
-        cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-        const size_t BH = (size_t)B * H, es = dtype_size(mode);
-        const size_t nqk = BH * T * dk * es, nv = BH * T * dv * es, ng = BH * T * sizeof(float);
-        const size_t nst = BH * (size_t)dk * dv * sizeof(float);
-        const size_t nso = nst * ((mode & GDN_BIDI) ? 2 : 1);
-        // one device block, 256-byte aligned sub-buffers
-        auto up = [](size_t n) { return (n + 255) & ~(size_t)255; };
-        const size_t total = 2 * up(nqk) + 2 * up(nv) + 2 * up(ng) + (state_in ? up(nst) : 0) +
-                             (state_out ? up(nso) : 0);
-        char *base = nullptr;
-        cudaError_t e = gdn::ws_alloc(reinterpret_cast<void **>(&base), total, stream);
-        if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device buffers: %s", cudaGetErrorString(e));
-        char *p = base;
-        auto take = [&p, &up](size_t n) { char *r = p; p += up(n); return r; };
-        char *dq = take(nqk), *dk_ = take(nqk), *dv_ = take(nv), *dout = take(nv);
-        float *db = reinterpret_cast<float *>(take(ng)), *da = reinterpret_cast<float *>(take(ng));
-        float *dsi = state_in ? reinterpret_cast<float *>(take(nst)) : nullptr;
-        float *dso = state_out ? reinterpret_cast<float *>(take(nso)) : nullptr;
+    return host_call(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv, mode, stream, true,
+                     "gdn_forward_host");
+}
 
-        struct Cp { void *dst; const void *src; size_t n; };
-        const Cp h2d[] = {{dq, q, nqk}, {dk_, k, nqk}, {dv_, v, nv}, {db, beta, ng}, {da, decay, ng},
-                          {dsi, state_in, dsi ? nst : 0}};
-        for (const Cp &c : h2d)
-            if (c.n && e == cudaSuccess)
-                e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, stream);
-        if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "host->device copy: %s", cudaGetErrorString(e));
-        if (rc == GDN_OK) {
-            gdn::FwdArgs a = make_args(dq, dk_, dv_, db, da, dsi, dso, dout, B, H, T, dk, dv, mode);
-            rc = dispatch(a, mode, stream);
-        }
-        if (rc == GDN_OK) {
-            e = cudaMemcpyAsync(o, dout, nv, cudaMemcpyDeviceToHost, stream);
-            if (e == cudaSuccess && dso)
-                e = cudaMemcpyAsync(state_out, dso, nso, cudaMemcpyDeviceToHost, stream);
-            if (e != cudaSuccess) rc = fail(GDN_ERR_CUDA, "device->host copy: %s", cudaGetErrorString(e));
-        }
-        e = gdn::ws_free(base, stream);
-        cudaError_t es2 = cudaStreamSynchronize(stream);
-        if (rc == GDN_OK && (e != cudaSuccess || es2 != cudaSuccess))
-            rc = fail(GDN_ERR_CUDA, "gdn_forward_host: %s",
-                      cudaGetErrorString(e != cudaSuccess ? e : es2));
-        return rc == GDN_OK ? ok() : rc;
-    } catch (...) {
-        return fail(GDN_ERR_CUDA, "internal error in gdn_forward_host");
-    }
+int gdn_forward_host_async(const void *q, const void *k, const void *v, const float *beta,
+                           const float *decay, const float *state_in, float *state_out, void *o,
+                           int B, int H, int T, int dk, int dv, int mode, void *stream)
+{
+    return host_call(q, k, v, beta, decay, state_in, state_out, o, B, H, T, dk, dv, mode, stream, false,
+                     "gdn_forward_host_async");
 }
 
 int gdn_forward_noalloc(const void *q, const void *k, const void *v, const float *beta,

@@ -43,6 +43,12 @@ cudaError_t pool_of(int dev, bool create, cudaMemPool_t *out)
         if (err != cudaSuccess) return err;
         uint64_t keep = UINT64_MAX;
         err = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+        // A block freed on one stream is not handed to an allocation on another
+        // by making that stream wait (calls on two streams stay concurrent); it
+        // is reused once its free has completed, or through existing event order.
+        int no_hidden_waits = 0;
+        if (err == cudaSuccess)
+            err = cudaMemPoolSetAttribute(p, cudaMemPoolReuseAllowInternalDependencies, &no_hidden_waits);
         if (err != cudaSuccess) {
             cudaMemPoolDestroy(p);
             return err;

@@ -47,6 +47,8 @@ def load_library():
         lib.gdn_forward.restype = i
         lib.gdn_forward_host.argtypes = [vp] * 8 + [i] * 6 + [vp]
         lib.gdn_forward_host.restype = i
+        lib.gdn_forward_host_async.argtypes = [vp] * 8 + [i] * 6 + [vp]
+        lib.gdn_forward_host_async.restype = i
         lib.gdn_forward_noalloc.argtypes = [vp] * 8 + [i] * 6 + [vp]
         lib.gdn_forward_noalloc.restype = i
         lib.gdn_forward_segmented.argtypes = [vp] * 8 + [i] * 7 + [vp]
@@ -305,6 +307,21 @@ def gdn_forward_host(q, k, v, beta, decay, state_in=None, *, bidi=False, recurre
     """gdn_forward on CPU (ideally pinned) tensors through the library's host-buffer
     entry point: the library copies inputs in, runs, copies o/state back and
     synchronises.  Returns CPU tensors."""
+    return _host(False, q, k, v, beta, decay, state_in, bidi, recurrent, o, state_out, want_state,
+                 stream, device)
+
+
+def gdn_forward_host_async(q, k, v, beta, decay, state_in=None, *, bidi=False, recurrent=False,
+                           o=None, state_out=None, want_state=True, stream=None, device=None):
+    """gdn_forward_host without the final synchronise: returns once the copies
+    and kernels are enqueued on `stream`.  Keep every tensor alive and the
+    outputs unread until the stream has passed the call."""
+    return _host(True, q, k, v, beta, decay, state_in, bidi, recurrent, o, state_out, want_state,
+                 stream, device)
+
+
+def _host(asynchronous, q, k, v, beta, decay, state_in, bidi, recurrent, o, state_out, want_state,
+          stream, device):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     for name, t in (("q", q), ("k", k), ("v", v), ("beta", beta), ("decay", decay)):
@@ -317,9 +334,9 @@ def gdn_forward_host(q, k, v, beta, decay, state_in=None, *, bidi=False, recurre
         state_out = torch.empty(s_shape, dtype=torch.float32, pin_memory=q.is_pinned())
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     lib = load_library()
-    _check(lib.gdn_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay),
-                                _ptr(state_in), _ptr(state_out), _ptr(o), B, H, T, dk, dv,
-                                _mode(q, bidi, recurrent), _stream_handle(stream, dev)))
+    fn = lib.gdn_forward_host_async if asynchronous else lib.gdn_forward_host
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(state_in), _ptr(state_out),
+              _ptr(o), B, H, T, dk, dv, _mode(q, bidi, recurrent), _stream_handle(stream, dev)))
     return o, state_out
 
 

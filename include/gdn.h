@@ -112,14 +112,34 @@ int gdn_rollout(const void *q, const void *k, const void *v,
 /*
  * gdn_forward_host -- gdn_forward on HOST buffers (same layouts).  Copies the
  * inputs to the device, runs gdn_forward, copies o (and state_out if given)
- * back, and synchronises `stream` before returning.  Device buffers are taken
- * stream-ordered and released before return.  Pinned host memory gives
- * asynchronous copies; pageable memory works but is slower.
+ * back, and synchronises `stream` before returning.  Device buffers come
+ * stream-ordered from the library's workspace pool and go back to it in the
+ * same call.  Pinned host memory gives asynchronous copies; pageable memory
+ * works but is slower.
  */
 int gdn_forward_host(const void *q, const void *k, const void *v,
                      const float *beta, const float *decay,
                      const float *state_in, float *state_out, void *o,
                      int B, int H, int T, int dk, int dv, int mode, void *stream);
+
+/*
+ * gdn_forward_host_async -- gdn_forward_host without the final synchronise:
+ * the copies in, the kernels and the copies out are enqueued on `stream` and
+ * the call returns.  The caller keeps the host buffers alive and untouched
+ * (inputs unchanged, outputs unread) until `stream` has passed the call, e.g.
+ * by synchronising it or waiting on an event recorded after the call.  With
+ * pinned host memory, calls on two streams overlap one call's copies with the
+ * other's kernels: the streaming loop of a video pipeline, where chunk i+1 is
+ * uploaded while chunk i runs and downloads.  The kernels of host-buffer
+ * calls on one device run one after another whatever their streams (a
+ * bidirectional launch counts on having the GPU's SMs to itself).  Errors of
+ * the enqueued copies and kernels surface at the caller's synchronise;
+ * argument errors are returned as for gdn_forward.
+ */
+int gdn_forward_host_async(const void *q, const void *k, const void *v,
+                           const float *beta, const float *decay,
+                           const float *state_in, float *state_out, void *o,
+                           int B, int H, int T, int dk, int dv, int mode, void *stream);
 
 /*
  * gdn_forward_noalloc -- gdn_forward that allocates no device memory.

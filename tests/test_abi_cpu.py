@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_header_declares_the_abi():
     names = declared_functions()
-    for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_forward_noalloc",
+    for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_forward_host_async", "gdn_forward_noalloc",
               "gdn_forward_segmented", "gdn_forward_blockcausal", "gdn_forward_normalized",
               "gdn_forward_fp8",
               "gdn_device_status",
@@ -95,8 +95,10 @@ def test_rollout_rejects_bidi_and_bad_chunks(lib):
 
 
 def test_host_entry_validates_first(lib):
-    rc = lib.gdn_forward_host(None, P, P, P, P, None, None, P, 1, 1, 64, 128, 128, 0, None)
-    assert rc == -1
+    for fn in (lib.gdn_forward_host, lib.gdn_forward_host_async):
+        assert fn(None, P, P, P, P, None, None, P, 1, 1, 64, 128, 128, 0, None) == -1
+        assert fn(P, P, P, P, P, None, None, P, 1, 1, 0, 128, 128, 0, None) == -1
+        assert fn(P, P, P, P, P, None, None, PM, 1, 1, 64, 128, 128, 0, None) == -3
 
 
 def test_last_error_is_per_call(lib):
