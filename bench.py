@@ -21,6 +21,8 @@ Also measured, and printed on the same JSON line:
                kernels and copies out;
   roofline     the main kernel's algorithmic bytes / its average event-timed
                duration, against the measured HBM copy bandwidth;
+  parity       rel-L2 of the last timed step's o and states against the fp64
+               oracle on the first and last head, whole sequences (rank 0);
   cpu_baseline the fp64 CPU oracle on a bounded sample of the same workload
                (rank 0, N = 1 only);
   clocks       SM clock and throttle reasons sampled (NVML) during the timed
@@ -303,6 +305,53 @@ def oracle_sample_throughput(wl, inp=None, target_s=15.0):
             "elapsed_s": el, "cpu": _cpu_model()}
 
 
+def sampled_parity(args, wl, inp, o_dev, s_dev, fp8=None):
+    """rel-L2 of this run's GPU results (the last timed step's o and states)
+    against the fp64 oracle on the same inputs, for the first and the last
+    head over their whole sequences (both scan directions when bidirectional):
+    the check the timing is reported beside."""
+    import numpy as np
+    import oracle
+    if args.normalized:
+        return {"checked": False,
+                "why": "normalised read-out: z.q of the benchmark's signed features can be ~0; "
+                       "the GPU tests check it on non-negative features"}
+    BH = wl.B * wl.H
+    heads = sorted({0, BH - 1})
+    flat = lambda t: t.reshape(BH, *t.shape[2:])
+    pick = lambda t: flat(t)[heads].double().numpy()[None]          # [1, n, ...]
+    s0 = None if inp.state0 is None else pick(inp.state0)
+    nproc = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    if fp8 is not None:
+        q8, k8, v8, sq, sk, sv = (t.cpu() for t in fp8)
+        codes = lambda t: flat(t)[heads].numpy()[None]
+        scale = lambda t: t.reshape(BH)[heads].double().numpy()[None]
+        o_ref, s_ref = oracle.gdn_forward_fp8(codes(q8), codes(k8), codes(v8), scale(sq), scale(sk), scale(sv),
+                                              pick(inp.beta), pick(inp.decay), state_in=s0, bidi=wl.bidi,
+                                              n_threads=nproc)
+    elif args.block > 0:
+        o_ref, s_ref = oracle.gdn_forward_blockcausal(pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.beta),
+                                                      pick(inp.decay), args.block, state_in=s0, n_threads=nproc)
+    else:
+        o_ref, s_ref = oracle.gdn_forward(pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.beta),
+                                          pick(inp.decay), state_in=s0, bidi=wl.bidi, n_threads=nproc)
+    elapsed = time.perf_counter() - t0
+    n = len(heads)
+    o = flat(o_dev)[heads].double().cpu().numpy()[None]
+    if wl.bidi:
+        st, st_ref = s_dev.reshape(2, BH, wl.dk, wl.dv)[:, heads], s_ref.reshape(2, n, wl.dk, wl.dv)
+    else:
+        st, st_ref = s_dev.reshape(BH, wl.dk, wl.dv)[heads], s_ref.reshape(n, wl.dk, wl.dv)
+    st = st.double().cpu().numpy()
+    rel = lambda x, y: float(np.linalg.norm(x - y) / np.linalg.norm(y))
+    tol = 1e-5 if wl.dtype == "fp32" else 1e-2
+    e_o, e_s = rel(o, o_ref), rel(st, st_ref)
+    return {"checked": True, "rel_l2_o": e_o, "rel_l2_state": e_s, "tol": tol, "pass": e_o <= tol and e_s <= tol,
+            "sample": f"heads {heads} of {BH}, all {wl.T} tokens"
+                      f"{', both scan directions' if wl.bidi else ''}; fp64 oracle, {elapsed:.1f} s"}
+
+
 def _cpu_model():
     try:
         for line in open("/proc/cpuinfo"):
@@ -525,6 +574,12 @@ def run_gpu(args, world, rank, local):
             "gpu_launches": int(launches),
             "roofline": roofline,
             "clocks": clk.summary()}
+    if rank == 0:
+        try:
+            line["parity"] = sampled_parity(args, wl, inp, o, s_out,
+                                            fp8=(q8, k8, v8, sq, sk, sv) if args.fp8 else None)
+        except Exception as e:   # reported, never a reason to lose the line
+            line["parity"] = {"checked": False, "error": repr(e)[:300]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample_throughput(wl, inp, target_s=args.ref_seconds)
     if rank == 0:
