@@ -144,8 +144,8 @@ int gdn_forward_host_async(const void *q, const void *k, const void *v,
 /*
  * gdn_forward_noalloc -- gdn_forward that allocates no device memory.
  *
- * The paper has no counterpart: this entry point exists for callers that
- * cannot allocate device memory while they run this library -- plugins hosted
+ * The pages describe no counterpart: this entry point exists for callers
+ * that cannot allocate device memory while they run this library -- plugins hosted
  * by a framework that owns all device memory (media and real-time video
  * pipelines, inference engines with a fixed memory plan) and streaming loops
  * that must never wait on an allocator mid-run.  gdn_forward takes its only
