@@ -31,7 +31,6 @@ Also measured, and printed on the same JSON line:
 there is no upstream code to run).
 """
 import argparse
-import ctypes
 import hashlib
 import re
 import json
@@ -269,7 +268,6 @@ def oracle_sample_throughput(wl, inp=None, target_s=15.0):
     """Times the fp64 oracle on a bounded sample of the workload's own inputs:
     whole heads (both scan directions for bidi) truncated to a token prefix,
     sized for about target_s seconds of wall time on the host cores."""
-    import math
     import oracle
     from gated_delta_rule_149_b200.inputs import make_inputs
     if inp is None:

@@ -5,7 +5,6 @@ bidirectional, both value widths, ragged sequence ends, a given state, and a
 full-size streaming call.  The codes come from the usual input recipe,
 quantised per (batch, head) with scale max|x| / 448."""
 import pytest
-import torch
 
 from gated_delta_rule_149_b200 import gdn_device_status, gdn_forward_fp8
 from gated_delta_rule_149_b200.inputs import WORKLOADS, make_custom, make_inputs, quantize_e4m3

@@ -7,7 +7,6 @@ more segments than chunks, a given initial state, both value widths, several
 heads, and the streaming workloads at full size."""
 import numpy as np
 import pytest
-import torch
 
 from gated_delta_rule_149_b200 import gdn_device_status, gdn_forward, gdn_forward_segmented
 from gated_delta_rule_149_b200.inputs import WORKLOADS, make_custom, make_inputs
