@@ -73,6 +73,10 @@ def load_library():
         lib.gdn_workspace_release.restype = i
         lib.gdn_workspace_reserved.argtypes = [i, ctypes.POINTER(ctypes.c_ulonglong)]
         lib.gdn_workspace_reserved.restype = i
+        lib.gdn_debug_kernel_select.argtypes = [i]
+        lib.gdn_debug_kernel_select.restype = None
+        lib.gdn_debug_ring.argtypes = [vp]
+        lib.gdn_debug_ring.restype = None
         _lib = lib
     return _lib
 
@@ -366,3 +370,17 @@ def gdn_workspace_reserved(device=None):
     v = ctypes.c_ulonglong(0)
     _check(load_library().gdn_workspace_reserved(_device_index(device), ctypes.byref(v)))
     return v.value
+
+
+def debug_kernel_select(which):
+    """Test hook: 0 picks the bf16 chunkwise kernel by shape (the paired-SM kernel
+    for dk = dv = 128 whole-sequence calls), 1 forces the single-CTA chunkwise
+    kernel for every bf16 call (for A/B comparisons of the two)."""
+    load_library().gdn_debug_kernel_select(int(which))
+
+
+def debug_ring(buf):
+    """Test hook: a CUDA uint8 tensor of at least dirs*B*H*4*49664 bytes that the
+    paired-SM kernel uses as its operand ring (None: workspace), so that the
+    prepared operands of the last four chunks of every scan can be read back."""
+    load_library().gdn_debug_ring(None if buf is None else ctypes.c_void_p(buf.data_ptr()))
