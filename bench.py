@@ -76,12 +76,31 @@ def load_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+# B200 nominal figures (dense bf16; HBM3e), beside the measured ones
+SPEC_HBM_GBS, SPEC_BF16_TFLOPS = 8000.0, 2250.0
+
+
+def workload_config(wl, world):
+    """The config dict of a bench line: the workload and how it is run, the same
+    for the GPU arm and the reference arm."""
+    bytes_ = algorithmic_bytes(wl)
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk, "dv": wl.dv,
+            "mode": "bidi" if wl.bidi else ("rollout of %d causal chunks" % wl.n_chunks if wl.n_chunks > 1
+                                            else "causal"),
+            "n_chunks": wl.n_chunks, "token_heads_per_gpu": wl.token_heads,
+            "l2": ("no flush: inputs of %.2f GB per step exceed the 126 MB L2" % (bytes_ / 1e9)
+                   if bytes_ >= (1 << 30) else
+                   "flushed: 512 MB written before each step (%.3f GB per step would fit in the 126 MB "
+                   "L2); step time from the steps' own events" % (bytes_ / 1e9)),
+            "parallelism": f"replicas x{world} (independent scans, no collective)"}
+
+
 def kernel_source_sha():
     """Hash of the chunkwise kernel's device code (its source and the PTX
     wrappers it includes; comments and whitespace removed), so that a recorded
     traffic figure stays tied to the kernel it was taken on."""
     h = hashlib.sha256()
-    for name in ("gdn_chunk_tc.cu", "sm100_ptx.cuh"):
+    for name in ("gdn_chunk_pair.cu", "gdn_chunk_tc.cu", "gdn_chunk_common.cuh", "sm100_ptx.cuh"):
         p = os.path.join(ROOT, "gated_delta_rule_149_b200", "csrc", name)
         if os.path.exists(p):
             src = open(p).read()
@@ -275,29 +294,33 @@ def oracle_sample_throughput(wl, inp=None, target_s=15.0):
     nproc = os.cpu_count() or 1
     ndir = 2 if wl.bidi else 1
     BH = wl.B * wl.H
-    flat = lambda t: t.reshape(BH, *t.shape[2:])
+    T_all = wl.T * wl.n_chunks
+    if wl.n_chunks > 1:   # a rollout is one scan over its chunks: time it as one sequence per head
+        flat = lambda t: t.movedim(0, 2).reshape(BH, T_all, *t.shape[4:])
+    else:
+        flat = lambda t: t.reshape(BH, *t.shape[2:])
 
     def run(n_heads, T):
         sl = lambda t: flat(t)[:n_heads, :T].double().numpy()[None]
         args = [sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.beta), sl(inp.decay)]
-        s0 = None if inp.state0 is None else flat(inp.state0)[:n_heads].double().numpy()[None]
+        s0 = None if inp.state0 is None else inp.state0.reshape(BH, wl.dk, wl.dv)[:n_heads].double().numpy()[None]
         t0 = time.perf_counter()
         oracle.gdn_forward(*args, state_in=s0, bidi=wl.bidi, n_threads=nproc)
         return time.perf_counter() - t0
 
     per_wave = max(1, nproc // ndir)            # heads whose scans fill the cores once
     n_heads = min(BH, per_wave)
-    T_cal = min(wl.T, 2048)
+    T_cal = min(T_all, 2048)
     per_tok = run(n_heads, T_cal) / T_cal       # seconds per token for one wave
-    T = int(min(wl.T, max(256, target_s / per_tok)))
-    if T == wl.T:                               # whole heads are cheap: add waves
+    T = int(min(T_all, max(256, target_s / per_tok)))
+    if T == T_all:                              # whole heads are cheap: add waves
         waves = max(1, int(target_s / (per_tok * T)))
         n_heads = min(BH, per_wave * waves)
     el = run(n_heads, T)
     value = n_heads * T / el
     threads = min(nproc, n_heads * ndir)
     return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n_heads} of {BH} heads x first {T} of {wl.T} tokens of {wl.name} "
+            "sample": f"{n_heads} of {BH} heads x first {T} of {T_all} tokens of {wl.name} "
                       f"({'both scan directions' if wl.bidi else 'causal'}), fp64, "
                       f"{el:.1f} s wall on {threads} threads",
             "elapsed_s": el, "cpu": _cpu_model()}
@@ -316,6 +339,22 @@ def sampled_parity(args, wl, inp, o_dev, s_dev, fp8=None):
                        "the GPU tests check it on non-negative features"}
     BH = wl.B * wl.H
     heads = sorted({0, BH - 1})
+    if wl.n_chunks > 1:   # rollout: chunk-major tensors, checked chunk by chunk
+        n = wl.n_chunks
+        cm = lambda t: t.reshape(n, BH, *t.shape[3:])[:, heads].double().numpy()[:, None]   # [n,1,h,..]
+        t0 = time.perf_counter()
+        o_ref, s_ref, _ = oracle.gdn_rollout(cm(inp.q), cm(inp.k), cm(inp.v), cm(inp.beta), cm(inp.decay),
+                                             inp.state0.reshape(BH, wl.dk, wl.dv)[heads].double().numpy()[None])
+        elapsed = time.perf_counter() - t0
+        o = o_dev.reshape(n, BH, wl.T, wl.dv)[:, heads].double().cpu().numpy()[:, None]
+        st = s_dev.reshape(BH, wl.dk, wl.dv)[heads].double().cpu().numpy()[None]
+        rel = lambda x, y: float(np.linalg.norm(x - y) / np.linalg.norm(y))
+        e_o = max(rel(o[c], o_ref[c]) for c in range(n))
+        e_s = rel(st, s_ref)
+        return {"checked": True, "rel_l2_o": e_o, "rel_l2_state": e_s, "tol": 1e-2,
+                "pass": e_o <= 1e-2 and e_s <= 1e-2,
+                "sample": f"heads {heads} of {BH}, all {n} chunks x {wl.T} tokens (o: worst chunk); "
+                          f"fp64 oracle, {elapsed:.1f} s"}
     flat = lambda t: t.reshape(BH, *t.shape[2:])
     pick = lambda t: flat(t)[heads].double().numpy()[None]          # [1, n, ...]
     s0 = None if inp.state0 is None else pick(inp.state0)
@@ -378,8 +417,7 @@ def run_reference(args, world, rank):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / len(vals), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk,
-                       "dv": wl.dv, "mode": "bidi" if wl.bidi else "causal"},
+            "config": workload_config(wl, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"],
                              "kind": "oracle", "sample": vals[0]["sample"],
                              "cpu": vals[0]["cpu"]},
@@ -397,18 +435,19 @@ def run_gpu(args, world, rank, local):
     import torch
     from gated_delta_rule_149_b200 import (gdn, gdn_forward, gdn_forward_blockcausal, gdn_forward_fp8,
                                            gdn_forward_host_async, gdn_forward_normalized, gdn_forward_segmented,
-                                           gdn_device_status)
+                                           gdn_device_status, gdn_rollout)
     from gated_delta_rule_149_b200.inputs import quantize_e4m3
     from gated_delta_rule_149_b200.inputs import WORKLOADS, make_inputs
 
     wl = WORKLOADS[args.workload]
-    assert wl.n_chunks == 1, "the benchmark times single-call workloads"
+    rollout = wl.n_chunks > 1
     dev = torch.device("cuda", torch.cuda.current_device())
+    gdn.debug_kernel_select({"single": 1, "pair": 2}.get(args.kernel, 0))
     inp = make_inputs(wl)
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
     beta, decay = inp.beta.to(dev), inp.decay.to(dev)
     s0 = None if inp.state0 is None else inp.state0.to(dev)
-    o = torch.empty(wl.B, wl.H, wl.T, wl.dv, dtype=q.dtype, device=dev)
+    o = torch.empty(((wl.n_chunks,) if rollout else ()) + (wl.B, wl.H, wl.T, wl.dv), dtype=q.dtype, device=dev)
     s_out = torch.empty(((2,) if wl.bidi else ()) + (wl.B, wl.H, wl.dk, wl.dv),
                         dtype=torch.float32, device=dev)
     recurrent = args.recurrent or wl.dtype == "fp32"
@@ -416,6 +455,8 @@ def run_gpu(args, world, rank, local):
     lib = gdn.load_library()
 
     segmented = args.segments > 0 or args.block > 0 or args.normalized or args.fp8
+    if rollout and (segmented or recurrent):
+        raise SystemExit("the rollout workload runs the plain bf16 chunkwise path only")
     if args.fp8:
         if recurrent:
             raise SystemExit("--fp8 runs bf16-output workloads only")
@@ -427,7 +468,9 @@ def run_gpu(args, world, rank, local):
         raise SystemExit("--normalized runs bf16 workloads only")
 
     def step():
-        if args.fp8:
+        if rollout:
+            gdn_rollout(q, k, v, beta, decay, s0, o=o, state_out=s_out, stream=stream)
+        elif args.fp8:
             gdn_forward_fp8(q8, k8, v8, sq, sk, sv, beta, decay, s0, bidi=wl.bidi, o=o, state_out=s_out,
                             stream=stream)
         elif args.normalized:
@@ -486,8 +529,12 @@ def run_gpu(args, world, rank, local):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": traffic,
                 "peak_kind": peak_kind, "algorithmic_bytes": bytes_,
+                "frac_spec": achieved / SPEC_HBM_GBS,
+                "tensor_frac_spec": algorithmic_flops(wl) / call_s / 1e12 / SPEC_BF16_TFLOPS,
                 "scope": ("the token-by-token kernel (and, bidirectional, the add of its partials)"
                           if recurrent else
+                          "the whole rollout call: %d chunkwise launches, one per chunk" % wl.n_chunks
+                          if rollout else
                           "the chunkwise kernel (the call's one kernel)" if not segmented else
                           "the whole call: the bf16 kernel's algorithmic bytes over the time of all "
                           "its launches (%s)" % ("dequantising pre-pass included" if args.fp8 else
@@ -512,7 +559,7 @@ def run_gpu(args, world, rank, local):
 
     def e2e_step(n):
         ho, hso = hos[n % 2], hsos[n % 2]
-        if segmented:   # the same call on device copies of pinned host buffers
+        if segmented or rollout:   # the same call on device copies of pinned host buffers
             pairs = ((hq, q8), (hk, k8), (hv, v8), (hsq, sq), (hsk, sk), (hsv, sv)) if args.fp8 else \
                 ((hq, q), (hk, k), (hv, v))
             for h, dst in pairs + ((hb, beta), (ha, decay), (hs0, s0)):
@@ -550,24 +597,19 @@ def run_gpu(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic",
-            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk,
-                       "dv": wl.dv, "mode": "bidi" if wl.bidi else "causal",
-                       "kernel": ("recurrent" if recurrent else
-                                  "chunk_tc, fp8 E4M3 inputs (dequantising pre-pass)" if args.fp8 else
-                                  "chunk_tc, normalised read-out (z state, second pass)" if args.normalized else
-                                  f"chunk_tc, frame-block read-out, blocks of {args.block}" if args.block > 0 else
-                                  f"chunk_tc, segment-parallel x{args.segments}" if segmented else "chunk_tc"),
-                       "token_heads_per_gpu": wl.token_heads,
-                       "l2": ("no flush: inputs of %.2f GB per step exceed the 126 MB L2" % (bytes_ / 1e9)
-                              if flush_buf is None else
-                              "flushed: 512 MB written before each step (%.3f GB per step would fit "
-                              "in the 126 MB L2); step time from the steps' own events" % (bytes_ / 1e9)),
-                       "parallelism": f"replicas x{world} (independent scans, no collective)"},
+            "config": workload_config(wl, world),
+            "kernel": ("recurrent" if recurrent else
+                       "chunk_tc, fp8 E4M3 inputs (dequantising pre-pass)" if args.fp8 else
+                       "chunk_tc, normalised read-out (z state, second pass)" if args.normalized else
+                       f"chunk_tc, frame-block read-out, blocks of {args.block}" if args.block > 0 else
+                       f"chunk_tc, segment-parallel x{args.segments}" if segmented else
+                       "chunkwise, 2-CTA cluster per scan (preparation + state chain)" if args.kernel == "pair" else
+                       "chunkwise, single CTA per (dv slice, scan)"),
             "e2e": {"value": world * wl.token_heads / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": nbytes(hq, hk, hv, hb, ha, hs0,
                                                  *((hsq, hsk, hsv) if args.fp8 else ())),
                     "d2h_bytes_per_step": nbytes(hos[0], hsos[0]),
-                    "calls": ("synchronous, one stream" if segmented else
+                    "calls": ("synchronous, one stream" if segmented or rollout else
                               "gdn_forward_host_async on two alternating streams (2 calls in flight)")},
             "gpu_launches": int(launches),
             "roofline": roofline,
@@ -603,6 +645,8 @@ def main():
                     help="causal workloads: frame-block read-out with blocks of this many tokens")
     ap.add_argument("--segments", type=int, default=0,
                     help="causal workloads: run the segment-parallel scan with this many segments")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "single", "pair"],
+                    help="bf16 chunkwise kernel: by shape (default), the single-CTA one, or the paired-SM one")
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="seconds of CPU work per oracle sample (default 15; 8 for --impl reference)")
     args = ap.parse_args()

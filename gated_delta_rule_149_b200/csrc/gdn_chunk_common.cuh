@@ -197,9 +197,11 @@ __device__ __forceinline__ void st_tpair(uint8_t *tile, int dir, int lr, int lj,
     *reinterpret_cast<uint32_t *>(tile + sw128_off(pr, pc)) = dir ? pack_bf16(v1, v0) : pack_bf16(v0, v1);
 }
 
+// BAR / NTHREADS: the named barrier that ends the step (or, with NTHREADS = 0,
+// the run-time bar_id / bar_threads).
 template <int BAR, int NTHREADS>
 __device__ __forceinline__ void solve_diag_blocks(float *As, const float *gt, uint8_t *sT1, uint8_t *sT2,
-                                               float *dbgT, int dir, int pt)
+                                               float *dbgT, int dir, int pt, int bar_id = 0, int bar_threads = 0)
 {
     if (pt < 64) {
         const int a = pt >> 4, c = pt & 15;
@@ -219,7 +221,8 @@ __device__ __forceinline__ void solve_diag_blocks(float *As, const float *gt, ui
         if (dbgT)
             for (int r = 0; r < 16; ++r) dbgT[(16 * a + r) * 64 + 16 * a + c] = x[r];
     }
-    named_bar(BAR, NTHREADS);
+    if (NTHREADS) named_bar(BAR, NTHREADS);
+    else named_bar(bar_id, bar_threads);
 }
 
 // T1, T2 of the four diagonal blocks, from D_a in place in A (64 threads: each

@@ -66,8 +66,10 @@ namespace {
 // 128 registers a thread (the chain's state threads hold 64 fp32 values).
 constexpr int kPThreads = 448;
 constexpr int kGroup = 256, kGroupB = 128;
-constexpr int kBarA = 1, kBarB = 2, kBarGate = 3;   // named barriers
-constexpr int kNG = 3;                    // gate buffers
+// named barriers: solver groups (2), finisher / output group, gate threads of each
+// solver group; the chain's state group uses kBarA
+constexpr int kBarA = 1, kBarB = 2, kBarGate = 3, kBarA2 = 4, kBarGate2 = 5;
+constexpr int kNG = 4;                    // gate buffers (each solver group computes its next chunk's)
 constexpr uint32_t kGateFloats = 9 * 64;
 constexpr int kNSlot = 4;                 // ring slots per scan
 
@@ -84,8 +86,9 @@ constexpr uint32_t kPStageBytes = 32768;
 constexpr uint32_t kPP = kPStage + 2 * kPStageBytes;      // 2 x 8 KB P
 constexpr uint32_t kPTB = kPP + 16384;                    // 2 x [PT1 | T1 | PT2 | T2], 8 KB each
 constexpr uint32_t kPA2 = kPTB + 65536;                   // A2 staging [kb][128 rows]
-constexpr uint32_t kPA = kPA2 + 32768;                    // fp32 [64][kLDA] solve buffer
-constexpr uint32_t kPGates = kPA + 64 * kLDA * 4;
+constexpr uint32_t kPA = kPA2 + 32768;                    // 2 x fp32 [64][kLDA] solve buffers
+constexpr uint32_t kPAStride = 64 * kLDA * 4;
+constexpr uint32_t kPGates = kPA + 2 * kPAStride;
 constexpr uint32_t kPGst = kPGates + kNG * kGateFloats * 4;   // 512 B: e, gamma_end of the slot
 constexpr uint32_t kPEnd = kPGst + 512;
 // chain
@@ -149,7 +152,7 @@ struct Bars {
     uint32_t tmem_slot;
     int abort_flag;
     int s_old;
-    float s_wsum;
+    float s_wsum[2];
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block");
 
@@ -338,21 +341,25 @@ __device__ __forceinline__ void mask_rows(uint32_t taddr, const float *gt, float
     }
 }
 
-// Solver group (8 warps): gates one chunk ahead, the masks, T = (I + A)^-1
-// written as T1 = T diag(b gamma) and T2 = T diag(b).  Warp w reads TMEM lane
-// quarter qd = w % 4 and columns [32 hf, +32) of each row it owns.
+// Solver groups (two groups of 4 warps, warp w reading TMEM lane quarter
+// qd = w % 4): group g takes the chunks i with i % 2 == g, so that two chunks'
+// solves, each a long chain of dependent steps, run at once.  Per chunk: the
+// masks of [Q;K] K^T, then T = (I + A)^-1 written as T1 = T diag(b gamma) and
+// T2 = T diag(b); meanwhile the group's gate threads prepare the gates of its
+// next chunk.  pt is the thread's index in its group (0..127).
 template <int DIR>
-__device__ __forceinline__ void prep_solver(const Ctx &x, const PairParams &p, int pt, int qd, int hf)
+__device__ __forceinline__ void prep_solver(const Ctx &x, const PairParams &p, int pt, int qd, int g)
 {
     Bars &B = *x.bars;
     const int lane = pt & 31;
-    float *As = reinterpret_cast<float *>(x.smem + kPA);
+    const int bar = g ? kBarA2 : kBarA, gbar = g ? kBarGate2 : kBarGate;
+    float *As = reinterpret_cast<float *>(x.smem + kPA + g * kPAStride);
     const uint32_t tm_lane = (uint32_t)(qd * 32) << 16;
     const float *beta_h = p.beta + (size_t)x.bh * x.T;
     const float *decay_h = p.decay + (size_t)x.bh * x.T;
 
     // gate threads: pt 64..127 (scan position gpt), on their own 64-thread barrier
-    const bool gate_thr = pt >= 64 && pt < 128;
+    const bool gate_thr = pt >= 64;
     const int gpt = pt - 64;
     float ra = 1.f, rb = 0.f;
     auto load_raw = [&](int j) {
@@ -373,16 +380,16 @@ __device__ __forceinline__ void prep_solver(const Ctx &x, const PairParams &p, i
         if (j >= kNG) wait_bar(&B.g_empty[gj], ((j / kNG) + 1) & 1, x.abort_flag, p.err, 8);
         float v = fmaxf(log2f(ra), -120.f);   // decay below 2^-120 acts as 2^-120
         const float bcur = rb;
-        load_raw(j + 1);
+        load_raw(j + 2);
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, v, off);
             if (lane >= off) v += y;
         }
-        if (gpt == 31) x.bars->s_wsum = v;
-        named_bar(kBarGate, 64);
+        if (gpt == 31) x.bars->s_wsum[g] = v;
+        named_bar(gbar, 64);
         {
-            const float G = (gpt >= 32) ? v + x.bars->s_wsum : v;
+            const float G = (gpt >= 32) ? v + x.bars->s_wsum[g] : v;
             const int pp = DIR ? (63 - gpt) : gpt;
             gt[gG * 64 + pp] = G;
             const float gam = exp2f(G);
@@ -390,7 +397,7 @@ __device__ __forceinline__ void prep_solver(const Ctx &x, const PairParams &p, i
             gt[gBet * 64 + pp] = bcur;
             gt[gBG * 64 + pp] = bcur * gam;
         }
-        named_bar(kBarGate, 64);
+        named_bar(gbar, 64);
         // references: scan positions 15 (first half), 47 (second half), 31 (boundary)
         const float R1 = gt[gG * 64 + (DIR ? 48 : 15)];
         const float R2 = gt[gG * 64 + (DIR ? 16 : 47)];
@@ -415,18 +422,18 @@ __device__ __forceinline__ void prep_solver(const Ctx &x, const PairParams &p, i
                 x.bars->gscal[gj][1] = fact ? 1.f : 0.f;
             }
         }
-        named_bar(kBarGate, 64);
+        named_bar(gbar, 64);
         if (gpt == 0) mbar_arrive(&B.g_full[gj]);
     };
-    load_raw(0);
+    load_raw(g);
 
-    // step i = -1 only computes the gates of chunk 0
+    // the first step only computes the gates of the group's first chunk
 #pragma unroll 1
-    for (int i = -1; i < x.NC; ++i) {
-        const int b = i & 1;
-        const int gi = (i + kNG) % kNG;
+    for (int i = g - 2; i < x.NC; i += 2) {
+        const int b = g;   // = i & 1: this group's P, T and D1 buffers
+        const int gi = (i + 2 * kNG) % kNG;
         float *gt = gates_buf(x, gi);
-        uint8_t *tb = x.smem + kPTB + (b & 1) * 32768;
+        uint8_t *tb = x.smem + kPTB + b * 32768;
         if (i >= 0) {
             const bool fact = x.bars->gscal[gi][1] != 0.f;
             if (pt == 0) tr(p, x, 0, 0, i);
@@ -435,31 +442,35 @@ __device__ __forceinline__ void prep_solver(const Ctx &x, const PairParams &p, i
             if (pt == 0) tr(p, x, 0, 1, i);
             tc_fence_after();
             uint8_t *sP = x.smem + kPP + b * 8192;
-            const uint32_t taddr = x.tmem + tm_lane + kTD1 + 64 * b + 32 * hf;
-            mask_rows<DIR>(taddr, gt, As, sP, qd, lane, hf, fact);
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf)
+                mask_rows<DIR>(x.tmem + tm_lane + kTD1 + 64 * b + 32 * hf, gt, As, sP, qd, lane, hf, fact);
             if (pt == 0) tr(p, x, 0, 7, i);
             tc_fence_before();
             fence_proxy_async_smem();
-            if (named_bar_any(kBarA, kGroup, *x.abort_flag)) return;
+            if (named_bar_any(bar, 128, *x.abort_flag)) return;
             if (pt == 0) mbar_arrive(&B.d1_empty[b]);
             if (pt == 0) tr(p, x, 0, 2, i);
         }
 
-        // T = (I + A)^-1; meanwhile the gate threads prepare the next chunk's gates
-        if (gate_thr && i + 1 < x.NC) compute_gates(i + 1);
+        // T = (I + A)^-1; meanwhile the gate threads prepare the group's next chunk's gates
+        if (gate_thr && i + 2 < x.NC) compute_gates(i + 2);
         if (i < 0) {
-            named_bar(kBarA, kGroup);
+            named_bar(bar, 128);
             continue;
         }
         // T1 / T2 of this buffer must be done with (chunk i - 2: its products and its ring copy)
         if (i >= 2) wait_bar(&B.t_free[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 11);
         if (pt == 0) tr(p, x, 0, 3, i);
-        solve_diag_blocks<kBarA, kGroup>(As, gt, tb + 8192, tb + 24576, nullptr, DIR, pt);
+        solve_diag_blocks<0, 0>(As, gt, tb + 8192, tb + 24576, nullptr, DIR, pt, bar, 128);
         if (pt == 0) tr(p, x, 0, 4, i);
+        // the six strips below the diagonal blocks and the diagonal blocks' T1, T2:
+        // eight pieces of work, two for each of the group's warps
         solve_off_diag_compact(As, gt, tb + 8192, tb + 24576, DIR, pt);
-        if ((pt & 31) == 0) tr(p, x, 0, 20 + (pt >> 5), i);
+        solve_off_diag_compact(As, gt, tb + 8192, tb + 24576, DIR, pt + 128);
+        if ((pt & 31) == 0) tr(p, x, 0, 20 + (pt >> 5) + 4 * g, i);
         fence_proxy_async_smem();
-        if (named_bar_any(kBarA, kGroup, *x.abort_flag)) return;
+        if (named_bar_any(bar, 128, *x.abort_flag)) return;
         if (pt == 0) mbar_arrive(&B.tp_full[b]);
         if (pt == 0) tr(p, x, 0, 5, i);
     }
@@ -964,7 +975,7 @@ gdn_chunk_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     }
     if (rank == 0) {
         float *As0 = reinterpret_cast<float *>(smem + kPA);
-        for (int i = tid; i < 64 * kLDA; i += kPThreads) As0[i] = 0.f;
+        for (int i = tid; i < 2 * 64 * kLDA; i += kPThreads) As0[i] = 0.f;
         // T1, T2: the triangle the solve never writes stays zero for the whole scan
         for (int b = 0; b < 2; ++b) {
             uint32_t *t1 = reinterpret_cast<uint32_t *>(smem + kPTB + b * 32768 + 8192);
@@ -987,9 +998,9 @@ gdn_chunk_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         } else if (warp == 1) {
             if (lane == 0) prep_mma(x, p);
         } else if (warp < 10) {
-            const int gt = tid - 64, qd = warp & 3, hf = (warp - 2) >> 2;
-            if (x.dir) prep_solver<1>(x, p, gt, qd, hf);
-            else prep_solver<0>(x, p, gt, qd, hf);
+            const int g = (warp - 2) >> 2, pt = tid - 64 - 128 * g, qd = warp & 3;
+            if (x.dir) prep_solver<1>(x, p, pt, qd, g);
+            else prep_solver<0>(x, p, pt, qd, g);
         } else {
             const int ft = tid - 320, qd = warp & 3;
             if (x.dir) prep_finisher<1>(x, p, ft, qd);
@@ -1102,7 +1113,9 @@ cudaError_t device_info(DevInfo **out)
 
 bool chunk_pair_supported(const FwdArgs &a)
 {
-    return g_kernel_select != 1 && !a.fp32 && a.dk == kDK && a.dv == 128 && a.n_seg == 1 &&
+    // chosen on request only (g_kernel_select == 2): on the measured workloads the
+    // single-CTA kernel is still the faster one
+    return g_kernel_select == 2 && !a.fp32 && a.dk == kDK && a.dv == 128 && a.n_seg == 1 &&
            a.seg0 == 0 && a.seg_chunks == 0;
 }
 
@@ -1178,6 +1191,7 @@ cudaError_t launch_chunk_pair(const FwdArgs &a, cudaStream_t stream)
 // paired kernel uses as its operand ring instead of workspace (NULL: off), so
 // a test can read the prepared operands of each chunk back.
 // gdn_debug_kernel_select: 0 picks the kernel by shape, 1 forces the
-// single-CTA chunkwise kernel for every bf16 call.
+// single-CTA chunkwise kernel for every bf16 call, 2 asks for the paired-SM
+// kernel wherever it applies (dk = dv = 128, whole sequences).
 extern "C" void gdn_debug_ring(void *device_buffer) { gdn::g_debug_ring = device_buffer; }
 extern "C" void gdn_debug_kernel_select(int which) { gdn::g_kernel_select = which; }

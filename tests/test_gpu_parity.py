@@ -16,16 +16,15 @@ from parity_util import TOL, assert_finite_bounded, f64, oracle_forward, rel_l2,
 
 pytestmark = pytest.mark.gpu
 
-# which kernels serve bf16 inputs: the default choice by shape (the paired-SM
-# chunkwise kernel for dk = dv = 128, the single-CTA one otherwise), the
-# single-CTA chunkwise kernel for every shape, and the token-by-token
-# cross-check kernel
+# which kernels serve bf16 inputs: the paired-SM chunkwise kernel (dk = dv = 128;
+# the single-CTA one for other shapes), the single-CTA chunkwise kernel, and the
+# token-by-token cross-check kernel
 BF16_KERNELS = ["pair", "single", "recurrent"]
 
 
 @contextlib.contextmanager
 def use_kernel(kernel):
-    gdn.debug_kernel_select(1 if kernel == "single" else 0)
+    gdn.debug_kernel_select({"pair": 2, "single": 1}.get(kernel, 0))
     try:
         yield kernel == "recurrent"
     finally:
