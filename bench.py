@@ -100,7 +100,7 @@ def kernel_source_sha():
     wrappers it includes; comments and whitespace removed), so that a recorded
     traffic figure stays tied to the kernel it was taken on."""
     h = hashlib.sha256()
-    for name in ("gdn_chunk_pair.cu", "gdn_chunk_tc.cu", "gdn_chunk_common.cuh", "sm100_ptx.cuh"):
+    for name in ("gdn_chunk_pool.cu", "gdn_chunk_tc.cu", "gdn_chunk_common.cuh", "sm100_ptx.cuh"):
         p = os.path.join(ROOT, "gated_delta_rule_149_b200", "csrc", name)
         if os.path.exists(p):
             src = open(p).read()
@@ -442,7 +442,7 @@ def run_gpu(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     rollout = wl.n_chunks > 1
     dev = torch.device("cuda", torch.cuda.current_device())
-    gdn.debug_kernel_select({"single": 1, "pair": 2}.get(args.kernel, 0))
+    gdn.debug_kernel_select(1 if args.kernel == "single" else 0)
     inp = make_inputs(wl)
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
     beta, decay = inp.beta.to(dev), inp.decay.to(dev)
@@ -603,8 +603,8 @@ def run_gpu(args, world, rank, local):
                        "chunk_tc, normalised read-out (z state, second pass)" if args.normalized else
                        f"chunk_tc, frame-block read-out, blocks of {args.block}" if args.block > 0 else
                        f"chunk_tc, segment-parallel x{args.segments}" if segmented else
-                       "chunkwise, 2-CTA cluster per scan (preparation + state chain)" if args.kernel == "pair" else
-                       "chunkwise, single CTA per (dv slice, scan)"),
+                       "chunkwise, single CTA per (dv slice, scan)" if args.kernel == "single" or wl.dv != 128 else
+                       "chunkwise, pooled: a state-chain CTA per scan beside preparation workers on the other SMs"),
             "e2e": {"value": world * wl.token_heads / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": nbytes(hq, hk, hv, hb, ha, hs0,
                                                  *((hsq, hsk, hsv) if args.fp8 else ())),
@@ -645,8 +645,9 @@ def main():
                     help="causal workloads: frame-block read-out with blocks of this many tokens")
     ap.add_argument("--segments", type=int, default=0,
                     help="causal workloads: run the segment-parallel scan with this many segments")
-    ap.add_argument("--kernel", default="auto", choices=["auto", "single", "pair"],
-                    help="bf16 chunkwise kernel: by shape (default), the single-CTA one, or the paired-SM one")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "single"],
+                    help="bf16 chunkwise kernel: by shape (default: the pooled kernel for dk = dv = 128), "
+                         "or the single-CTA one for every shape")
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="seconds of CPU work per oracle sample (default 15; 8 for --impl reference)")
     args = ap.parse_args()

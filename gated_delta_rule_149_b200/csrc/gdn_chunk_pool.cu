@@ -1,6 +1,6 @@
-// Chunkwise GDN recurrence on sm_100a, split across the two CTAs of a cluster:
-// one CTA prepares every chunk's state-independent operands, the other runs
-// only the serial state chain.
+// Chunkwise GDN recurrence on sm_100a: one CTA per SM, split between the
+// serial state chains (one CTA per scan) and a pool of preparation workers
+// that serve every scan.
 //
 // The recurrence (librediffusion PR #21 page, "What's added": the GDN
 // linear-attention recurrence; the causal-streaming and bidirectional forms
@@ -17,29 +17,33 @@
 // Substituting U into O gives both from one product with the previous state:
 //     [O; U] = [P T2; T2] V + [Q'; -W] H_prev,   Q' = diag(gamma) Q - P T1 K,  W = T1 K,
 // so everything except that product and the state update is independent of
-// the state, and a chunk's operands A1 = [P T2; T2] (128 x 64) and
-// A2 = [Q'; -W] (128 x dk) can be formed ahead of the chain.
+// the state: a chunk's operands A1 = [P T2; T2] (128 x 64) and
+// A2 = [Q'; -W] (128 x dk) can be formed by any SM, ahead of the chain.
 //
-// One 2-CTA cluster per (direction, batch*head):
-//   rank 0, prep:  gates, the masks of [Q;K] K^T, the 64 x 64 solve, the
-//                  products P [T1 | T2] and [P T1; T1] K and their epilogues
-//                  (tcgen05 MMAs, fp32 accumulators in TMEM); writes A1, A2,
-//                  e and gamma_end of each chunk into a small ring of slots in
-//                  global memory (it stays in L2: a few chunks per scan);
-//   rank 1, chain: loads V, K and the ring slot of each chunk, and runs
-//                  D = V^T A1^T + H^T A2^T   (M = dv = 128, N = 128: O^T and U^T)
-//                  S = Ubar^T K              (Ubar = diag(e) U; M = dv, N = dk)
-//                  H^T <- gamma_end H^T + S  (fp32 in registers)
-//                  with H^T and Ubar^T as bf16 A operands in TMEM, and writes O.
-// The two CTAs hand slots over with mbarrier arrivals across the cluster; the
-// data itself travels through L2 because the shared-memory path between the
-// SMs of a cluster is several times slower than L2 for this volume (48 KB per
-// chunk).  Bidirectional: both scans run in the same launch; for each output
-// tile the first writer stores its bf16 partial and the second adds its fp32
-// partial to it and rounds once, after an arrival counter shows the first is
-// visible.  With a cooperative launch every cluster is resident and the first
-// writer of each tile is known in advance; otherwise a claim on the counter
-// decides it at run time.
+// Roles (CTA = blockIdx.x):
+//   CTA < n_scans, chain of scan CTA: loads V, K and the scan's prepared
+//       operands of each chunk, and runs
+//           D = V^T A1^T + H^T A2^T   (M = dv = 128, N = 128: O^T and U^T)
+//           S = Ubar^T K              (Ubar = diag(e) U; M = dv, N = dk)
+//           H^T <- gamma_end H^T + S  (fp32 in registers)
+//       with H^T and Ubar^T as bf16 A operands in TMEM, and writes O.
+//   CTA >= n_scans, worker: takes (scan, chunk) items from a global counter in
+//       chunk-major order and prepares them: gates, the masks of [Q;K] K^T,
+//       the 64 x 64 solve, the products P [T1 | T2] and [P T1; T1] K and their
+//       epilogues (tcgen05 MMAs, fp32 accumulators in TMEM); writes A1, A2, e
+//       and gamma_end into the scan's ring of slots in global memory (a few
+//       chunks per scan, so it stays in L2).
+// A preparation is a long chain of dependent steps, independent from chunk to
+// chunk; the chains are serial.  Giving the preparations their own pool of
+// SMs lets as many run at once as the pool holds, whatever the number of
+// scans.  Each slot carries a sequence word (chunk + 1 once filled) and each
+// scan a count of chunks its chain has taken out, so a worker fills a slot
+// only after its previous chunk was consumed; every wait is bounded.
+// Bidirectional: both scans run in the same launch; for each output tile the
+// first writer stores its bf16 partial and the second adds its fp32 partial
+// to it and rounds once, after an arrival counter shows the first is visible
+// (the forward scan writes first in the first half of the sequence).  The
+// launch is cooperative: every CTA is resident, or the launch is refused.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -61,34 +65,32 @@ int g_kernel_select = 0;
 
 namespace {
 
-// 14 warps: TMA, MMA, group A (8 warps: two per TMEM lane quarter), group B
-// (4 warps: one per quarter).  At most four warps per SM sub-partition leave
-// 128 registers a thread (the chain's state threads hold 64 fp32 values).
-constexpr int kPThreads = 448;
+// 16 warps: TMA, MMA, group A (8 warps: two per TMEM lane quarter), group B
+// (4 warps: one per quarter), 2 gate warps (workers).  Four warps per SM
+// sub-partition leave 128 registers a thread (a chain's state threads hold 64
+// fp32 values).
+constexpr int kThreads = 512;
 constexpr int kGroup = 256, kGroupB = 128;
-// named barriers: solver groups (2), finisher / output group, gate threads of each
-// solver group; the chain's state group uses kBarA
-constexpr int kBarA = 1, kBarB = 2, kBarGate = 3, kBarA2 = 4, kBarGate2 = 5;
-constexpr int kNG = 4;                    // gate buffers (each solver group computes its next chunk's)
+constexpr int kBarA = 1, kBarB = 2, kBarGate = 3;   // named barriers
+constexpr int kNG = 3;                    // gate buffers
+constexpr int kNS = 3;                    // worker input stages
 constexpr uint32_t kGateFloats = 9 * 64;
-constexpr int kNSlot = 4;                 // ring slots per scan
+constexpr int kNSlot = 8;                 // ring slots per scan
 
 // ring slot: A1 [128 rows x 64] bf16, A2 [kb][128 rows x 64] bf16 (both 128B-swizzled
 // images), then e[64] and gamma_end (fp32)
 constexpr uint32_t kSlotA1 = 0, kSlotA2 = 16384, kSlotGates = 49152, kSlotBytes = 49664;
 
-// shared memory (from a 1024-aligned base); the barrier block sits at the same
-// offset in both CTAs so that remote arrivals can address it
+// shared memory (from a 1024-aligned base)
 constexpr uint32_t kOffBar = 0;
-// prep
-constexpr uint32_t kPStage = 1024;                        // 2 x [kb0: Q|K][kb1: Q|K]
-constexpr uint32_t kPStageBytes = 32768;
-constexpr uint32_t kPP = kPStage + 2 * kPStageBytes;      // 2 x 8 KB P
-constexpr uint32_t kPTB = kPP + 16384;                    // 2 x [PT1 | T1 | PT2 | T2], 8 KB each
+// worker
+constexpr uint32_t kWStage = 1024;                        // kNS x [kb0: Q|K][kb1: Q|K]
+constexpr uint32_t kWStageBytes = 32768;
+constexpr uint32_t kPP = kWStage + kNS * kWStageBytes;    // 8 KB P
+constexpr uint32_t kPTB = kPP + 8192;                     // 2 x [PT1 | T1 | PT2 | T2], 8 KB each
 constexpr uint32_t kPA2 = kPTB + 65536;                   // A2 staging [kb][128 rows]
-constexpr uint32_t kPA = kPA2 + 32768;                    // 2 x fp32 [64][kLDA] solve buffers
-constexpr uint32_t kPAStride = 64 * kLDA * 4;
-constexpr uint32_t kPGates = kPA + 2 * kPAStride;
+constexpr uint32_t kPA = kPA2 + 32768;                    // fp32 [64][kLDA] solve buffer
+constexpr uint32_t kPGates = kPA + 64 * kLDA * 4;
 constexpr uint32_t kPGst = kPGates + kNG * kGateFloats * 4;   // 512 B: e, gamma_end of the slot
 constexpr uint32_t kPEnd = kPGst + 512;
 // chain
@@ -102,14 +104,15 @@ constexpr uint32_t kSmemBytes = (kPEnd > kCEnd ? kPEnd : kCEnd);
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(kPP % 1024 == 0 && kPTB % 1024 == 0 && kPA2 % 1024 == 0 && kCA % 1024 == 0 &&
-              kCABytes % 1024 == 0 && kCO % 1024 == 0 && kPGst % 16 == 0, "tile alignment");
+              kCABytes % 1024 == 0 && kCO % 1024 == 0 && kPGst % 16 == 0,
+              "tile alignment");
 
 // TMEM columns
-constexpr uint32_t kTD1 = 0, kTD2 = 128, kTD3 = 256;                 // prep
+constexpr uint32_t kTD1 = 0, kTD2 = 128, kTD3 = 256;                 // worker
 constexpr uint32_t kTD = 0, kTS = 256, kTH = 384, kTUb = 448;         // chain
 constexpr uint32_t kTmemCols = 512;
 
-// Chunk-0 products of scan (0, 0) can be dumped for debugging in builds with
+// Chunk-0 products of scan 0 can be dumped for debugging in builds with
 // GDN_DEBUG_DUMP; production builds compile the dump code out.
 #ifdef GDN_DEBUG_DUMP
 constexpr bool kDbgOn = true;
@@ -124,35 +127,40 @@ constexpr uint32_t kIdA = idesc_bf16(128, 128, true, false);    // V^T A1^T
 constexpr uint32_t kIdB = idesc_bf16(128, 128, false, false);   // H^T A2^T (A in TMEM)
 constexpr uint32_t kIdC = idesc_bf16(128, 128, false, true);    // Ubar^T K (A in TMEM)
 
-struct PairParams {
+struct PoolParams {
     const float *beta, *decay, *state_in;
     float *state_out;
     __nv_bfloat16 *o;
-    uint8_t *ring;       // [dirs][BH][kNSlot] slots
-    int *counters;       // bidi arrival counters [BH][n_chunks], zeroed
+    uint8_t *ring;       // [n_scans][kNSlot] slots
+    int *slot_seq;       // [n_scans][kNSlot]: chunk + 1 once the slot holds that chunk, zeroed
+    int *consumed;       // [n_scans]: chunks the scan's chain has taken out of its ring, zeroed
+    int *work;           // next item to hand out, zeroed
+    int *counters;       // bidi arrival counters [BH][n_chunks] of this launch's heads, zeroed
     int *err;            // device error word
-    float *debug;        // optional: chunk-0 D and S of scan (0, 0)
-    long long *trace;    // tracing builds: clock64 marks of scan (0, 0)
-    int BH, T, n_chunks;
-    int predict;         // bidi: every cluster resident, first writer known in advance
+    float *debug;        // optional: chunk-0 D and S of scan 0
+    long long *trace;    // tracing builds: clock64 marks of scan 0 / worker 0
+    int BH;              // heads in this launch
+    int bh0;             // index of its first head in the tensors
+    int BH_all;          // heads in the tensors (the reverse direction's state_out offset)
+    int T, n_chunks, n_scans, n_items;
 };
 
 struct Bars {
-    // prep
-    uint64_t st_full[2], st_empty[2], d1_full[2], d1_empty[2], tp_full[2], p_free[2], t_free[2];
+    // worker
+    uint64_t it_full[kNS], st_full[kNS], st_empty[kNS], d1_full[2], d1_empty[2], tp_full[2], p_free, t_free[2];
     uint64_t d2_full, d2_empty, e2_done, d3_full, d3_empty;
     uint64_t g_full[kNG], g_empty[kNG];
-    uint64_t slot_empty[kNSlot];
     // chain
     uint64_t vk_full[kNVK], vk_empty[kNVK], a_full[2], a_empty[2], d_full[2], d_empty[2], o_full[2];
     uint64_t u_full, s_full, h_full;
-    uint64_t slot_full[kNSlot];
     uint64_t drain;
     float gscal[kNG][2];   // per gate buffer: G_end, factorised (1) or not (0)
+    int gitem[kNG];        // per gate buffer: the item, or -1 after the last
+    int sitem[kNS];        // per input stage: the item, or -1 after the last
     uint32_t tmem_slot;
     int abort_flag;
     int s_old;
-    float s_wsum[2];
+    float s_wsum;
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block");
 
@@ -162,9 +170,28 @@ struct Ctx {
     Bars *bars;
     volatile int *abort_flag;
     uint32_t tmem;
-    int dir, bh, NC, T;
-    uint8_t *ring;   // this scan's kNSlot slots
+    int NC, T;
+    // chain CTAs
+    int scan, dir, bhl, bh;   // scan, its direction, head in this launch, head in the tensors
+    uint8_t *ring;            // the scan's kNSlot slots
 };
+
+// An item's scan, direction, head (in the tensors), and chunk in scan order
+// (items are handed out chunk-major: every scan's first chunk, then every
+// scan's second, ...).
+struct Item {
+    int scan, dir, bh, ci, c;   // ci: scan-order position, c: chunk index in the sequence
+};
+__device__ __forceinline__ Item decode_item(const PoolParams &p, int k)
+{
+    Item it;
+    it.ci = k / p.n_scans;
+    it.scan = k - it.ci * p.n_scans;
+    it.dir = it.scan >= p.BH ? 1 : 0;
+    it.bh = p.bh0 + it.scan - it.dir * p.BH;
+    it.c = it.dir ? p.n_chunks - 1 - it.ci : it.ci;
+    return it;
+}
 
 template <int DIR>
 __device__ __forceinline__ int chunk_of(const Ctx &x, int i) { return DIR ? (x.NC - 1 - i) : i; }
@@ -173,37 +200,18 @@ __device__ __forceinline__ float *gates_buf(const Ctx &x, int g)
     return reinterpret_cast<float *>(x.smem + kPGates) + g * kGateFloats;
 }
 
-// Tracing builds (-DGDN_TRACE): clock64() at role marks of scan (0, 0) for chunks
-// kTr0 .. kTr0 + 7, stored at trace[(rank * 32 + mark) * 8 + chunk - kTr0].
-constexpr int kTr0 = 100;
-__device__ __forceinline__ void tr(const PairParams &p, const Ctx &x, int rank, int mark, int i)
+// Tracing builds (-DGDN_TRACE): clock64() at role marks of scan 0's chain
+// (rank 1) and of worker 0 (rank 0) for local steps kTr0 .. kTr0 + 7, stored at
+// trace[(rank * 32 + mark) * 8 + step - kTr0].
+__device__ __forceinline__ void tr(const PoolParams &p, int rank, int mark, int i)
 {
 #ifdef GDN_TRACE
-    if (p.trace && x.dir == 0 && x.bh == 0 && i >= kTr0 && i < kTr0 + 8)
+    constexpr int kTr0 = 100;
+    if (p.trace && blockIdx.x == (rank ? 0 : p.n_scans) && i >= kTr0 && i < kTr0 + 8)
         p.trace[(rank * 32 + mark) * 8 + i - kTr0] = (long long)clock64();
+#else
+    (void)p; (void)rank; (void)mark; (void)i;
 #endif
-}
-
-// Bounded wait on a phase completed by arrivals from the other CTA of the cluster.
-__device__ __noinline__ bool wait_cluster_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                               int *err, int code)
-{
-    const unsigned long long t0 = globaltimer();
-    for (uint32_t it = 0; it < (1u << 30); ++it) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if ((it & 255) == 255 && globaltimer() - t0 > kWaitLimitNs) break;
-    }
-    atomicOr(err, code);
-    *abort_flag = 1;
-    return false;
-}
-
-__device__ __forceinline__ bool wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             int *err, int code)
-{
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    return wait_cluster_slow(bar, parity, abort_flag, err, code);
 }
 
 // Lets every MMA this thread issued complete (bounded) before TMEM is released.
@@ -221,88 +229,213 @@ __device__ __forceinline__ void drain_copies(uint64_t *bar, uint32_t parity)
     while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < 200000000ull) {}
 }
 
-// ================================================================== prep CTA
+__device__ __forceinline__ void st_release_gpu(int *addr, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
 
-template <int DIR>
-__device__ __forceinline__ void prep_tma(const Ctx &x, const CUtensorMap *tmQ, const CUtensorMap *tmK,
-                                         const PairParams &p)
+// Bounded wait until a device-wide word reaches `target`; on timeout the error
+// is recorded and the CTA's abort flag raised.  false on timeout or abort.
+__device__ __forceinline__ bool wait_global(const int *word, int target, const Ctx &x, const PoolParams &p,
+                                            int code)
+{
+    if (spin_global_at_least(word, target, x.abort_flag)) return true;
+    if (!*x.abort_flag) atomicOr(p.err, code);
+    *x.abort_flag = 1;
+    return false;
+}
+
+// ================================================================== workers
+
+// TMA: hands out the items (one per input stage: published on it_full before
+// its q, k tiles are loaded) and loads their q, k tiles; an item past the last
+// one marks the end.
+__device__ __forceinline__ void worker_tma(const Ctx &x, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                                           const PoolParams &p)
 {
     Bars &B = *x.bars;
     int issued = 0;
-    for (int i = 0; i < x.NC; ++i) {
-        const int s = i & 1;
-        if (i >= 2 && !wait_bar(&B.st_empty[s], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 1)) break;
-        const int c = chunk_of<DIR>(x, i);
-        uint8_t *st = x.smem + kPStage + s * kPStageBytes;
+    for (int i = 0;; ++i) {
+        const int s = i % kNS;
+        if (i >= kNS && !wait_bar(&B.st_empty[s], ((i / kNS) + 1) & 1, x.abort_flag, p.err, 1)) break;
+        const int k = atomicAdd(p.work, 1);
+        if (k >= p.n_items) {
+            B.sitem[s] = -1;
+            mbar_arrive(&B.it_full[s]);
+            mbar_arrive(&B.st_full[s]);
+            break;
+        }
+        const Item it = decode_item(p, k);
+        B.sitem[s] = k;
+        mbar_arrive(&B.it_full[s]);
+        uint8_t *st = x.smem + kWStage + s * kWStageBytes;
         mbar_arrive_expect_tx(&B.st_full[s], 32768);
         for (int kb = 0; kb < 2; ++kb) {
-            tma_load_3d(st + kb * 16384, tmQ, &B.st_full[s], kb * 64, c * kC, x.bh);
-            tma_load_3d(st + kb * 16384 + 8192, tmK, &B.st_full[s], kb * 64, c * kC, x.bh);
+            tma_load_3d(st + kb * 16384, tmQ, &B.st_full[s], kb * 64, it.c * kC, it.bh);
+            tma_load_3d(st + kb * 16384 + 8192, tmK, &B.st_full[s], kb * 64, it.c * kC, it.bh);
         }
         issued = i + 1;
     }
     if (*x.abort_flag)
-        for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) drain_copies(&B.st_full[i & 1], (i >> 1) & 1);
+        for (int i = (issued > kNS ? issued - kNS : 0); i < issued; ++i) drain_copies(&B.st_full[i % kNS], (i / kNS) & 1);
 }
 
-// MMA issue: [Q;K] K^T of chunk i, then P [T1 | T2] and [P T1; T1] K of chunk i - 1.
-__device__ __forceinline__ void prep_mma(const Ctx &x, const PairParams &p)
+// Gate warps (64 threads): the gates of each item in log2 form, as soon as the
+// item is handed out: G (inclusive prefix sum of log2 a in scan order), gamma,
+// b, b gamma, e = 2^(G_end - G), and the row/column factors of the decay ratios.
+__device__ __forceinline__ void worker_gates(const Ctx &x, const PoolParams &p, int gpt)
+{
+    Bars &B = *x.bars;
+    const int lane = gpt & 31;
+    for (int i = 0;; ++i) {
+        const int s = i % kNS, gj = i % kNG;
+        if (!wait_bar(&B.it_full[s], (i / kNS) & 1, x.abort_flag, p.err, 2)) break;
+        if (i >= kNG && !wait_bar(&B.g_empty[gj], ((i / kNG) + 1) & 1, x.abort_flag, p.err, 3)) break;
+        const int k = B.sitem[s];
+        if (k < 0) {   // past the last item: pass the end on
+            named_bar(kBarGate, 64);
+            if (gpt == 0) {
+                B.gitem[gj] = -1;
+                mbar_arrive(&B.g_full[gj]);
+            }
+            break;
+        }
+        const Item it = decode_item(p, k);
+        const int dir = it.dir;
+        float *gt = gates_buf(x, gj);
+        // scan position gpt is token pp of the chunk; tokens past T are identity tokens
+        const int pp = dir ? (63 - gpt) : gpt;
+        const int t = it.c * kC + pp;
+        float v = 0.f, bcur = 0.f;
+        if (t < x.T) {
+            v = fmaxf(log2f(__ldg(p.decay + (size_t)it.bh * x.T + t)), -120.f);   // decay below 2^-120 acts as 2^-120
+            bcur = __ldg(p.beta + (size_t)it.bh * x.T + t);
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += y;
+        }
+        if (gpt == 31) B.s_wsum = v;
+        named_bar(kBarGate, 64);
+        {
+            const float G = (gpt >= 32) ? v + B.s_wsum : v;
+            gt[gG * 64 + pp] = G;
+            const float gam = exp2f(G);
+            gt[gGam * 64 + pp] = gam;
+            gt[gBet * 64 + pp] = bcur;
+            gt[gBG * 64 + pp] = bcur * gam;
+        }
+        named_bar(kBarGate, 64);
+        // references: scan positions 15 (first half), 47 (second half), 31 (boundary)
+        const float R1 = gt[gG * 64 + (dir ? 48 : 15)];
+        const float R2 = gt[gG * 64 + (dir ? 16 : 47)];
+        const float Rm = gt[gG * 64 + (dir ? 32 : 31)];
+        const float G0 = gt[gG * 64 + (dir ? 63 : 0)];
+        const float G32 = gt[gG * 64 + (dir ? 31 : 32)];
+        const float Gend = gt[gG * 64 + (dir ? 0 : 63)];
+        // factorised decay products are exact while every factor is a normal float
+        const bool fact = (G0 - R1) <= 120.f && (R1 - Rm) <= 120.f && (G32 - R2) <= 120.f &&
+                          (R2 - Gend) <= 120.f;
+        {
+            const float G = gt[gG * 64 + gpt];
+            const int lp = dir ? 63 - gpt : gpt;
+            const float Rh = (lp >= 32) ? R2 : R1;
+            gt[gEb * 64 + gpt] = exp2f(Gend - G);
+            gt[gRA * 64 + gpt] = exp2f(G - Rh);
+            gt[gCA * 64 + gpt] = exp2f(Rh - G);
+            gt[gRB * 64 + gpt] = exp2f(G - Rm);
+            gt[gCB * 64 + gpt] = exp2f(Rm - G);
+            if (gpt == 0) {
+                B.gscal[gj][0] = Gend;
+                B.gscal[gj][1] = fact ? 1.f : 0.f;
+                B.gitem[gj] = k;
+            }
+        }
+        named_bar(kBarGate, 64);
+        if (gpt == 0) mbar_arrive(&B.g_full[gj]);
+    }
+}
+
+// MMA issue, per item j: P [T1 | T2] of item j, then [Q;K] K^T of item j + 2 (its
+// D1 buffer is free once item j's masks are read, which P [T1 | T2] follows),
+// then [P T1; T1] K of item j (after the finisher has read P [T1 | T2]).  The
+// [Q;K] K^T products run two items ahead of the solver.
+__device__ __forceinline__ void worker_mma(const Ctx &x, const PoolParams &p)
 {
     Bars &B = *x.bars;
     const uint32_t tm = x.tmem;
-    for (int i = 0; i <= x.NC; ++i) {
-        if (i < x.NC) {
-            const int s = i & 1;
-            if (!wait_bar(&B.st_full[s], (i >> 1) & 1, x.abort_flag, p.err, 2)) break;
-            if (i >= 2 && !wait_bar(&B.d1_empty[s], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 3)) break;
-            const uint32_t sQK = x.sbase + kPStage + s * kPStageBytes;
-            const uint64_t a = sw128_desc(sQK, 16, 1024), b = sw128_desc(sQK + 8192, 16, 1024);
-            tc_fence_after();
-            mma_run<4, 2, 2>(tm + kTD1 + 64 * s, a, b, kIdM1, false);
-            mma_run<4, 2, 2>(tm + kTD1 + 64 * s, a + 1024, b + 1024, kIdM1, true);
-            mma_commit(&B.d1_full[s]);
-            tr(p, x, 0, 16, i);
-        }
-        if (i == 0) continue;
-        const int j = i - 1, bj = j & 1;
-        if (!wait_bar(&B.tp_full[bj], (j >> 1) & 1, x.abort_flag, p.err, 4)) break;
-        if (j >= 1 && !wait_bar(&B.d2_empty, (j - 1) & 1, x.abort_flag, p.err, 5)) break;
+    // [Q;K] K^T of item i: 1 issued, 0 no such item (the end), -1 inputs not ready
+    // yet (only when !block), -2 abort
+    auto issue_m1 = [&](int i, bool block) -> int {
+        const int s = i % kNS, b1 = i & 1;
+        if (!block && !(mbar_test_wait(&B.st_full[s], (i / kNS) & 1) &&
+                        (i < 2 || mbar_test_wait(&B.d1_empty[b1], ((i >> 1) + 1) & 1))))
+            return -1;
+        if (!wait_bar(&B.st_full[s], (i / kNS) & 1, x.abort_flag, p.err, 4)) return -2;
+        if (B.sitem[s] < 0) return 0;
+        if (i >= 2 && !wait_bar(&B.d1_empty[b1], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 5)) return -2;
+        const uint32_t sQK = x.sbase + kWStage + s * kWStageBytes;
+        const uint64_t a = sw128_desc(sQK, 16, 1024), b = sw128_desc(sQK + 8192, 16, 1024);
+        tc_fence_after();
+        mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a, b, kIdM1, false);
+        mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a + 1024, b + 1024, kIdM1, true);
+        mma_commit(&B.d1_full[b1]);
+        tr(p, 0, 16, i);
+        return 1;
+    };
+    int last = -1;   // the number of items, once the end has been seen
+    int next = 0;    // next item whose [Q;K] K^T is to be issued
+    auto step_m1 = [&](bool block) -> bool {   // false on abort
+        if (last >= 0) return true;
+        const int r = issue_m1(next, block);
+        if (r == -2) return false;
+        if (r == 0) last = next;
+        if (r == 1) ++next;
+        return true;
+    };
+    bool ok = step_m1(true) && step_m1(true);
+    for (int j = 0; ok && (last < 0 || j < last); ++j) {
+        const int bj = j & 1;
+        if (!wait_bar(&B.tp_full[bj], (j >> 1) & 1, x.abort_flag, p.err, 6)) break;
+        if (j >= 1 && !wait_bar(&B.d2_empty, (j - 1) & 1, x.abort_flag, p.err, 7)) break;
         const uint32_t tb = x.sbase + kPTB + bj * 32768;
         tc_fence_after();
         // P [T1 | T2]: B is MN-major, the T1 and T2 tiles are its two 64-column groups
-        mma_run<4, 2, 128>(tm + kTD2, sw128_desc(x.sbase + kPP + bj * 8192, 16, 1024),
+        mma_run<4, 2, 128>(tm + kTD2, sw128_desc(x.sbase + kPP, 16, 1024),
                            sw128_desc(tb + 8192, 16384, 1024), kIdM2, false);
         mma_commit(&B.d2_full);
-        mma_commit(&B.p_free[bj]);
-        tr(p, x, 0, 17, j);
-        if (!wait_bar(&B.e2_done, j & 1, x.abort_flag, p.err, 6)) break;
-        if (j >= 1 && !wait_bar(&B.d3_empty, (j - 1) & 1, x.abort_flag, p.err, 7)) break;
+        mma_commit(&B.p_free);
+        tr(p, 0, 17, j);
+        // item j + 2's [Q;K] K^T now if its tiles are in, else after [P T1; T1] K
+        if (next == j + 2 && !step_m1(false)) break;
+        if (!wait_bar(&B.e2_done, j & 1, x.abort_flag, p.err, 8)) break;
+        if (j >= 1 && !wait_bar(&B.d3_empty, (j - 1) & 1, x.abort_flag, p.err, 9)) break;
         tc_fence_after();
         // [P T1; T1] K: B = K [token][dk] MN-major, dk groups 16 KB apart in the stage
         mma_run<4, 2, 128>(tm + kTD3, sw128_desc(tb, 16, 1024),
-                           sw128_desc(x.sbase + kPStage + bj * kPStageBytes + 8192, 16384, 1024), kIdM3, false);
+                           sw128_desc(x.sbase + kWStage + (j % kNS) * kWStageBytes + 8192, 16384, 1024), kIdM3, false);
         mma_commit(&B.d3_full);
         mma_commit(&B.t_free[bj]);
-        tr(p, x, 0, 18, j);
+        tr(p, 0, 18, j);
+        if (next == j + 2 && !step_m1(true)) break;
     }
     drain_mmas(B);
 }
 
 // Mask epilogue of this warp's 32 physical columns [32 hf, +32) of one row of
-// [Q;K] K^T, in four groups of 8 (a loop: this code runs once per chunk, so its
-// size costs more than its instruction count).  Rows 0-63 (TMEM quarters 0-1)
-// give P row r: j kept at or before r in scan order; rows 64-127 give A row r,
-// written in scan order: j strictly before r, times b_r.  The decay ratio
-// 2^(G_r - G_j) is a product of a row and a column factor when the chunk's
-// factors are all normal floats (`fact`), else one exp2 of the difference.
-template <int DIR>
+// [Q;K] K^T, in four groups of 8.  Rows 0-63 (TMEM quarters 0-1) give P row r:
+// j kept at or before r in scan order; rows 64-127 give A row r, written in
+// scan order: j strictly before r, times b_r.  The decay ratio 2^(G_r - G_j) is
+// a product of a row and a column factor when the chunk's factors are all
+// normal floats (`fact`), else one exp2 of the difference.
 __device__ __forceinline__ void mask_rows(uint32_t taddr, const float *gt, float *As, uint8_t *sP, int qd,
-                                          int lane, int hf, bool fact)
+                                          int lane, int hf, bool fact, int dir)
 {
     const int r = (qd & 1) * 32 + lane;                  // physical token row
-    const int lr = DIR ? 63 - r : r;                     // its scan position
+    const int lr = dir ? 63 - r : r;                     // its scan position
     const bool pm = qd < 2;                              // P (else A)
-    const bool useB = lr >= 32 && (DIR ? (hf == 1) : (hf == 0));   // cross-half pairs
+    const bool useB = lr >= 32 && (dir ? (hf == 1) : (hf == 0));   // cross-half pairs
     const float *cf = gt + (useB ? gCB : gCA) * 64 + 32 * hf;
     const float br = pm ? 1.f : gt[gBet * 64 + r];
     const float rf = br * gt[(useB ? gRB : gRA) * 64 + r];
@@ -320,16 +453,16 @@ __device__ __forceinline__ void mask_rows(uint32_t taddr, const float *gt, float
 #pragma unroll
             for (int u = 0; u < 8; ++u) xv[u] *= br * exp2f(Gr - gt[gG * 64 + j0 + u]);
         }
+        // kept columns of the group: u in [lo, hi)
+        const int rel = r - j0;
+        const int lo = dir ? (pm ? rel : rel + 1) : 0;
+        const int hi = dir ? 8 : (pm ? rel + 1 : rel);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = j0 + u;
-            const bool keep = pm ? (DIR ? (j >= r) : (j <= r)) : (DIR ? (j > r) : (j < r));
-            if (!keep) xv[u] = 0.f;
-        }
+        for (int u = 0; u < 8; ++u) xv[u] = (u >= lo && u < hi) ? xv[u] : 0.f;
         if (pm) {
             st_tile_v4(sP, sw128_off(r, j0), pack_bf16(xv[0], xv[1]), pack_bf16(xv[2], xv[3]),
                        pack_bf16(xv[4], xv[5]), pack_bf16(xv[6], xv[7]));
-        } else if (DIR) {   // scan-order columns 63 - j run backwards
+        } else if (dir) {   // scan-order columns 63 - j run backwards
             float4 *dst = reinterpret_cast<float4 *>(As + lr * kLDA + 56 - j0);
             dst[0] = make_float4(xv[7], xv[6], xv[5], xv[4]);
             dst[1] = make_float4(xv[3], xv[2], xv[1], xv[0]);
@@ -341,167 +474,90 @@ __device__ __forceinline__ void mask_rows(uint32_t taddr, const float *gt, float
     }
 }
 
-// Solver groups (two groups of 4 warps, warp w reading TMEM lane quarter
-// qd = w % 4): group g takes the chunks i with i % 2 == g, so that two chunks'
-// solves, each a long chain of dependent steps, run at once.  Per chunk: the
-// masks of [Q;K] K^T, then T = (I + A)^-1 written as T1 = T diag(b gamma) and
-// T2 = T diag(b); meanwhile the group's gate threads prepare the gates of its
-// next chunk.  pt is the thread's index in its group (0..127).
-template <int DIR>
-__device__ __forceinline__ void prep_solver(const Ctx &x, const PairParams &p, int pt, int qd, int g)
+// Solver group (8 warps; warp w reads TMEM lane quarter qd = w % 4 and columns
+// [32 hf, +32) of each row it owns): per item, the masks of [Q;K] K^T, then
+// T = (I + A)^-1 written as T1 = T diag(b gamma) and T2 = T diag(b).
+__device__ __forceinline__ void worker_solver(const Ctx &x, const PoolParams &p, int pt, int qd, int hf)
 {
     Bars &B = *x.bars;
     const int lane = pt & 31;
-    const int bar = g ? kBarA2 : kBarA, gbar = g ? kBarGate2 : kBarGate;
-    float *As = reinterpret_cast<float *>(x.smem + kPA + g * kPAStride);
+    float *As = reinterpret_cast<float *>(x.smem + kPA);
     const uint32_t tm_lane = (uint32_t)(qd * 32) << 16;
-    const float *beta_h = p.beta + (size_t)x.bh * x.T;
-    const float *decay_h = p.decay + (size_t)x.bh * x.T;
-
-    // gate threads: pt 64..127 (scan position gpt), on their own 64-thread barrier
-    const bool gate_thr = pt >= 64;
-    const int gpt = pt - 64;
-    float ra = 1.f, rb = 0.f;
-    auto load_raw = [&](int j) {
-        ra = 1.f;
-        rb = 0.f;
-        if (gate_thr && j < x.NC) {
-            const int pp = DIR ? (63 - gpt) : gpt;
-            const int t = chunk_of<DIR>(x, j) * kC + pp;
-            if (t < x.T) {   // padded tokens: identity (b = 0, log decay = 0)
-                ra = __ldg(decay_h + t);
-                rb = __ldg(beta_h + t);
-            }
-        }
-    };
-    auto compute_gates = [&](int j) {
-        const int gj = j % kNG;
-        float *gt = gates_buf(x, gj);
-        if (j >= kNG) wait_bar(&B.g_empty[gj], ((j / kNG) + 1) & 1, x.abort_flag, p.err, 8);
-        float v = fmaxf(log2f(ra), -120.f);   // decay below 2^-120 acts as 2^-120
-        const float bcur = rb;
-        load_raw(j + 2);
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, v, off);
-            if (lane >= off) v += y;
-        }
-        if (gpt == 31) x.bars->s_wsum[g] = v;
-        named_bar(gbar, 64);
-        {
-            const float G = (gpt >= 32) ? v + x.bars->s_wsum[g] : v;
-            const int pp = DIR ? (63 - gpt) : gpt;
-            gt[gG * 64 + pp] = G;
-            const float gam = exp2f(G);
-            gt[gGam * 64 + pp] = gam;
-            gt[gBet * 64 + pp] = bcur;
-            gt[gBG * 64 + pp] = bcur * gam;
-        }
-        named_bar(gbar, 64);
-        // references: scan positions 15 (first half), 47 (second half), 31 (boundary)
-        const float R1 = gt[gG * 64 + (DIR ? 48 : 15)];
-        const float R2 = gt[gG * 64 + (DIR ? 16 : 47)];
-        const float Rm = gt[gG * 64 + (DIR ? 32 : 31)];
-        const float G0 = gt[gG * 64 + (DIR ? 63 : 0)];
-        const float G32 = gt[gG * 64 + (DIR ? 31 : 32)];
-        const float Gend = gt[gG * 64 + (DIR ? 0 : 63)];
-        // factorised decay products are exact while every factor is a normal float
-        const bool fact = (G0 - R1) <= 120.f && (R1 - Rm) <= 120.f && (G32 - R2) <= 120.f &&
-                          (R2 - Gend) <= 120.f;
-        {
-            const float G = gt[gG * 64 + gpt];
-            const int lp = DIR ? 63 - gpt : gpt;
-            const float Rh = (lp >= 32) ? R2 : R1;
-            gt[gEb * 64 + gpt] = exp2f(Gend - G);
-            gt[gRA * 64 + gpt] = exp2f(G - Rh);
-            gt[gCA * 64 + gpt] = exp2f(Rh - G);
-            gt[gRB * 64 + gpt] = exp2f(G - Rm);
-            gt[gCB * 64 + gpt] = exp2f(Rm - G);
-            if (gpt == 0) {
-                x.bars->gscal[gj][0] = Gend;
-                x.bars->gscal[gj][1] = fact ? 1.f : 0.f;
-            }
-        }
-        named_bar(gbar, 64);
-        if (gpt == 0) mbar_arrive(&B.g_full[gj]);
-    };
-    load_raw(g);
-
-    // the first step only computes the gates of the group's first chunk
 #pragma unroll 1
-    for (int i = g - 2; i < x.NC; i += 2) {
-        const int b = g;   // = i & 1: this group's P, T and D1 buffers
-        const int gi = (i + 2 * kNG) % kNG;
-        float *gt = gates_buf(x, gi);
+    for (int i = 0;; ++i) {
+        const int b = i & 1, gi = i % kNG;
+        const float *gt = gates_buf(x, gi);
         uint8_t *tb = x.smem + kPTB + b * 32768;
-        if (i >= 0) {
-            const bool fact = x.bars->gscal[gi][1] != 0.f;
-            if (pt == 0) tr(p, x, 0, 0, i);
-            wait_bar(&B.d1_full[b], (i >> 1) & 1, x.abort_flag, p.err, 9);
-            if (i >= 2) wait_bar(&B.p_free[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 10);
-            if (pt == 0) tr(p, x, 0, 1, i);
-            tc_fence_after();
-            uint8_t *sP = x.smem + kPP + b * 8192;
-#pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf)
-                mask_rows<DIR>(x.tmem + tm_lane + kTD1 + 64 * b + 32 * hf, gt, As, sP, qd, lane, hf, fact);
-            if (pt == 0) tr(p, x, 0, 7, i);
-            tc_fence_before();
-            fence_proxy_async_smem();
-            if (named_bar_any(bar, 128, *x.abort_flag)) return;
-            if (pt == 0) mbar_arrive(&B.d1_empty[b]);
-            if (pt == 0) tr(p, x, 0, 2, i);
-        }
-
-        // T = (I + A)^-1; meanwhile the gate threads prepare the group's next chunk's gates
-        if (gate_thr && i + 2 < x.NC) compute_gates(i + 2);
-        if (i < 0) {
-            named_bar(bar, 128);
-            continue;
-        }
-        // T1 / T2 of this buffer must be done with (chunk i - 2: its products and its ring copy)
-        if (i >= 2) wait_bar(&B.t_free[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 11);
-        if (pt == 0) tr(p, x, 0, 3, i);
-        solve_diag_blocks<0, 0>(As, gt, tb + 8192, tb + 24576, nullptr, DIR, pt, bar, 128);
-        if (pt == 0) tr(p, x, 0, 4, i);
-        // the six strips below the diagonal blocks and the diagonal blocks' T1, T2:
-        // eight pieces of work, two for each of the group's warps
-        solve_off_diag_compact(As, gt, tb + 8192, tb + 24576, DIR, pt);
-        solve_off_diag_compact(As, gt, tb + 8192, tb + 24576, DIR, pt + 128);
-        if ((pt & 31) == 0) tr(p, x, 0, 20 + (pt >> 5) + 4 * g, i);
+        if (pt == 0) tr(p, 0, 0, i);
+        wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 10);
+        const int k = B.gitem[gi];
+        if (named_bar_any(kBarA, kGroup, *x.abort_flag || k < 0)) return;
+        const int dir = decode_item(p, k).dir;
+        const bool fact = B.gscal[gi][1] != 0.f;
+        wait_bar(&B.d1_full[b], (i >> 1) & 1, x.abort_flag, p.err, 11);
+        if (i >= 1) wait_bar(&B.p_free, (i - 1) & 1, x.abort_flag, p.err, 12);   // P of item i - 1 is read
+        if (pt == 0) tr(p, 0, 1, i);
+        tc_fence_after();
+        mask_rows(x.tmem + tm_lane + kTD1 + 64 * b + 32 * hf, gt, As, x.smem + kPP, qd, lane, hf, fact, dir);
+        tc_fence_before();
         fence_proxy_async_smem();
-        if (named_bar_any(bar, 128, *x.abort_flag)) return;
+        if (named_bar_any(kBarA, kGroup, *x.abort_flag)) return;
+        if (pt == 0) mbar_arrive(&B.d1_empty[b]);
+        if (pt == 0) tr(p, 0, 2, i);
+        // T1 / T2 of this buffer must be done with (item i - 2: its products and its ring copy)
+        if (i >= 2) wait_bar(&B.t_free[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 13);
+        if (pt == 0) tr(p, 0, 3, i);
+        solve_diag_blocks<kBarA, kGroup>(As, gt, tb + 8192, tb + 24576, nullptr, dir, pt);
+        if (pt == 0) tr(p, 0, 4, i);
+        solve_off_diag_compact(As, gt, tb + 8192, tb + 24576, dir, pt);
+        fence_proxy_async_smem();
+        if (named_bar_any(kBarA, kGroup, *x.abort_flag)) return;
         if (pt == 0) mbar_arrive(&B.tp_full[b]);
-        if (pt == 0) tr(p, x, 0, 5, i);
+        if (pt == 0) tr(p, 0, 5, i);
     }
 }
 
-// Finisher group (4 warps, warp w reads TMEM lane quarter qd = w % 4): P T1 and
-// P T2 into the operand tiles, Q' = gamma Q - P T1 K and -W = -T1 K into A2,
-// then the chunk's ring slot.
-template <int DIR>
-__device__ __forceinline__ void prep_finisher(const Ctx &x, const PairParams &p, int ft, int qd)
+// Finisher group (4 warps, warp w reads TMEM lane quarter qd = w % 4): per item,
+// P T1 and P T2 into the operand tiles, Q' = gamma Q - P T1 K and -W = -T1 K into
+// A2, then the item's slot in its scan's ring.
+__device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &p, int ft, int qd)
 {
     Bars &B = *x.bars;
     const int lane = ft & 31;
     const uint32_t tm_lane = (uint32_t)(qd * 32) << 16;
-    const uint32_t slot_full_remote = mapa_shared(smem_u32(&B.slot_full[0]), 1);
-    int issued = 0;   // leader: chunks whose ring copies were issued
-    // leader, once chunk j's copies have completed: publish the slot to the chain
-    auto publish = [&](int j) {
+    int pend_scan = -1, pend_c = 0, pend_b = -1;   // leader: the item whose ring copies are in flight
+    // leader: once the copies have read their sources, the A1 tile goes back to the
+    // solver and A2 staging is free again
+    auto release_sources = [&]() {
+        if (pend_b < 0) return;
+        bulk_wait_read0();
+        mbar_arrive(&B.t_free[pend_b]);
+        pend_b = -1;
+    };
+    // leader: once the copies have completed, the slot is published to the scan's chain
+    auto publish = [&]() {
+        if (pend_scan < 0) return;
+        release_sources();
+        bulk_wait0();
         fence_proxy_async_global();
-        mbar_arrive_remote(slot_full_remote + 8u * (j % kNSlot));
+        __threadfence();
+        st_release_gpu(p.slot_seq + (size_t)pend_scan * kNSlot + pend_c % kNSlot, pend_c + 1);
+        pend_scan = -1;
     };
 #pragma unroll 1
-    for (int i = 0; i < x.NC; ++i) {
+    for (int i = 0;; ++i) {
         const int b = i & 1, gi = i % kNG;
         uint8_t *tb = x.smem + kPTB + b * 32768;
         const float *gt = gates_buf(x, gi);
+        wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 14);
+        const int k = B.gitem[gi];
+        if (named_bar_any(kBarB, kGroupB, *x.abort_flag || k < 0)) break;
+        const Item it = decode_item(p, k);
 
         // ---- P [T1 | T2] (M = 64: lanes 0-15 of quarter qd hold rows 16 qd ..)
-        if (ft == 0) tr(p, x, 0, 8, i);
-        wait_bar(&B.d2_full, i & 1, x.abort_flag, p.err, 12);
-        if (ft == 0) tr(p, x, 0, 9, i);
+        if (ft == 0) tr(p, 0, 8, i);
+        wait_bar(&B.d2_full, i & 1, x.abort_flag, p.err, 15);
+        if (ft == 0) tr(p, 0, 9, i);
         tc_fence_after();
         {
             float v[32];
@@ -518,24 +574,23 @@ __device__ __forceinline__ void prep_finisher(const Ctx &x, const PairParams &p,
         }
         tc_fence_before();
         fence_proxy_async_smem();
-        // the previous chunk's ring copies have completed: its slot can be published
-        if (ft == 0 && i > 0) bulk_wait0();
+        // the previous item's ring copies complete here (measured: the best place;
+        // releasing the A1 tile earlier stalls the finisher's leader instead)
+        if (ft == 0) publish();
         if (named_bar_any(kBarB, kGroupB, *x.abort_flag)) break;
         if (ft == 0) {
             mbar_arrive(&B.e2_done);
             mbar_arrive(&B.d2_empty);
-            if (i > 0) publish(i - 1);
         }
-        if (ft == 0) tr(p, x, 0, 10, i);
+        if (ft == 0) tr(p, 0, 10, i);
 
         // ---- A2 = [gamma Q - P T1 K; -T1 K]
-        // (the waits below also order this group's reads of the gates, of the Q tile
-        // and of the solver's T2 rows after the writes that published them)
-        wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 13);
-        wait_bar(&B.st_full[b], (i >> 1) & 1, x.abort_flag, p.err, 16);
+        // (the waits below also order this group's reads of the Q tile and of the
+        // solver's T2 rows after the writes that published them)
+        wait_bar(&B.st_full[i % kNS], (i / kNS) & 1, x.abort_flag, p.err, 16);
         wait_bar(&B.tp_full[b], (i >> 1) & 1, x.abort_flag, p.err, 17);
-        wait_bar(&B.d3_full, i & 1, x.abort_flag, p.err, 14);
-        if (ft == 0) tr(p, x, 0, 11, i);
+        wait_bar(&B.d3_full, i & 1, x.abort_flag, p.err, 18);
+        if (ft == 0) tr(p, 0, 11, i);
         tc_fence_after();
         {
             const int n = 32 * qd + lane;   // row of [P T1; T1] K
@@ -543,7 +598,7 @@ __device__ __forceinline__ void prep_finisher(const Ctx &x, const PairParams &p,
             float v[32];
 #pragma unroll 1
             for (int kb = 0; kb < 2; ++kb) {
-                const uint8_t *qrow = x.smem + kPStage + b * kPStageBytes + kb * 16384;   // Q, key block kb
+                const uint8_t *qrow = x.smem + kWStage + (i % kNS) * kWStageBytes + kb * 16384;   // Q, key block kb
                 uint8_t *a2 = x.smem + kPA2 + kb * 16384;
 #pragma unroll 1
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -574,51 +629,49 @@ __device__ __forceinline__ void prep_finisher(const Ctx &x, const PairParams &p,
                 *reinterpret_cast<const float4 *>(gt + gEb * 64 + 4 * ft);
         } else if (ft == 16) {
             *reinterpret_cast<float4 *>(x.smem + kPGst + 256) =
-                make_float4(exp2f(x.bars->gscal[gi][0]), 0.f, 0.f, 0.f);
+                make_float4(exp2f(B.gscal[gi][0]), 0.f, 0.f, 0.f);
         }
         tc_fence_before();
         fence_proxy_async_smem();
         if (named_bar_any(kBarB, kGroupB, *x.abort_flag)) break;
         if (ft == 0) {
             mbar_arrive(&B.d3_empty);
-            mbar_arrive(&B.st_empty[b]);
+            mbar_arrive(&B.st_empty[i % kNS]);
             mbar_arrive(&B.g_empty[gi]);
         }
-        if (ft == 0) tr(p, x, 0, 12, i);
+        if (ft == 0) tr(p, 0, 12, i);
 
-        // ---- ring slot: A1, A2, e, gamma_end (bulk copies, published a chunk later)
+        // ---- the item's slot: A1, A2, e, gamma_end (bulk copies, published an item later)
         if (ft == 0) {
-            tr(p, x, 0, 13, i);
-            const int s = i % kNSlot;
-            if (i < kNSlot || wait_cluster(&B.slot_empty[s], ((i / kNSlot) + 1) & 1, x.abort_flag, p.err, 15)) {
-                uint8_t *slot = x.ring + (size_t)s * kSlotBytes;
+            // the slot's previous chunk must have been taken out by the chain
+            if (it.ci < kNSlot || wait_global(p.consumed + it.scan, it.ci - kNSlot + 1, x, p, 64)) {
+                uint8_t *slot = p.ring + ((size_t)it.scan * kNSlot + it.ci % kNSlot) * kSlotBytes;
                 bulk_store(slot + kSlotA1, tb + 16384, 16384);
                 bulk_store(slot + kSlotA2, x.smem + kPA2, 32768);
                 bulk_store(slot + kSlotGates, x.smem + kPGst, 512);
                 bulk_commit();
-                issued = i + 1;
-                // once the copies have read them, the A1 tile goes back to the solver
-                // and A2 staging may be rewritten
-                bulk_wait_read0();
-                mbar_arrive(&B.t_free[b]);
+                pend_scan = it.scan;
+                pend_c = it.ci;
+                pend_b = b;
             }
-            tr(p, x, 0, 14, i);
+            tr(p, 0, 13, i);
         }
     }
     if (ft == 0) {
+        if (!*x.abort_flag) publish();
         bulk_wait0();
-        if (!*x.abort_flag && issued == x.NC) publish(x.NC - 1);
     }
 }
 
-// ================================================================== chain CTA
+// ================================================================== chains
 
 template <int DIR>
 __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, const CUtensorMap *tmV,
-                                          const PairParams &p)
+                                          const PoolParams &p)
 {
     Bars &B = *x.bars;
     int vk_issued = 0, a_issued = 0;
+    const int *seq = p.slot_seq + (size_t)x.scan * kNSlot;
     for (int i = 0; i < x.NC; ++i) {
         const int st = i % kNVK, ab = i & 1, s = i % kNSlot;
         if (i >= kNVK && !wait_bar(&B.vk_empty[st], ((i / kNVK) + 1) & 1, x.abort_flag, p.err, 21)) break;
@@ -631,9 +684,9 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
         tma_load_3d(sv + 24576, tmK, &B.vk_full[st], 64, c * kC, x.bh);
         vk_issued = i + 1;
         if (i >= 2 && !wait_bar(&B.a_empty[ab], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 22)) break;
-        tr(p, x, 1, 0, i);
-        if (!wait_cluster(&B.slot_full[s], (i / kNSlot) & 1, x.abort_flag, p.err, 23)) break;
-        tr(p, x, 1, 1, i);
+        tr(p, 1, 0, i);
+        if (!wait_global(seq + s, i + 1, x, p, 65)) break;
+        tr(p, 1, 1, i);
         fence_proxy_async_global();
         const uint8_t *slot = x.ring + (size_t)s * kSlotBytes;
         uint8_t *dst = x.smem + kCA + ab * kCABytes;
@@ -651,19 +704,18 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
     }
 }
 
-__device__ __forceinline__ void chain_mma(const Ctx &x, const PairParams &p)
+__device__ __forceinline__ void chain_mma(const Ctx &x, const PoolParams &p)
 {
     Bars &B = *x.bars;
     const uint32_t tm = x.tmem;
-    const uint32_t slot_empty_remote = mapa_shared(smem_u32(&B.slot_empty[0]), 0);
     for (int i = 0; i < x.NC; ++i) {
         const int st = i % kNVK, ab = i & 1, db = i & 1;
         if (!wait_bar(&B.vk_full[st], (i / kNVK) & 1, x.abort_flag, p.err, 24)) break;
         if (!wait_bar(&B.a_full[ab], (i >> 1) & 1, x.abort_flag, p.err, 25)) break;
-        mbar_arrive_remote(slot_empty_remote + 8u * (i % kNSlot));   // the slot's data has landed
-        tr(p, x, 1, 2, i);
+        st_release_gpu(p.consumed + x.scan, i + 1);   // the slot's data has landed: it may be refilled
+        tr(p, 1, 2, i);
         if (i >= 2 && !wait_bar(&B.d_empty[db], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 26)) break;
-        tr(p, x, 1, 3, i);
+        tr(p, 1, 3, i);
         const uint32_t sv = x.sbase + kCStage + st * 32768;
         const uint32_t sa = x.sbase + kCA + ab * kCABytes;
         const uint32_t dD = tm + kTD + 128 * db;
@@ -671,7 +723,7 @@ __device__ __forceinline__ void chain_mma(const Ctx &x, const PairParams &p)
         // D = V^T A1^T: A = V (MN-major, dv groups 8 KB apart), B = A1 (K-major)
         mma_run<4, 128, 2>(dD, sw128_desc(sv, 8192, 1024), sw128_desc(sa + kSlotA1, 16, 1024), kIdA, false);
         if (!wait_bar(&B.h_full, i & 1, x.abort_flag, p.err, 27)) break;
-        tr(p, x, 1, 4, i);
+        tr(p, 1, 4, i);
         tc_fence_after();
         // D += H^T A2^T: A = H^T (bf16 in TMEM), B = A2 (K-major, key blocks 16 KB apart)
         {
@@ -683,7 +735,7 @@ __device__ __forceinline__ void chain_mma(const Ctx &x, const PairParams &p)
         mma_commit(&B.d_full[db]);
         mma_commit(&B.a_empty[ab]);
         if (!wait_bar(&B.u_full, i & 1, x.abort_flag, p.err, 28)) break;
-        tr(p, x, 1, 5, i);
+        tr(p, 1, 5, i);
         tc_fence_after();
         // S = Ubar^T K: A = Ubar^T (bf16 in TMEM), B = K (MN-major, dk groups 8 KB apart)
         {
@@ -703,12 +755,12 @@ __device__ __forceinline__ void chain_mma(const Ctx &x, const PairParams &p)
 // of U^T, scaled by e, into Ubar^T (bf16, TMEM); state epilogue: H^T <-
 // gamma_end H^T + S into registers and its bf16 copy into TMEM.
 template <int DIR>
-__device__ __forceinline__ void chain_state(const Ctx &x, const PairParams &p, int ct, int q, int h)
+__device__ __forceinline__ void chain_state(const Ctx &x, const PoolParams &p, int ct, int q, int h)
 {
     Bars &B = *x.bars;
     const int lane = ct & 31, d = 32 * q + lane;
     const uint32_t tl = (uint32_t)(32 * q) << 16;
-    const bool dbg = kDbgOn && p.debug != nullptr && x.dir == 0 && x.bh == 0;
+    const bool dbg = kDbgOn && p.debug != nullptr && x.scan == 0;
     float hs[64];
     {
         const float *s0 = (DIR == 0 && p.state_in) ? p.state_in + (size_t)x.bh * kDK * 128 + (size_t)(64 * h) * 128 + d
@@ -735,7 +787,7 @@ __device__ __forceinline__ void chain_state(const Ctx &x, const PairParams &p, i
         // ---- Ubar^T (e and gamma_end come with the chunk's ring slot)
         wait_bar(&B.a_full[ab], (i >> 1) & 1, x.abort_flag, p.err, 34);
         wait_bar(&B.d_full[db], (i >> 1) & 1, x.abort_flag, p.err, 31);
-        if (ct == 0) tr(p, x, 1, 8, i);
+        if (ct == 0) tr(p, 1, 8, i);
         tc_fence_after();
         {
             uint32_t w[16];
@@ -763,10 +815,10 @@ __device__ __forceinline__ void chain_state(const Ctx &x, const PairParams &p, i
             mbar_arrive(&B.u_full);
             mbar_arrive(&B.d_empty[db]);
         }
-        if (ct == 0) tr(p, x, 1, 9, i);
+        if (ct == 0) tr(p, 1, 9, i);
         // ---- H^T <- gamma_end H^T + S
         wait_bar(&B.s_full, i & 1, x.abort_flag, p.err, 32);
-        if (ct == 0) tr(p, x, 1, 10, i);
+        if (ct == 0) tr(p, 1, 10, i);
         tc_fence_after();
         {
             const float ge = eg[64];
@@ -796,10 +848,10 @@ __device__ __forceinline__ void chain_state(const Ctx &x, const PairParams &p, i
             mbar_arrive(&B.h_full);
             mbar_arrive(&B.a_empty[ab]);
         }
-        if (ct == 0) tr(p, x, 1, 11, i);
+        if (ct == 0) tr(p, 1, 11, i);
     }
     if (p.state_out) {
-        float *so = p.state_out + ((size_t)DIR * p.BH + x.bh) * kDK * 128 + (size_t)(64 * h) * 128 + d;
+        float *so = p.state_out + ((size_t)DIR * p.BH_all + x.bh) * kDK * 128 + (size_t)(64 * h) * 128 + d;
 #pragma unroll
         for (int j = 0; j < 64; ++j) so[(size_t)j * 128] = hs[j];
     }
@@ -810,28 +862,30 @@ __device__ __forceinline__ void chain_state(const Ctx &x, const PairParams &p, i
 // rows (the TMA layout of o) and written with one TMA store.  Bidirectional:
 // the first writer of a tile stores its bf16 partial and then publishes it on
 // the tile's counter; the second loads that partial by TMA (requested a chunk
-// ahead when the first writer is known in advance), adds its fp32 partial and
-// rounds once.
+// ahead), adds its fp32 partial and rounds once.
 template <int DIR>
-__device__ __forceinline__ void chain_out(const Ctx &x, const PairParams &p, const CUtensorMap *tmO, int ot, int q)
+__device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, const CUtensorMap *tmO, int ot, int q)
 {
     Bars &B = *x.bars;
     const int lane = ot & 31, d = 32 * q + lane;
     const uint32_t tl = (uint32_t)(32 * q) << 16;
     const bool lead = ot == 0;
-    const bool dbg = kDbgOn && p.debug != nullptr && x.dir == 0 && x.bh == 0;
+    const bool dbg = kDbgOn && p.debug != nullptr && x.scan == 0;
     // this thread's column in a staging tile: dv block d / 64, column d % 64
     const uint32_t dblk = (uint32_t)(d >> 6) * 8192u;
-    int nload[2] = {0, 0};   // partial loads issued into each staging tile so far
-    int loaded_ahead = -1;   // leader: the chunk whose partial load is already in flight
-    int nissued[2] = {0, 0}; // leader: partial loads issued into each staging tile
-    auto pred_first = [&](int c) { return DIR == ((2 * c < x.NC) ? 0 : 1); };
-    auto counter = [&](int c) { return p.counters + (size_t)x.bh * x.NC + c; };
+    int nload0 = 0, nload1 = 0;       // partial loads waited for, per staging tile
+    int nissued0 = 0, nissued1 = 0;   // leader: partial loads issued, per staging tile
+    int loaded_ahead = -1;            // leader: the chunk whose partial load is already in flight
+    const bool bidi = p.counters != nullptr;
+    // every CTA is resident: the forward scan reaches the first half of the
+    // chunks first, the reverse scan the second half
+    auto first_of = [&](int c) { return DIR == ((2 * c < x.NC) ? 0 : 1); };
+    auto counter = [&](int c) { return p.counters + (size_t)x.bhl * x.NC + c; };
     auto load_partial = [&](int c, int ob) {
         uint8_t *stg = x.smem + kCO + ob * 16384;
         fence_proxy_async_global();
         mbar_arrive_expect_tx(&B.o_full[ob], 16384);
-        ++nissued[ob];
+        if (ob) ++nissued1; else ++nissued0;
         tma_load_3d(stg, tmO, &B.o_full[ob], 0, c * kC, x.bh);
         tma_load_3d(stg + 8192, tmO, &B.o_full[ob], 64, c * kC, x.bh);
     };
@@ -839,29 +893,11 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PairParams &p, con
     for (int i = 0; i < x.NC; ++i) {
         const int db = i & 1, ob = i & 1, c = chunk_of<DIR>(x, i);
         uint8_t *stg = x.smem + kCO + ob * 16384;
-        const bool bidi = p.counters != nullptr;
-        bool first = true;
-        if (bidi) {
-            if (p.predict) {
-                // every cluster resident: the forward scan reaches the first half of the
-                // chunks first, the reverse scan the second half
-                first = pred_first(c);
-            } else {
-                // arrival order decided at run time by a claim on the counter
-                // (0 -> 1 -> 2); the first writer's published partial brings it to 3
-                if (lead) x.bars->s_old = atomicAdd(counter(c), 1);
-                named_bar(kBarB, kGroupB);
-                first = x.bars->s_old == 0;
-            }
-            if (!first && lead && loaded_ahead != i) {
-                bool ok = spin_global_at_least(counter(c), p.predict ? 1 : 3, x.abort_flag);
-                if (!ok) {
-                    if (!*x.abort_flag) atomicOr(p.err, 32);
-                    *x.abort_flag = 1;
-                } else {
-                    bulk_wait_read1();   // the staging tile's previous store has read it
-                    load_partial(c, ob);
-                }
+        const bool first = !bidi || first_of(c);
+        if (!first && lead && loaded_ahead != i) {
+            if (wait_global(counter(c), 1, x, p, 32)) {
+                bulk_wait_read1();   // the staging tile's previous store has read it
+                load_partial(c, ob);
             }
         }
         wait_bar(&B.d_full[db], (i >> 1) & 1, x.abort_flag, p.err, 33);
@@ -869,8 +905,9 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PairParams &p, con
         if (lead) bulk_wait_read1();
         if (named_bar_any(kBarB, kGroupB, *x.abort_flag)) break;
         if (!first) {
-            wait_bar(&B.o_full[ob], nload[ob] & 1, x.abort_flag, p.err, 35);
-            ++nload[ob];
+            int &nl = ob ? nload1 : nload0;
+            wait_bar(&B.o_full[ob], nl & 1, x.abort_flag, p.err, 35);
+            ++nl;
         }
         tc_fence_after();
 #pragma unroll 1
@@ -903,10 +940,10 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PairParams &p, con
                 __threadfence();
                 atomicAdd(counter(c), 1);
             }
-            // request the next tile's partial now if its first writer is known and done
-            if (bidi && p.predict && i + 1 < x.NC) {
+            // request the next tile's partial now if its first writer is done
+            if (bidi && i + 1 < x.NC) {
                 const int cn = chunk_of<DIR>(x, i + 1);
-                if (!pred_first(cn)) {
+                if (!first_of(cn)) {
                     int seen;
                     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(counter(cn)) : "memory");
                     if (seen >= 1) {
@@ -920,33 +957,35 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PairParams &p, con
     }
     if (lead) {
         bulk_wait0();   // every store performed before the CTA exits
-        for (int ob = 0; ob < 2; ++ob)   // partial loads still in flight after an abort
-            for (int k = nload[ob]; k < nissued[ob]; ++k) drain_copies(&B.o_full[ob], k & 1);
+        for (int k = nload0; k < nissued0; ++k) drain_copies(&B.o_full[0], k & 1);   // after an abort
+        for (int k = nload1; k < nissued1; ++k) drain_copies(&B.o_full[1], k & 1);
     }
 }
 
 // ================================================================== kernel
 
-__global__ void __launch_bounds__(kPThreads, 1)
-gdn_chunk_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                      const PairParams p)
+                      const PoolParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t rank = cluster_ctarank();
+    const bool chain = (int)blockIdx.x < p.n_scans;
 
     Ctx x;
     x.smem = smem;
     x.sbase = smem_u32(smem);
     x.bars = reinterpret_cast<Bars *>(smem + kOffBar);
     x.abort_flag = &x.bars->abort_flag;
-    x.dir = blockIdx.y;
-    x.bh = blockIdx.z;
     x.T = p.T;
     x.NC = p.n_chunks;
-    x.ring = p.ring + ((size_t)x.dir * p.BH + x.bh) * kNSlot * kSlotBytes;
+    x.scan = chain ? (int)blockIdx.x : 0;
+    x.dir = x.scan >= p.BH ? 1 : 0;
+    x.bhl = x.scan - x.dir * p.BH;
+    x.bh = p.bh0 + x.bhl;
+    x.ring = p.ring + (size_t)x.scan * kNSlot * kSlotBytes;
     Bars &B = *x.bars;
 
     if (tid == 0) {
@@ -954,57 +993,51 @@ gdn_chunk_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         const int nbar = (int)(offsetof(Bars, gscal) / sizeof(uint64_t));
         for (int k = 0; k < nbar; ++k) mbar_init(&all[k], 1);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&B.t_free[b], 2);    // [P T1; T1] K done, ring copy done
+            mbar_init(&B.t_free[b], 2);    // [P T1; T1] K done, ring copy read A1
             mbar_init(&B.a_empty[b], 2);   // D += H^T A2^T done, state epilogue done
             mbar_init(&B.d_empty[b], 2);   // output epilogue, U epilogue
         }
         B.abort_flag = 0;
         fence_mbar_init();
-        if (rank == 0) {
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-        } else {
+        if (chain) {
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmO);
+        } else {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
         }
     }
     if (warp == 0) {
         tmem_alloc(&B.tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (rank == 0) {
+    if (!chain) {
         float *As0 = reinterpret_cast<float *>(smem + kPA);
-        for (int i = tid; i < 2 * 64 * kLDA; i += kPThreads) As0[i] = 0.f;
-        // T1, T2: the triangle the solve never writes stays zero for the whole scan
+        for (int i = tid; i < 64 * kLDA; i += kThreads) As0[i] = 0.f;
+        // T1, T2: the triangle the solve never writes stays zero throughout
         for (int b = 0; b < 2; ++b) {
             uint32_t *t1 = reinterpret_cast<uint32_t *>(smem + kPTB + b * 32768 + 8192);
             uint32_t *t2 = reinterpret_cast<uint32_t *>(smem + kPTB + b * 32768 + 24576);
-            for (int i = tid; i < 8192 / 4; i += kPThreads) t1[i] = t2[i] = 0u;
+            for (int i = tid; i < 8192 / 4; i += kThreads) t1[i] = t2[i] = 0u;
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     x.tmem = B.tmem_slot;
-    cluster_sync_all();   // both CTAs' barriers are initialised before any remote arrival
 
-    if (rank == 0) {
+    if (!chain) {
         if (warp == 0) {
-            if (lane == 0) {
-                if (x.dir) prep_tma<1>(x, &tmQ, &tmK, p);
-                else prep_tma<0>(x, &tmQ, &tmK, p);
-            }
+            if (lane == 0) worker_tma(x, &tmQ, &tmK, p);
         } else if (warp == 1) {
-            if (lane == 0) prep_mma(x, p);
+            if (lane == 0) worker_mma(x, p);
         } else if (warp < 10) {
-            const int g = (warp - 2) >> 2, pt = tid - 64 - 128 * g, qd = warp & 3;
-            if (x.dir) prep_solver<1>(x, p, pt, qd, g);
-            else prep_solver<0>(x, p, pt, qd, g);
+            worker_solver(x, p, tid - 64, warp & 3, (warp - 2) >> 2);
+        } else if (warp < 14) {
+            worker_finisher(x, p, tid - 320, warp & 3);
         } else {
-            const int ft = tid - 320, qd = warp & 3;
-            if (x.dir) prep_finisher<1>(x, p, ft, qd);
-            else prep_finisher<0>(x, p, ft, qd);
+            worker_gates(x, p, tid - 448);
         }
     } else {
         if (warp == 0) {
@@ -1018,7 +1051,7 @@ gdn_chunk_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             const int ct = tid - 64, q = warp & 3, h = (warp - 2) >> 2;
             if (x.dir) chain_state<1>(x, p, ct, q, h);
             else chain_state<0>(x, p, ct, q, h);
-        } else {
+        } else if (warp < 14) {
             const int ot = tid - 320, q = warp & 3;
             if (x.dir) chain_out<1>(x, p, &tmO, ot, q);
             else chain_out<0>(x, p, &tmO, ot, q);
@@ -1028,7 +1061,6 @@ gdn_chunk_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(x.tmem, kTmemCols);
-    cluster_sync_all();   // the partner may address this CTA's barriers until it is done
 }
 
 // ------------------------------------------------------------------ host side
@@ -1069,11 +1101,10 @@ bool make_map(CUtensorMap *m, const void *base, int T, int BH)
 
 struct DevInfo {
     bool init = false;
-    int max_clusters = 0;   // 2-CTA clusters resident at once
+    int sms = 0;
 };
 
-// Per device: the kernel's shared-memory attribute and how many of its
-// clusters fit on the GPU at once.
+// Per device: the kernel's shared-memory attribute and the SM count.
 cudaError_t device_info(DevInfo **out)
 {
     static std::mutex mu;
@@ -1085,97 +1116,87 @@ cudaError_t device_info(DevInfo **out)
     std::lock_guard<std::mutex> lock(mu);
     DevInfo &d = info[dev];
     if (!d.init) {
-        err = cudaFuncSetAttribute(gdn_chunk_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        err = cudaFuncSetAttribute(gdn_chunk_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)kSmemAlloc);
+        if (err == cudaSuccess) err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
         if (err != cudaSuccess) return err;
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute at[1];
-        cfg.gridDim = dim3(2, 1, 1);
-        cfg.blockDim = dim3(kPThreads);
-        cfg.dynamicSmemBytes = kSmemAlloc;
-        at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = 2;
-        at[0].val.clusterDim.y = 1;
-        at[0].val.clusterDim.z = 1;
-        cfg.attrs = at;
-        cfg.numAttrs = 1;
-        int n = 0;
-        err = cudaOccupancyMaxActiveClusters(&n, gdn_chunk_pair_kernel, &cfg);
-        if (err != cudaSuccess) return err;
-        d.max_clusters = n;
         d.init = true;
     }
     *out = &d;
     return cudaSuccess;
 }
 
+// Workers kept beside the chains: a quarter of the SMs at least.
+int min_workers(int sms) { return sms / 4 > 8 ? sms / 4 : 8; }
+
 }  // namespace
 
-bool chunk_pair_supported(const FwdArgs &a)
+bool chunk_pool_supported(const FwdArgs &a)
 {
-    // chosen on request only (g_kernel_select == 2): on the measured workloads the
-    // single-CTA kernel is still the faster one
-    return g_kernel_select == 2 && !a.fp32 && a.dk == kDK && a.dv == 128 && a.n_seg == 1 &&
-           a.seg0 == 0 && a.seg_chunks == 0;
+    return g_kernel_select != 1 && !a.fp32 && a.dk == kDK && a.dv == 128 && a.n_seg == 1 && a.seg0 == 0 &&
+           a.seg_chunks == 0;
 }
 
-cudaError_t launch_chunk_pair(const FwdArgs &a, cudaStream_t stream)
+cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream)
 {
     CUtensorMap mq, mk, mv, mo;
-    const int BH = a.B * a.H;
-    if (!make_map(&mq, a.q, a.T, BH) || !make_map(&mk, a.k, a.T, BH) || !make_map(&mv, a.v, a.T, BH) ||
-        !make_map(&mo, a.o, a.T, BH))
+    const int BH_all = a.B * a.H;
+    if (!make_map(&mq, a.q, a.T, BH_all) || !make_map(&mk, a.k, a.T, BH_all) ||
+        !make_map(&mv, a.v, a.T, BH_all) || !make_map(&mo, a.o, a.T, BH_all))
         return cudaErrorInvalidValue;
     DevInfo *info = nullptr;
     cudaError_t err = device_info(&info);
     if (err != cudaSuccess) return err;
-
-    PairParams p;
-    p.beta = a.beta; p.decay = a.decay; p.state_in = a.state_in; p.state_out = a.state_out;
-    p.o = static_cast<__nv_bfloat16 *>(a.o);
-    p.BH = BH; p.T = a.T;
-    p.n_chunks = (a.T + kC - 1) / kC;
-    p.debug = g_debug_dump;
-    p.trace = g_prof_buf;
-    err = device_error_word(&p.err);
-    if (err != cudaSuccess) return err;
-
     const int dirs = a.bidi ? 2 : 1;
-    const size_t ring_bytes = (size_t)dirs * BH * kNSlot * kSlotBytes;
-    const size_t cnt_bytes = a.bidi ? (size_t)BH * p.n_chunks * sizeof(int) : 0;
-    uint8_t *ws = nullptr;
-    err = ws_alloc(reinterpret_cast<void **>(&ws), ring_bytes + cnt_bytes, stream);
-    if (err != cudaSuccess) return err;
-    p.ring = g_debug_ring ? static_cast<uint8_t *>(g_debug_ring) : ws;
-    p.counters = a.bidi ? reinterpret_cast<int *>(ws + ring_bytes) : nullptr;
-    if (a.bidi) err = cudaMemsetAsync(p.counters, 0, cnt_bytes, stream);
+    const int n_chunks = (a.T + kC - 1) / kC;
+    // heads per launch: every chain of a launch resident beside enough workers
+    const int wave = (info->sms - min_workers(info->sms)) / dirs;
+    if (wave < 1) return cudaErrorInvalidConfiguration;
+    const int heads = BH_all < wave ? BH_all : wave;
 
-    if (err == cudaSuccess) {
+    const size_t n_scans_max = (size_t)dirs * heads;
+    const size_t ring_bytes = n_scans_max * kNSlot * kSlotBytes;
+    const size_t flag_ints = n_scans_max * kNSlot + n_scans_max + 1 + (a.bidi ? (size_t)heads * n_chunks : 0);
+    uint8_t *ws = nullptr;
+    err = ws_alloc(reinterpret_cast<void **>(&ws), ring_bytes + flag_ints * sizeof(int), stream);
+    if (err != cudaSuccess) return err;
+    int *flags = reinterpret_cast<int *>(ws + ring_bytes);
+
+    for (int h0 = 0; h0 < BH_all && err == cudaSuccess; h0 += heads) {
+        PoolParams p;
+        p.beta = a.beta; p.decay = a.decay; p.state_in = a.state_in; p.state_out = a.state_out;
+        p.o = static_cast<__nv_bfloat16 *>(a.o);
+        p.BH = BH_all - h0 < heads ? BH_all - h0 : heads;
+        p.bh0 = h0;
+        p.BH_all = BH_all;
+        p.T = a.T;
+        p.n_chunks = n_chunks;
+        p.n_scans = dirs * p.BH;
+        p.n_items = p.n_scans * n_chunks;
+        p.debug = g_debug_dump;
+        p.trace = g_prof_buf;
+        p.ring = g_debug_ring ? static_cast<uint8_t *>(g_debug_ring) : ws;
+        p.slot_seq = flags;
+        p.consumed = flags + (size_t)p.n_scans * kNSlot;
+        p.work = p.consumed + p.n_scans;
+        p.counters = a.bidi ? p.work + 1 : nullptr;
+        err = device_error_word(&p.err);
+        if (err != cudaSuccess) break;
+        err = cudaMemsetAsync(flags, 0, flag_ints * sizeof(int), stream);
+        if (err != cudaSuccess) break;
+
         cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute at[2];
-        cfg.gridDim = dim3(2, dirs, BH);
-        cfg.blockDim = dim3(kPThreads);
+        cudaLaunchAttribute at[1];
+        cfg.gridDim = dim3(info->sms);
+        cfg.blockDim = dim3(kThreads);
         cfg.dynamicSmemBytes = kSmemAlloc;
         cfg.stream = stream;
-        at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = 2;
-        at[0].val.clusterDim.y = 1;
-        at[0].val.clusterDim.z = 1;
-        at[1].id = cudaLaunchAttributeCooperative;
-        at[1].val.cooperative = 1;
+        // chains and workers wait for one another: every CTA must be resident
+        at[0].id = cudaLaunchAttributeCooperative;
+        at[0].val.cooperative = 1;
         cfg.attrs = at;
-        // bidirectional: a cooperative launch makes every cluster resident (or is
-        // refused), so the first writer of each output tile can be fixed in advance
-        const bool coop = a.bidi && dirs * BH <= info->max_clusters;
-        cfg.numAttrs = coop ? 2 : 1;
-        p.predict = coop ? 1 : 0;
-        err = cudaLaunchKernelEx(&cfg, gdn_chunk_pair_kernel, mq, mk, mv, mo, p);
-        if (err != cudaSuccess && coop) {
-            (void)cudaGetLastError();
-            cfg.numAttrs = 1;
-            p.predict = 0;
-            err = cudaLaunchKernelEx(&cfg, gdn_chunk_pair_kernel, mq, mk, mv, mo, p);
-        }
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, gdn_chunk_pool_kernel, mq, mk, mv, mo, p);
         if (err == cudaSuccess) err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }
@@ -1187,11 +1208,11 @@ cudaError_t launch_chunk_pair(const FwdArgs &a, cudaStream_t stream)
 }  // namespace gdn
 
 // Test hooks (not part of the documented ABI).
-// gdn_debug_ring: a device buffer of at least dirs*B*H*4*49664 bytes that the
-// paired kernel uses as its operand ring instead of workspace (NULL: off), so
-// a test can read the prepared operands of each chunk back.
-// gdn_debug_kernel_select: 0 picks the kernel by shape, 1 forces the
-// single-CTA chunkwise kernel for every bf16 call, 2 asks for the paired-SM
-// kernel wherever it applies (dk = dv = 128, whole sequences).
+// gdn_debug_ring: a device buffer of at least dirs*B*H*8*49664 bytes that the
+// pooled kernel uses as its operand ring instead of workspace (NULL: off), so a
+// test can read back the prepared operands of each scan's last eight chunks.
+// gdn_debug_kernel_select: 0 or 2 pick the kernel by shape (the pooled kernel
+// for dk = dv = 128 whole sequences), 1 forces the single-CTA chunkwise kernel
+// for every bf16 call.
 extern "C" void gdn_debug_ring(void *device_buffer) { gdn::g_debug_ring = device_buffer; }
 extern "C" void gdn_debug_kernel_select(int which) { gdn::g_kernel_select = which; }

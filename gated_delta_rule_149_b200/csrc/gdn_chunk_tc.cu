@@ -1057,7 +1057,7 @@ bool chunk_tc_supported(const FwdArgs &a)
 
 cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
 {
-    if (chunk_pair_supported(a)) return launch_chunk_pair(a, stream);
+    if (chunk_pool_supported(a)) return launch_chunk_pool(a, stream);
     CUtensorMap mq, mk, mv;
     const int BH = a.B * a.H;
     if (!make_map(&mq, a.q, a.dk, a.T, BH) || !make_map(&mk, a.k, a.dk, a.T, BH) ||

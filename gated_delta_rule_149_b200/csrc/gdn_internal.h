@@ -31,11 +31,11 @@ cudaError_t launch_recurrent(const FwdArgs &a, cudaStream_t stream);
 bool chunk_tc_supported(const FwdArgs &a);
 cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream);
 
-// Chunkwise kernel split across a 2-CTA cluster per scan (preparation and
-// state chain on separate SMs): bf16, dk = dv = 128, whole sequences (no
-// segments).  launch_chunk_tc hands such calls to it.
-bool chunk_pair_supported(const FwdArgs &a);
-cudaError_t launch_chunk_pair(const FwdArgs &a, cudaStream_t stream);
+// Chunkwise kernel with one CTA per SM: a state chain per scan beside a pool of
+// preparation workers that serve every scan (bf16, dk = dv = 128, whole
+// sequences, no segments).  launch_chunk_tc hands such calls to it.
+bool chunk_pool_supported(const FwdArgs &a);
+cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream);
 
 // Allocation-free variant of launch_chunk_tc: the bidirectional arrival
 // counters come from a fixed static device array of noalloc_capacity() ints.

@@ -373,14 +373,14 @@ def gdn_workspace_reserved(device=None):
 
 
 def debug_kernel_select(which):
-    """Test hook: 0 picks the bf16 chunkwise kernel by shape, 1 forces the
-    single-CTA chunkwise kernel for every bf16 call, 2 asks for the paired-SM
-    kernel wherever it applies (dk = dv = 128, whole sequences)."""
+    """Test hook: 0 (or 2) picks the bf16 chunkwise kernel by shape (the pooled
+    kernel for dk = dv = 128 whole-sequence calls), 1 forces the single-CTA
+    chunkwise kernel for every bf16 call (for A/B comparisons of the two)."""
     load_library().gdn_debug_kernel_select(int(which))
 
 
 def debug_ring(buf):
-    """Test hook: a CUDA uint8 tensor of at least dirs*B*H*4*49664 bytes that the
-    paired-SM kernel uses as its operand ring (None: workspace), so that the
-    prepared operands of the last four chunks of every scan can be read back."""
+    """Test hook: a CUDA uint8 tensor of at least dirs*B*H*8*49664 bytes that the
+    pooled kernel uses as its operand ring (None: workspace), so that the
+    prepared operands of the last eight chunks of every scan can be read back."""
     load_library().gdn_debug_ring(None if buf is None else ctypes.c_void_p(buf.data_ptr()))

@@ -16,15 +16,16 @@ from parity_util import TOL, assert_finite_bounded, f64, oracle_forward, rel_l2,
 
 pytestmark = pytest.mark.gpu
 
-# which kernels serve bf16 inputs: the paired-SM chunkwise kernel (dk = dv = 128;
-# the single-CTA one for other shapes), the single-CTA chunkwise kernel, and the
-# token-by-token cross-check kernel
-BF16_KERNELS = ["pair", "single", "recurrent"]
+# which kernels serve bf16 inputs: the default choice by shape (the pooled
+# chunkwise kernel for dk = dv = 128, the single-CTA one otherwise), the
+# single-CTA chunkwise kernel for every shape, and the token-by-token
+# cross-check kernel
+BF16_KERNELS = ["pool", "single", "recurrent"]
 
 
 @contextlib.contextmanager
 def use_kernel(kernel):
-    gdn.debug_kernel_select({"pair": 2, "single": 1}.get(kernel, 0))
+    gdn.debug_kernel_select(1 if kernel == "single" else 0)
     try:
         yield kernel == "recurrent"
     finally:
@@ -109,11 +110,12 @@ def test_bf16_fast_decay(oracle_mod, kernel):
     check(oracle_mod, inp, True, kernel)
 
 
-@pytest.mark.parametrize("kernel,dv", [("single", 64), ("single", 128), ("pair", 128)])
+@pytest.mark.parametrize("kernel,dv", [("single", 64), ("single", 128), ("pool", 128)])
 def test_bf16_bidi_more_ctas_than_sms(oracle_mod, kernel, dv):
-    """More scans than fit on the GPU at once (single-CTA kernel: 160 CTAs on 148
-    SMs; paired kernel: 160 clusters of two where 74 fit): the order in which the
-    two scans reach an output tile is decided at run time instead of in advance."""
+    """More scans than fit on the GPU at once.  Single-CTA kernel: 160 CTAs on 148
+    SMs, so the order in which the two scans reach an output tile is decided at
+    run time instead of in advance.  Pooled kernel: 80 heads (160 chains) run as
+    successive launches of as many heads as fit beside the preparation workers."""
     heads = 160 // (2 * (dv // 64)) if kernel == "single" else 80
     inp = make_custom(1, heads, 333, 128, dv, dtype="bf16", seed=11 + dv, bidi=True)
     check(oracle_mod, inp, True, kernel)
