@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/gdn.h"
+#include "../../include/gdn_debug.h"
 #include "gdn_internal.h"
 
 namespace {
@@ -96,10 +97,11 @@ int dispatch(const gdn::FwdArgs &a, int mode, cudaStream_t stream)
 size_t dtype_size(int mode) { return (mode & GDN_FP32) ? 4 : 2; }
 
 // The kernels of host-buffer calls on one device run one after another
-// whatever their streams: a bidirectional launch whose CTAs all fit on the GPU
-// counts on being resident at once, which two such launches side by side would
-// not be.  Each call's kernels wait for the previous call's (an event per
-// device) and record their own completion.
+// whatever their streams: a chunkwise launch takes every SM (the pooled
+// kernel's grid is one CTA per SM, launched cooperatively), so two side by side
+// would only queue behind each other; in call order, each call's copies overlap
+// the previous call's kernel.  Each call's kernels wait for the previous call's
+// (an event per device) and record their own completion.
 constexpr int kMaxOrderDev = 64;
 std::mutex g_order_mu;
 cudaEvent_t g_order_ev[kMaxOrderDev] = {};
@@ -433,6 +435,15 @@ int gdn_device_status(void *stream)
     cudaError_t e = gdn::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &err);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device status: %s", cudaGetErrorString(e));
     if (err) return fail(GDN_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (code %d)", err);
+    return ok();
+}
+
+int gdn_debug_wait_limit(unsigned long long ns)
+{
+    const unsigned long long v = ns ? ns : 4000000000ull;
+    cudaError_t e = gdn::set_wait_limit_pool(v);
+    if (e == cudaSuccess) e = gdn::set_wait_limit_tc(v);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "wait limit: %s", cudaGetErrorString(e));
     return ok();
 }
 

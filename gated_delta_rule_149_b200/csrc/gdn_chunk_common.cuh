@@ -28,6 +28,16 @@ enum GateIdx { gG = 0, gGam, gBet, gBG, gEb, gRA, gRB, gCA, gCB };
 
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s per wait
 
+// The limit the bounded waits below apply (one copy per module that includes
+// this header; kWaitLimitNs unless a test lowers it to make a wait run out).
+static __device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
+// Sets this module's wait limit on the current device (synchronous).
+static inline cudaError_t set_module_wait_limit(unsigned long long ns)
+{
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
+
 __device__ __forceinline__ unsigned long long globaltimer()
 {
     unsigned long long t;
@@ -45,7 +55,7 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, volat
     for (uint32_t it = 0; it < (1u << 30); ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if ((it & 255) == 255 && globaltimer() - t0 > kWaitLimitNs) break;
+        if ((it & 255) == 255 && globaltimer() - t0 > g_wait_limit_ns) break;
     }
     atomicOr(err, code);
     *abort_flag = 1;
@@ -82,7 +92,7 @@ __device__ __noinline__ bool wait_smem_slow(const int *addr, int target, volatil
     for (uint32_t it = 0; it < (1u << 30); ++it) {
         if (ld_acquire_cta(addr) >= target) return true;
         if (*abort_flag) return false;
-        if ((it & 255) == 255 && globaltimer() - t0 > kWaitLimitNs) break;
+        if ((it & 255) == 255 && globaltimer() - t0 > g_wait_limit_ns) break;
     }
     atomicOr(err, code);
     *abort_flag = 1;
@@ -107,7 +117,7 @@ __device__ __noinline__ bool spin_global_at_least(const int *cnt, int target, vo
         if (seen >= target) return true;
         if (*abort_flag) return false;
         if ((it & 63) == 63) {
-            if (globaltimer() - t0 > kWaitLimitNs) return false;
+            if (globaltimer() - t0 > g_wait_limit_ns) return false;
             __nanosleep(64);
         }
     }

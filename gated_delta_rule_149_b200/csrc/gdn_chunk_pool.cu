@@ -49,12 +49,14 @@
 #include <cuda_runtime.h>
 
 #include <cstddef>
+#include <climits>
 #include <cstdint>
 #include <mutex>
 
 #include "gdn_internal.h"
 #include "sm100_ptx.cuh"
 #include "gdn_chunk_common.cuh"
+#include "../../include/gdn_debug.h"
 
 namespace gdn {
 
@@ -62,6 +64,8 @@ extern float *g_debug_dump;
 extern long long *g_prof_buf;
 void *g_debug_ring = nullptr;
 int g_kernel_select = 0;
+int g_stall_chunk = -1;
+bool g_plain_launch = false;
 
 namespace {
 
@@ -143,6 +147,7 @@ struct PoolParams {
     int bh0;             // index of its first head in the tensors
     int BH_all;          // heads in the tensors (the reverse direction's state_out offset)
     int T, n_chunks, n_scans, n_items;
+    int stall_chunk;     // testing: scan 0's chain waits for this chunk's slot without end (-1: never)
 };
 
 struct Bars {
@@ -289,11 +294,13 @@ __device__ __forceinline__ void worker_gates(const Ctx &x, const PoolParams &p, 
     const int lane = gpt & 31;
     for (int i = 0;; ++i) {
         const int s = i % kNS, gj = i % kNG;
-        if (!wait_bar(&B.it_full[s], (i / kNS) & 1, x.abort_flag, p.err, 2)) break;
-        if (i >= kNG && !wait_bar(&B.g_empty[gj], ((i / kNG) + 1) & 1, x.abort_flag, p.err, 3)) break;
+        bool ok = wait_bar(&B.it_full[s], (i / kNS) & 1, x.abort_flag, p.err, 2);
+        if (ok && i >= kNG) ok = wait_bar(&B.g_empty[gj], ((i / kNG) + 1) & 1, x.abort_flag, p.err, 3);
+        // both gate warps leave together: a thread whose wait gave up never
+        // leaves the other waiting at the group's barrier
+        if (named_bar_any(kBarGate, 64, !ok || *x.abort_flag)) break;
         const int k = B.sitem[s];
         if (k < 0) {   // past the last item: pass the end on
-            named_bar(kBarGate, 64);
             if (gpt == 0) {
                 B.gitem[gj] = -1;
                 mbar_arrive(&B.g_full[gj]);
@@ -685,7 +692,8 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
         vk_issued = i + 1;
         if (i >= 2 && !wait_bar(&B.a_empty[ab], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 22)) break;
         tr(p, 1, 0, i);
-        if (!wait_global(seq + s, i + 1, x, p, 65)) break;
+        const int want = (x.scan == 0 && i == p.stall_chunk) ? INT_MAX : i + 1;
+        if (!wait_global(seq + s, want, x, p, 65)) break;
         tr(p, 1, 1, i);
         fence_proxy_async_global();
         const uint8_t *slot = x.ring + (size_t)s * kSlotBytes;
@@ -1180,6 +1188,7 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream)
         p.consumed = flags + (size_t)p.n_scans * kNSlot;
         p.work = p.consumed + p.n_scans;
         p.counters = a.bidi ? p.work + 1 : nullptr;
+        p.stall_chunk = h0 == 0 ? g_stall_chunk : -1;
         err = device_error_word(&p.err);
         if (err != cudaSuccess) break;
         err = cudaMemsetAsync(flags, 0, flag_ints * sizeof(int), stream);
@@ -1195,7 +1204,7 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream)
         at[0].id = cudaLaunchAttributeCooperative;
         at[0].val.cooperative = 1;
         cfg.attrs = at;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = g_plain_launch ? 0 : 1;
         err = cudaLaunchKernelEx(&cfg, gdn_chunk_pool_kernel, mq, mk, mv, mo, p);
         if (err == cudaSuccess) err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
@@ -1207,12 +1216,23 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream)
 
 }  // namespace gdn
 
-// Test hooks (not part of the documented ABI).
+// Test hooks (declared in gdn_debug.h).
 // gdn_debug_ring: a device buffer of at least dirs*B*H*8*49664 bytes that the
 // pooled kernel uses as its operand ring instead of workspace (NULL: off), so a
 // test can read back the prepared operands of each scan's last eight chunks.
 // gdn_debug_kernel_select: 0 or 2 pick the kernel by shape (the pooled kernel
 // for dk = dv = 128 whole sequences), 1 forces the single-CTA chunkwise kernel
 // for every bf16 call.
+// gdn_debug_stall: chunk c >= 0 makes scan 0's chain of the pooled kernel wait
+// for chunk c's operands with a target nothing reaches, so the wait runs out
+// (with a lowered limit, see gdn_debug_wait_limit) and the call ends with
+// GDN_ERR_DEVICE_TIMEOUT; -1 (the default) turns it off.
+// gdn_debug_plain_launch: 1 launches the pooled kernel without the cooperative
+// attribute (same grid, one CTA per SM), for profilers that replay launches
+// one at a time; 0 (the default) restores the cooperative launch.
 extern "C" void gdn_debug_ring(void *device_buffer) { gdn::g_debug_ring = device_buffer; }
 extern "C" void gdn_debug_kernel_select(int which) { gdn::g_kernel_select = which; }
+extern "C" void gdn_debug_stall(int chunk) { gdn::g_stall_chunk = chunk; }
+extern "C" void gdn_debug_plain_launch(int on) { gdn::g_plain_launch = on != 0; }
+
+cudaError_t gdn::set_wait_limit_pool(unsigned long long ns) { return set_module_wait_limit(ns); }

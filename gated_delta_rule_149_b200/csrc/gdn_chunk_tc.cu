@@ -57,6 +57,7 @@
 #include "gdn_internal.h"
 #include "sm100_ptx.cuh"
 #include "gdn_chunk_common.cuh"
+#include "../../include/gdn_debug.h"
 
 namespace gdn {
 
@@ -1033,15 +1034,37 @@ cudaError_t set_smem_attribute()
     return err;
 }
 
-// Whether every CTA of the grid is resident at once (one CTA per SM, as the
-// shared-memory footprint forces), so that each bidirectional output tile's
-// first writer can be fixed in advance.
+// Whether every CTA of the grid fits on the GPU at once (one CTA per SM, as
+// the shared-memory footprint forces), so that each bidirectional output
+// tile's first writer can be fixed in advance; such grids are launched
+// cooperatively, which makes every CTA resident together.
 cudaError_t all_resident(int n_ctas, int *out)
 {
     int dev = 0, sms = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     *out = (err == cudaSuccess && n_ctas <= sms) ? 1 : 0;
+    return err;
+}
+
+// Launches the kernel; cooperatively when its CTAs count on one another being
+// resident (a bidirectional grid with the writer order fixed in advance).
+cudaError_t launch_tc_kernel(dim3 grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                             const TcParams &p, bool cooperative, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemAlloc;
+    cfg.stream = stream;
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = cooperative ? 1 : 0;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, gdn_chunk_tc_kernel, mq, mk, mv, p);
+    if (err == cudaSuccess) err = cudaGetLastError();
+    if (err == cudaSuccess) count_launches(1);
     return err;
 }
 
@@ -1093,12 +1116,9 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
         if (err != cudaSuccess) return err;
         err = cudaMemsetAsync(p.counters, 0, n_cnt * sizeof(int), stream);
     }
-    if (err == cudaSuccess) {
-        dim3 grid(p.n_slices, a.bidi ? 2 : 1, BH * a.n_seg);
-        gdn_chunk_tc_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, p);
-        err = cudaGetLastError();
-        if (err == cudaSuccess) count_launches(1);
-    }
+    if (err == cudaSuccess)
+        err = launch_tc_kernel(dim3(p.n_slices, a.bidi ? 2 : 1, BH * a.n_seg), mq, mk, mv, p,
+                               a.bidi && p.predict, stream);
     if (p.counters) {
         cudaError_t e2 = ws_free(p.counters, stream);
         if (err == cudaSuccess) err = e2;
@@ -1120,12 +1140,6 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream)
 
 constexpr size_t kNoAllocCounters = (size_t)1 << 18;   // 262,144 counters = 1 MiB
 static __device__ __align__(256) int g_noalloc_counters[kNoAllocCounters];
-
-namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-int *g_noalloc_ptr[kMaxDevices] = {};
-}  // namespace
 
 size_t noalloc_capacity() { return kNoAllocCounters; }
 
@@ -1159,36 +1173,22 @@ cudaError_t launch_chunk_tc_noalloc(const FwdArgs &a, cudaStream_t stream)
     if (a.bidi) {
         const size_t n_cnt = (size_t)BH * p.n_chunks * p.n_slices;
         if (n_cnt > kNoAllocCounters) return cudaErrorInvalidValue;   // checked by the caller too
-        int dev = 0;
-        err = cudaGetDevice(&dev);
+        // Host code cannot use the array's name as a device address: look the
+        // address up on every call (cheap), with the caller's device current.
+        void *ptr = nullptr;
+        err = cudaGetSymbolAddress(&ptr, g_noalloc_counters);
         if (err != cudaSuccess) return err;
-        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-        {
-            // Host code cannot use the array's name as a device address: look the
-            // address up once per device, with that device current.
-            std::lock_guard<std::mutex> lock(g_noalloc_mu);
-            if (!g_noalloc_ptr[dev]) {
-                void *ptr = nullptr;
-                err = cudaGetSymbolAddress(&ptr, g_noalloc_counters);
-                if (err != cudaSuccess) return err;
-                g_noalloc_ptr[dev] = static_cast<int *>(ptr);
-            }
-            p.counters = g_noalloc_ptr[dev];
-        }
+        p.counters = static_cast<int *>(ptr);
         // the array keeps the previous call's contents: the counters must start at zero
         err = cudaMemsetAsync(p.counters, 0, n_cnt * sizeof(int), stream);
         if (err != cudaSuccess) return err;
     }
-    dim3 grid(p.n_slices, a.bidi ? 2 : 1, BH);
-    gdn_chunk_tc_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, p);
-    err = cudaGetLastError();
-    if (err == cudaSuccess) count_launches(1);
-    return err;
+    return launch_tc_kernel(dim3(p.n_slices, a.bidi ? 2 : 1, BH), mq, mk, mv, p, a.bidi && p.predict, stream);
 }
 
 }  // namespace gdn
 
-// Test hook (not part of the documented ABI): when set to a device buffer of
+// Test hook (declared in gdn_debug.h): when set to a device buffer of
 // 53248 floats, the next chunkwise launches dump the first chunk's
 // intermediates of CTA (0,0,0) there.  NULL turns it off.
 extern "C" void gdn_debug_dump(float *device_buffer) { gdn::g_debug_dump = device_buffer; }
@@ -1196,3 +1196,5 @@ extern "C" void gdn_debug_dump(float *device_buffer) { gdn::g_debug_dump = devic
 // Test hook for profiling builds: per-phase cycle counters of CTA (0,0,0),
 // 32 long longs (zeroed by the caller).  Ignored unless built with GDN_PROFILE.
 extern "C" void gdn_debug_profile(long long *device_buffer) { gdn::g_prof_buf = device_buffer; }
+
+cudaError_t gdn::set_wait_limit_tc(unsigned long long ns) { return set_module_wait_limit(ns); }

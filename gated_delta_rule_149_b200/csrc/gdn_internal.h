@@ -76,6 +76,11 @@ cudaError_t ws_reserved(int dev, uint64_t *bytes);
 // Device-side error word (set by bounded waits that gave up).
 cudaError_t device_error_word(int **ptr);
 
+// The limit of the bounded waits in the chunkwise kernels (each module holds
+// its own copy), on the current device.
+cudaError_t set_wait_limit_pool(unsigned long long ns);
+cudaError_t set_wait_limit_tc(unsigned long long ns);
+
 // Launch accounting (gdn_kernel_launches).
 void count_launches(int n);
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *err);

@@ -77,6 +77,12 @@ def load_library():
         lib.gdn_debug_kernel_select.restype = None
         lib.gdn_debug_ring.argtypes = [vp]
         lib.gdn_debug_ring.restype = None
+        lib.gdn_debug_stall.argtypes = [i]
+        lib.gdn_debug_stall.restype = None
+        lib.gdn_debug_plain_launch.argtypes = [i]
+        lib.gdn_debug_plain_launch.restype = None
+        lib.gdn_debug_wait_limit.argtypes = [ctypes.c_ulonglong]
+        lib.gdn_debug_wait_limit.restype = i
         _lib = lib
     return _lib
 
@@ -384,3 +390,22 @@ def debug_ring(buf):
     pooled kernel uses as its operand ring (None: workspace), so that the
     prepared operands of the last eight chunks of every scan can be read back."""
     load_library().gdn_debug_ring(None if buf is None else ctypes.c_void_p(buf.data_ptr()))
+
+
+def debug_stall(chunk):
+    """Test hook: chunk >= 0 makes scan 0's state chain of the pooled kernel wait
+    for that chunk's operands with a target nothing reaches, so the wait runs
+    out and the call ends with a device timeout status; -1 turns it off."""
+    load_library().gdn_debug_stall(int(chunk))
+
+
+def debug_plain_launch(on):
+    """Test hook: launch the pooled kernel without the cooperative attribute (for
+    profilers that replay one launch at a time); False restores the default."""
+    load_library().gdn_debug_plain_launch(1 if on else 0)
+
+
+def debug_wait_limit(ns):
+    """Test hook: the limit in nanoseconds of every bounded device wait of the
+    chunkwise kernels on the current device; 0 restores the default (4 s)."""
+    _check(load_library().gdn_debug_wait_limit(int(ns)))

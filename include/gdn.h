@@ -79,14 +79,13 @@ enum gdn_status {
  *   fp32, or any dtype with GDN_RECURRENT: dk, dv multiples of 32, <= 128.
  * T >= 1 of any value (a ragged last chunk is handled).  B*H <= 65535.
  *
- * Bidirectional bf16 calls whose CTAs (B*H*2*dv/64) fit on the GPU's SMs fix
- * the order in which the two directions write each output tile in advance and
- * wait for one another inside the kernel: they count on every CTA being
- * resident at once.  If other work on other streams keeps SMs busy meanwhile,
- * a wait can run out (4 s) and the call reports GDN_ERR_DEVICE_TIMEOUT through
- * gdn_device_status (no hang, no silent result); run such calls without
- * concurrent kernels.  Larger grids decide the order at run time and have no
- * such requirement.
+ * Kernels whose CTAs wait for one another (the pooled chunkwise kernel used
+ * for dk = dv = 128, and bidirectional single-CTA launches that fit on the
+ * GPU's SMs) are launched cooperatively: CUDA starts them only with every CTA
+ * resident, so work on other streams delays them but cannot starve them.
+ * Every such wait is bounded (4 s); one that runs out sets the device error
+ * word (GDN_ERR_DEVICE_TIMEOUT from gdn_device_status) and the kernel
+ * returns: no hang, no silent result.
  */
 int gdn_forward(const void *q, const void *k, const void *v,
                 const float *beta, const float *decay,
@@ -131,8 +130,9 @@ int gdn_forward_host(const void *q, const void *k, const void *v,
  * pinned host memory, calls on two streams overlap one call's copies with the
  * other's kernels: the streaming loop of a video pipeline, where chunk i+1 is
  * uploaded while chunk i runs and downloads.  The kernels of host-buffer
- * calls on one device run one after another whatever their streams (a
- * bidirectional launch counts on having the GPU's SMs to itself).  Errors of
+ * calls on one device run one after another whatever their streams (each
+ * takes every SM; in call order the copies of one overlap the kernel of the
+ * other).  Errors of
  * the enqueued copies and kernels surface at the caller's synchronise;
  * argument errors are returned as for gdn_forward.
  */
@@ -164,9 +164,10 @@ int gdn_forward_host_async(const void *q, const void *k, const void *v,
  * load the library's device code): make that first call before any stream
  * capture.  All calls share the one array; the library clears the counters a
  * call uses before its kernel runs, so back-to-back calls on one stream are
- * fine, but calls that overlap on the GPU (other streams, other threads) race
- * on it and give wrong results.  Never allocates, frees or calls an allocating
- * library routine.
+ * fine, but bidirectional calls that overlap on the GPU (other streams, other
+ * threads) race on it: they give wrong results, or a wait on a counter runs
+ * out and gdn_device_status reports GDN_ERR_DEVICE_TIMEOUT.  Never allocates,
+ * frees or calls an allocating library routine.
  */
 int gdn_forward_noalloc(const void *q, const void *k, const void *v,
                         const float *beta, const float *decay,

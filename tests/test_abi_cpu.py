@@ -3,6 +3,7 @@ header declares, and rejects bad arguments with the documented codes before
 launching anything.  No call here reaches a CUDA API (every case fails
 validation first), so these run without a GPU."""
 import ctypes
+import glob
 import os
 import re
 
@@ -18,14 +19,17 @@ def lib():
     return gdn.load_library()
 
 
-def declared_functions():
-    src = open(os.path.join(ROOT, "include", "gdn.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^[A-Za-z_][\w ]*[\s*]+(gdn_\w+)\s*\(", src, flags=re.M)))
+def declared_functions(header=None):
+    names = set()
+    for h in ([header] if header else sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))):
+        src = open(os.path.join(ROOT, "include", h) if header else h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names.update(re.findall(r"^[A-Za-z_][\w ]*[\s*]+(gdn_\w+)\s*\(", src, flags=re.M))
+    return sorted(names)
 
 
 def test_header_declares_the_abi():
-    names = declared_functions()
+    names = declared_functions("gdn.h")
     for n in ("gdn_forward", "gdn_rollout", "gdn_forward_host", "gdn_forward_host_async", "gdn_forward_noalloc",
               "gdn_forward_segmented", "gdn_forward_blockcausal", "gdn_forward_normalized",
               "gdn_forward_fp8",
@@ -35,9 +39,15 @@ def test_header_declares_the_abi():
         assert n in names
 
 
+def test_debug_header_declares_the_hooks():
+    names = declared_functions("gdn_debug.h")
+    assert names == sorted(["gdn_debug_kernel_select", "gdn_debug_ring", "gdn_debug_dump", "gdn_debug_profile",
+                            "gdn_debug_stall", "gdn_debug_plain_launch", "gdn_debug_wait_limit"])
+
+
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
-        assert hasattr(lib, name), f"{name} declared in include/gdn.h but not exported"
+        assert hasattr(lib, name), f"{name} declared in a header under include/ but not exported"
 
 
 def test_version(lib):
