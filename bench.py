@@ -443,6 +443,7 @@ def run_gpu(args, world, rank, local):
     rollout = wl.n_chunks > 1
     dev = torch.device("cuda", torch.cuda.current_device())
     gdn.debug_kernel_select(1 if args.kernel == "single" else 0)
+    gdn.debug_plain_launch(args.plain_launch)
     inp = make_inputs(wl)
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
     beta, decay = inp.beta.to(dev), inp.decay.to(dev)
@@ -614,6 +615,8 @@ def run_gpu(args, world, rank, local):
             "gpu_launches": int(launches),
             "roofline": roofline,
             "clocks": clk.summary()}
+    if args.plain_launch:
+        line["kernel"] += " (plain launch, for profiling)"
     if rank == 0:
         try:
             line["parity"] = sampled_parity(args, wl, inp, o, s_out,
@@ -648,6 +651,9 @@ def main():
     ap.add_argument("--kernel", default="auto", choices=["auto", "single"],
                     help="bf16 chunkwise kernel: by shape (default: the pooled kernel for dk = dv = 128), "
                          "or the single-CTA one for every shape")
+    ap.add_argument("--plain-launch", action="store_true",
+                    help="launch the pooled kernel without the cooperative attribute (same grid), "
+                         "for profilers that replay one launch at a time")
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="seconds of CPU work per oracle sample (default 15; 8 for --impl reference)")
     args = ap.parse_args()
