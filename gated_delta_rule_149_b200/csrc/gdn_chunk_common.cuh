@@ -362,12 +362,16 @@ __device__ __forceinline__ void mma_run(uint32_t d, uint64_t a, uint64_t b, uint
         mma_bf16(d, a + (uint64_t)(k * A_STEP), b + (uint64_t)(k * B_STEP), idesc, (k > 0 || acc) ? 1u : 0u);
 }
 
-// solve_off_diag with the walk down the block rows kept as a loop (about a third
-// of the code): for kernels whose per-chunk code is larger than the
-// instruction cache, where each instruction fetched costs more than the work
-// it does.  Same arithmetic, same results.
-__device__ __forceinline__ void solve_off_diag_compact(const float *As, const float *gt, uint8_t *sT1,
-                                                       uint8_t *sT2, int dir, int pt)
+// The off-diagonal blocks of T for 8 warps: warp pw walks the strip of block
+// column jb = pw / 2, columns [16 jb + 8 (pw % 2), +8), down the block rows
+// below it; the two warps of block column 3 (no block below it) write the
+// diagonal blocks' T1, T2 instead.  One block row per loop step (compact code:
+// the prep shares its SM's instruction caches with the other roles): every A
+// fragment of the row is loaded before its products start, and the block
+// products go to independent accumulators, so that a step waits on one round
+// of shared loads and on the tensor products of its own chain.
+__device__ __forceinline__ void solve_off_diag_strips(const float *As, const float *gt, uint8_t *sT1,
+                                                      uint8_t *sT2, int dir, int pt)
 {
     const int pw = pt >> 5, lane = pt & 31, g = lane >> 2, q = lane & 3, hs = pw & 1, jb = pw >> 1;
     if (jb == 3) {   // no strip below block column 3: write the diagonal blocks' T1, T2
@@ -375,12 +379,16 @@ __device__ __forceinline__ void solve_off_diag_compact(const float *As, const fl
         return;
     }
     const int c0 = 16 * jb + 8 * hs;
-    uint32_t tb0[2][2], tb1[2][2], tb2[2][2];   // B fragments of the strip's blocks in block rows jb, jb+1, jb+2
+    uint32_t tb[3][2][2];   // B fragments of the strip's blocks in block rows jb, jb+1, jb+2
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
-        tb0[ks][0] = to_tf32(As[(16 * jb + 8 * ks + q) * kLDA + c0 + g]);
-        tb0[ks][1] = to_tf32(As[(16 * jb + 8 * ks + q + 4) * kLDA + c0 + g]);
+        tb[0][ks][0] = to_tf32(As[(16 * jb + 8 * ks + q) * kLDA + c0 + g]);
+        tb[0][ks][1] = to_tf32(As[(16 * jb + 8 * ks + q + 4) * kLDA + c0 + g]);
     }
+#pragma unroll
+    for (int kb = 1; kb < 3; ++kb)
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) tb[kb][ks][0] = tb[kb][ks][1] = 0u;
     const int lj = c0 + 2 * q;
     const int pc0 = dir ? 63 - lj : lj, pc1 = dir ? 62 - lj : lj + 1;
     const float sg0 = gt[gBG * 64 + pc0], sg1 = gt[gBG * 64 + pc1];
@@ -388,48 +396,52 @@ __device__ __forceinline__ void solve_off_diag_compact(const float *As, const fl
 #pragma unroll 1
     for (int io = 1; io <= 3 - jb; ++io) {
         const int ib = jb + io;   // block row
-        // S = sum_k A_{ib,k} T_{k,jb}, two accumulators to halve the chain
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t a[4];
-        if (hs == 0) {   // D_jb is zero above the strip's diagonal
-            ld_afrag(a, As, 16 * ib, 16 * jb, g, q);
-            mma_tf32(s0, a, tb0[0]);
-        }
-        ld_afrag(a, As, 16 * ib, 16 * jb + 8, g, q);
-        mma_tf32(s1, a, tb0[1]);
-        if (io > 1) {
-            ld_afrag(a, As, 16 * ib, 16 * (jb + 1), g, q);
-            mma_tf32(s0, a, tb1[0]);
-            ld_afrag(a, As, 16 * ib, 16 * (jb + 1) + 8, g, q);
-            mma_tf32(s1, a, tb1[1]);
-        }
-        if (io > 2) {
-            ld_afrag(a, As, 16 * ib, 16 * (jb + 2), g, q);
-            mma_tf32(s0, a, tb2[0]);
-            ld_afrag(a, As, 16 * ib, 16 * (jb + 2) + 8, g, q);
-            mma_tf32(s1, a, tb2[1]);
-        }
+        // the row's fragments: A_{ib, jb + kb} for kb < io, and D_ib
+        uint32_t a[3][2][4], d[2][4];
+#pragma unroll
+        for (int kb = 0; kb < 3; ++kb)
+            if (kb < io) {
+                ld_afrag(a[kb][0], As, 16 * ib, 16 * (jb + kb), g, q);
+                ld_afrag(a[kb][1], As, 16 * ib, 16 * (jb + kb) + 8, g, q);
+            }
+        ld_afrag(d[0], As, 16 * ib, 16 * ib, g, q);
+        ld_afrag(d[1], As, 16 * ib, 16 * ib + 8, g, q);
+        // S = sum_k A_{ib,k} T_{k,jb}, one accumulator per product
+        float sp[3][2][4];
+#pragma unroll
+        for (int kb = 0; kb < 3; ++kb)
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) sp[kb][ks][u] = 0.f;
+        if (hs == 0) mma_tf32(sp[0][0], a[0][0], tb[0][0]);   // D_jb is zero above the strip's diagonal
+        mma_tf32(sp[0][1], a[0][1], tb[0][1]);
+#pragma unroll
+        for (int kb = 1; kb < 3; ++kb)
+            if (kb < io) {
+                mma_tf32(sp[kb][0], a[kb][0], tb[kb][0]);
+                mma_tf32(sp[kb][1], a[kb][1], tb[kb][1]);
+            }
         float sv[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) sv[u] = s0[u] + s1[u];
+        for (int u = 0; u < 4; ++u)
+            sv[u] = (sp[0][0][u] + sp[0][1][u]) + (sp[1][0][u] + sp[1][1][u]) + (sp[2][0][u] + sp[2][1][u]);
         uint32_t sbf[2][2];
         c_to_b(sv, sbf, g, q);
         // T_{ib,jb} = -D_ib S
-        float t[4] = {0.f, 0.f, 0.f, 0.f};
+        float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_tf32(t0, d[0], sbf[0]);
+        mma_tf32(t1, d[1], sbf[1]);
+        float t[4];
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            ld_afrag(a, As, 16 * ib, 16 * ib + 8 * ks, g, q);
-            mma_tf32(t, a, sbf[ks]);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) t[u] = -t[u];
+        for (int u = 0; u < 4; ++u) t[u] = -(t0[u] + t1[u]);
         const int lr = 16 * ib + g;
         st_tpair(sT1, dir, lr, lj, t[0] * sg0, t[1] * sg1);
         st_tpair(sT1, dir, lr + 8, lj, t[2] * sg0, t[3] * sg1);
         st_tpair(sT2, dir, lr, lj, t[0] * sb0, t[1] * sb1);
         st_tpair(sT2, dir, lr + 8, lj, t[2] * sb0, t[3] * sb1);
-        if (io == 1) c_to_b(t, tb1, g, q);
-        else if (io == 2) c_to_b(t, tb2, g, q);
+        if (io == 1) c_to_b(t, tb[1], g, q);
+        else if (io == 2) c_to_b(t, tb[2], g, q);
     }
 }
 

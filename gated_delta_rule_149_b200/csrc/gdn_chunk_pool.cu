@@ -368,37 +368,44 @@ __device__ __forceinline__ void worker_gates(const Ctx &x, const PoolParams &p, 
 // D1 buffer is free once item j's masks are read, which P [T1 | T2] follows),
 // then [P T1; T1] K of item j (after the finisher has read P [T1 | T2]).  The
 // [Q;K] K^T products run two items ahead of the solver.
+// [Q;K] K^T of item i (one thread; out of line, as it is issued from several
+// places): 1 issued, 0 no such item (the end), -1 inputs not ready yet (only
+// when !block), -2 abort.
+__device__ __noinline__ int issue_qk(Bars *Bp, volatile int *abort_flag, int *err, uint32_t sbase, uint32_t tm,
+                                     int i, bool block)
+{
+    Bars &B = *Bp;
+    const int s = i % kNS, b1 = i & 1;
+    if (!block && !(mbar_test_wait(&B.st_full[s], (i / kNS) & 1) &&
+                    (i < 2 || mbar_test_wait(&B.d1_empty[b1], ((i >> 1) + 1) & 1))))
+        return -1;
+    if (!wait_bar(&B.st_full[s], (i / kNS) & 1, abort_flag, err, 4)) return -2;
+    if (B.sitem[s] < 0) return 0;
+    if (i >= 2 && !wait_bar(&B.d1_empty[b1], ((i >> 1) + 1) & 1, abort_flag, err, 5)) return -2;
+    const uint32_t sQK = sbase + kWStage + s * kWStageBytes;
+    const uint64_t a = sw128_desc(sQK, 16, 1024), b = sw128_desc(sQK + 8192, 16, 1024);
+    tc_fence_after();
+    mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a, b, kIdM1, false);
+    mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a + 1024, b + 1024, kIdM1, true);
+    mma_commit(&B.d1_full[b1]);
+    return 1;
+}
+
 __device__ __forceinline__ void worker_mma(const Ctx &x, const PoolParams &p)
 {
     Bars &B = *x.bars;
     const uint32_t tm = x.tmem;
-    // [Q;K] K^T of item i: 1 issued, 0 no such item (the end), -1 inputs not ready
-    // yet (only when !block), -2 abort
-    auto issue_m1 = [&](int i, bool block) -> int {
-        const int s = i % kNS, b1 = i & 1;
-        if (!block && !(mbar_test_wait(&B.st_full[s], (i / kNS) & 1) &&
-                        (i < 2 || mbar_test_wait(&B.d1_empty[b1], ((i >> 1) + 1) & 1))))
-            return -1;
-        if (!wait_bar(&B.st_full[s], (i / kNS) & 1, x.abort_flag, p.err, 4)) return -2;
-        if (B.sitem[s] < 0) return 0;
-        if (i >= 2 && !wait_bar(&B.d1_empty[b1], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 5)) return -2;
-        const uint32_t sQK = x.sbase + kWStage + s * kWStageBytes;
-        const uint64_t a = sw128_desc(sQK, 16, 1024), b = sw128_desc(sQK + 8192, 16, 1024);
-        tc_fence_after();
-        mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a, b, kIdM1, false);
-        mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a + 1024, b + 1024, kIdM1, true);
-        mma_commit(&B.d1_full[b1]);
-        tr(p, 0, 16, i);
-        return 1;
-    };
     int last = -1;   // the number of items, once the end has been seen
     int next = 0;    // next item whose [Q;K] K^T is to be issued
     auto step_m1 = [&](bool block) -> bool {   // false on abort
         if (last >= 0) return true;
-        const int r = issue_m1(next, block);
+        const int r = issue_qk(x.bars, x.abort_flag, p.err, x.sbase, tm, next, block);
         if (r == -2) return false;
         if (r == 0) last = next;
-        if (r == 1) ++next;
+        if (r == 1) {
+            tr(p, 0, 16, next);
+            ++next;
+        }
         return true;
     };
     bool ok = step_m1(true) && step_m1(true);
@@ -431,11 +438,11 @@ __device__ __forceinline__ void worker_mma(const Ctx &x, const PoolParams &p)
 }
 
 // Mask epilogue of this warp's 32 physical columns [32 hf, +32) of one row of
-// [Q;K] K^T, in four groups of 8.  Rows 0-63 (TMEM quarters 0-1) give P row r:
-// j kept at or before r in scan order; rows 64-127 give A row r, written in
-// scan order: j strictly before r, times b_r.  The decay ratio 2^(G_r - G_j) is
-// a product of a row and a column factor when the chunk's factors are all
-// normal floats (`fact`), else one exp2 of the difference.
+// [Q;K] K^T, read from TMEM in one load.  Rows 0-63 (TMEM quarters 0-1) give
+// P row r: j kept at or before r in scan order; rows 64-127 give A row r,
+// written in scan order: j strictly before r, times b_r.  The decay ratio
+// 2^(G_r - G_j) is a product of a row and a column factor when the chunk's
+// factors are all normal floats (`fact`), else one exp2 of the difference.
 __device__ __forceinline__ void mask_rows(uint32_t taddr, const float *gt, float *As, uint8_t *sP, int qd,
                                           int lane, int hf, bool fact, int dir)
 {
@@ -446,38 +453,34 @@ __device__ __forceinline__ void mask_rows(uint32_t taddr, const float *gt, float
     const float *cf = gt + (useB ? gCB : gCA) * 64 + 32 * hf;
     const float br = pm ? 1.f : gt[gBet * 64 + r];
     const float rf = br * gt[(useB ? gRB : gRA) * 64 + r];
-    const float Gr = gt[gG * 64 + r];
-#pragma unroll 1
-    for (int g8 = 0; g8 < 4; ++g8) {
-        float xv[8];
-        tmem_ld8(taddr + 8 * g8, xv);
-        tmem_wait_ld();
-        const int j0 = 32 * hf + 8 * g8;   // physical column of xv[0]
-        if (fact) {
+    const int j0 = 32 * hf;                              // physical column of xv[0]
+    float xv[32];
+    tmem_ld32(taddr, xv);
+    tmem_wait_ld();
+    // kept columns: u in [lo, hi)
+    const int rel = r - j0;
+    const int lo = dir ? (pm ? rel : rel + 1) : 0;
+    const int hi = dir ? 32 : (pm ? rel + 1 : rel);
+    if (fact) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) xv[u] *= rf * cf[8 * g8 + u];
-        } else {
+        for (int u = 0; u < 32; ++u) xv[u] = (u >= lo && u < hi) ? xv[u] * (rf * cf[u]) : 0.f;
+    } else {
+        const float Gr = gt[gG * 64 + r];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) xv[u] *= br * exp2f(Gr - gt[gG * 64 + j0 + u]);
-        }
-        // kept columns of the group: u in [lo, hi)
-        const int rel = r - j0;
-        const int lo = dir ? (pm ? rel : rel + 1) : 0;
-        const int hi = dir ? 8 : (pm ? rel + 1 : rel);
+        for (int u = 0; u < 32; ++u)
+            xv[u] = (u >= lo && u < hi) ? xv[u] * (br * exp2f(Gr - gt[gG * 64 + j0 + u])) : 0.f;
+    }
+    if (pm) {
+        store_half_row_bf16(sP, r, hf, xv);
+    } else if (dir) {   // scan-order columns 63 - j run backwards
+        float4 *dst = reinterpret_cast<float4 *>(As + lr * kLDA + 32 - j0);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) xv[u] = (u >= lo && u < hi) ? xv[u] : 0.f;
-        if (pm) {
-            st_tile_v4(sP, sw128_off(r, j0), pack_bf16(xv[0], xv[1]), pack_bf16(xv[2], xv[3]),
-                       pack_bf16(xv[4], xv[5]), pack_bf16(xv[6], xv[7]));
-        } else if (dir) {   // scan-order columns 63 - j run backwards
-            float4 *dst = reinterpret_cast<float4 *>(As + lr * kLDA + 56 - j0);
-            dst[0] = make_float4(xv[7], xv[6], xv[5], xv[4]);
-            dst[1] = make_float4(xv[3], xv[2], xv[1], xv[0]);
-        } else {
-            float4 *dst = reinterpret_cast<float4 *>(As + lr * kLDA + j0);
-            dst[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
-            dst[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
-        }
+        for (int m = 0; m < 8; ++m)
+            dst[m] = make_float4(xv[31 - 4 * m], xv[30 - 4 * m], xv[29 - 4 * m], xv[28 - 4 * m]);
+    } else {
+        float4 *dst = reinterpret_cast<float4 *>(As + lr * kLDA + j0);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) dst[m] = make_float4(xv[4 * m], xv[4 * m + 1], xv[4 * m + 2], xv[4 * m + 3]);
     }
 }
 
@@ -516,7 +519,7 @@ __device__ __forceinline__ void worker_solver(const Ctx &x, const PoolParams &p,
         if (pt == 0) tr(p, 0, 3, i);
         solve_diag_blocks<kBarA, kGroup>(As, gt, tb + 8192, tb + 24576, nullptr, dir, pt);
         if (pt == 0) tr(p, 0, 4, i);
-        solve_off_diag_compact(As, gt, tb + 8192, tb + 24576, dir, pt);
+        solve_off_diag_strips(As, gt, tb + 8192, tb + 24576, dir, pt);
         fence_proxy_async_smem();
         if (named_bar_any(kBarA, kGroup, *x.abort_flag)) return;
         if (pt == 0) mbar_arrive(&B.tp_full[b]);
