@@ -209,16 +209,6 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
 
-
-// o[0..8) += x (eight bf16 values packed in four words), added in L2
-__device__ __forceinline__ void red_add_bf16x8(__nv_bfloat16 *addr, uint32_t a, uint32_t b, uint32_t c,
-                                               uint32_t d)
-{
-    asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};" ::"l"(addr), "r"(a), "r"(b),
-                 "r"(c), "r"(d) : "memory");
-}
-
-
 __device__ __forceinline__ void dbg_half(float *dst, int row, int h, const float *x)
 {
 #pragma unroll
@@ -754,10 +744,21 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
                 for (int q = 0; q < 4; ++q)
                     *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
             } else if (add) {
-                // bf16 add in L2: the partials are rounded to bf16 on each side
+                // the first writer's stored partial plus this direction's fp32
+                // partial, rounded to bf16 once (read past L1: the partial was
+                // written by another SM)
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    red_add_bf16x8(orow + 8 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(orow + 8 * q));
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+                    uint32_t r4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 f = __bfloat1622float2(h2[u]);
+                        r4[u] = pack_bf16(f.x + xv[8 * q + 2 * u], f.y + xv[8 * q + 2 * u + 1]);
+                    }
+                    *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+                }
             }
         }
         tc_fence_before();

@@ -60,9 +60,12 @@ cudaError_t launch_fp8(const FwdArgs &a, const float *q_scale, const float *k_sc
     const struct { const void *in; const float *s; __nv_bfloat16 *out; size_t n, per; } job[3] = {
         {a.q, q_scale, q, nk, (size_t)a.T * a.dk}, {a.k, k_scale, k, nk, (size_t)a.T * a.dk},
         {a.v, v_scale, v, nv, (size_t)a.T * a.dv}};
+    int dev = 0, sms = 0;
+    if (err == cudaSuccess) err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     for (int j = 0; j < 3 && err == cudaSuccess; ++j) {
-        // HBM-bound: enough blocks in flight on every SM (148 SMs x 16)
-        dequant_e4m3_kernel<<<148 * 16, 256, 0, stream>>>(static_cast<const uint8_t *>(job[j].in), job[j].s,
+        // HBM-bound: enough blocks in flight on every SM (16 per SM)
+        dequant_e4m3_kernel<<<sms * 16, 256, 0, stream>>>(static_cast<const uint8_t *>(job[j].in), job[j].s,
                                                           job[j].out, job[j].n / 16, job[j].per);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
