@@ -48,12 +48,14 @@ METRIC = "GDN tokens*heads/s (bf16, 1xB200)"
 UNIT = "tokens*heads/s"
 
 
-def algorithmic_bytes(wl):
+def algorithmic_bytes(wl, fp8=False):
     """Bytes a perfect kernel moves once: q, k, v, gates read and o written once
-    per scan direction, plus the fp32 states (in if present, out always)."""
+    per scan direction, plus the fp32 states (in if present, out always).  fp8
+    inputs: q, k and v are one byte per element (o stays bf16)."""
     es = 2 if wl.dtype == "bf16" else 4
+    es_in = 1 if fp8 else es
     ndir = 2 if wl.bidi else 1
-    per_tok = ndir * ((2 * wl.dk + wl.dv) * es + 8) + wl.dv * es
+    per_tok = ndir * ((2 * wl.dk + wl.dv) * es_in + 8) + wl.dv * es
     st = wl.dk * wl.dv * 4
     n_heads = wl.B * wl.H
     states = n_heads * st * (ndir + (1 if wl.state0 else 0))
@@ -455,7 +457,9 @@ def run_gpu(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     lib = gdn.load_library()
 
-    segmented = args.segments > 0 or args.block > 0 or args.normalized or args.fp8
+    # fp8 with dv = 128 runs as the one pooled kernel (codes widened in-kernel)
+    fp8_prepass = args.fp8 and (wl.dv != 128 or args.kernel == "single")
+    segmented = args.segments > 0 or args.block > 0 or args.normalized or fp8_prepass
     if rollout and (segmented or recurrent):
         raise SystemExit("the rollout workload runs the plain bf16 chunkwise path only")
     if args.fp8:
@@ -493,7 +497,7 @@ def run_gpu(args, world, rank, local):
 
     # Workloads whose bytes per step do not dwarf the 126 MB L2 are timed with
     # L2 flushed before every step (a 512 MB write, outside the step's events).
-    bytes_ = algorithmic_bytes(wl)
+    bytes_ = algorithmic_bytes(wl, fp8=args.fp8)
     flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if bytes_ < (1 << 30) else None
     launches0 = lib.gdn_kernel_launches()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -536,7 +540,8 @@ def run_gpu(args, world, rank, local):
                           if recurrent else
                           "the whole rollout call: %d chunkwise launches, one per chunk" % wl.n_chunks
                           if rollout else
-                          "the chunkwise kernel (the call's one kernel)" if not segmented else
+                          "the chunkwise kernel (the call's one kernel)%s" % (
+                              ", E4M3 codes read at one byte per element" if args.fp8 else "") if not segmented else
                           "the whole call: the bf16 kernel's algorithmic bytes over the time of all "
                           "its launches (%s)" % ("dequantising pre-pass included" if args.fp8 else
                                                  "every pass and combine included")),
@@ -560,7 +565,7 @@ def run_gpu(args, world, rank, local):
 
     def e2e_step(n):
         ho, hso = hos[n % 2], hsos[n % 2]
-        if segmented or rollout:   # the same call on device copies of pinned host buffers
+        if segmented or rollout or args.fp8:   # the same call on device copies of pinned host buffers
             pairs = ((hq, q8), (hk, k8), (hv, v8), (hsq, sq), (hsk, sk), (hsv, sv)) if args.fp8 else \
                 ((hq, q), (hk, k), (hv, v))
             for h, dst in pairs + ((hb, beta), (ha, decay), (hs0, s0)):
@@ -600,7 +605,8 @@ def run_gpu(args, world, rank, local):
             "dtype": wl.dtype, "data": "synthetic",
             "config": workload_config(wl, world),
             "kernel": ("recurrent" if recurrent else
-                       "chunk_tc, fp8 E4M3 inputs (dequantising pre-pass)" if args.fp8 else
+                       "chunk_tc, fp8 E4M3 inputs (dequantising pre-pass)" if fp8_prepass else
+                       "chunkwise, pooled, fp8 E4M3 inputs widened to bf16 in shared memory" if args.fp8 else
                        "chunk_tc, normalised read-out (z state, second pass)" if args.normalized else
                        f"chunk_tc, frame-block read-out, blocks of {args.block}" if args.block > 0 else
                        f"chunk_tc, segment-parallel x{args.segments}" if segmented else
@@ -610,7 +616,7 @@ def run_gpu(args, world, rank, local):
                     "h2d_bytes_per_step": nbytes(hq, hk, hv, hb, ha, hs0,
                                                  *((hsq, hsk, hsv) if args.fp8 else ())),
                     "d2h_bytes_per_step": nbytes(hos[0], hsos[0]),
-                    "calls": ("synchronous, one stream" if segmented or rollout else
+                    "calls": ("synchronous, one stream" if segmented or rollout or args.fp8 else
                               "gdn_forward_host_async on two alternating streams (2 calls in flight)")},
             "gpu_launches": int(launches),
             "roofline": roofline,
@@ -641,7 +647,7 @@ def main():
                     help="time the token-by-token SIMT kernel instead of the chunkwise one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fp8", action="store_true",
-                    help="fp8 (E4M3) q, k, v with per-head scales (dequantising pre-pass)")
+                    help="fp8 (E4M3) q, k, v with per-head scales (widened in-kernel for dv = 128)")
     ap.add_argument("--normalized", action="store_true",
                     help="normalised read-out with a z state (eps 1e-6)")
     ap.add_argument("--block", type=int, default=0,

@@ -46,6 +46,8 @@
 // launch is cooperative: every CTA is resident, or the launch is refused.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -75,7 +77,7 @@ namespace {
 // fp32 values).
 constexpr int kThreads = 512;
 constexpr int kGroup = 256, kGroupB = 128;
-constexpr int kBarA = 1, kBarB = 2, kBarGate = 3;   // named barriers
+constexpr int kBarA = 1, kBarB = 2, kBarGate = 3, kBarConv = 4;   // named barriers
 constexpr int kNG = 3;                    // gate buffers
 constexpr int kNS = 3;                    // worker input stages
 constexpr uint32_t kGateFloats = 9 * 64;
@@ -104,11 +106,13 @@ constexpr uint32_t kCA = kCStage + kNVK * 32768;          // 2 ring-slot images
 constexpr uint32_t kCABytes = 50176;
 constexpr uint32_t kCO = kCA + 2 * kCABytes;              // 2 output tiles [dv block][64 tokens][64]
 constexpr uint32_t kCEnd = kCO + 2 * 16384;
-constexpr uint32_t kSmemBytes = (kPEnd > kCEnd ? kPEnd : kCEnd);
+constexpr uint32_t kC8 = kCEnd;                           // fp8 inputs: staging of one chunk's v, k codes
+constexpr uint32_t kCEnd8 = kC8 + 16384;
+constexpr uint32_t kSmemBytes = (kPEnd > kCEnd8 ? kPEnd : kCEnd8);
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(kPP % 1024 == 0 && kPTB % 1024 == 0 && kPA2 % 1024 == 0 && kCA % 1024 == 0 &&
-              kCABytes % 1024 == 0 && kCO % 1024 == 0 && kPGst % 16 == 0,
+              kCABytes % 1024 == 0 && kCO % 1024 == 0 && kC8 % 1024 == 0 && kPGst % 16 == 0,
               "tile alignment");
 
 // TMEM columns
@@ -148,6 +152,8 @@ struct PoolParams {
     int BH_all;          // heads in the tensors (the reverse direction's state_out offset)
     int T, n_chunks, n_scans, n_items;
     int stall_chunk;     // testing: scan 0's chain waits for this chunk's slot without end (-1: never)
+    // fp8 inputs (the FP8 kernel): q, k, v are E4M3 codes with one scale per head
+    const float *q_scale, *k_scale, *v_scale;
 };
 
 struct Bars {
@@ -155,9 +161,11 @@ struct Bars {
     uint64_t it_full[kNS], st_full[kNS], st_empty[kNS], d1_full[2], d1_empty[2], tp_full[2], p_free, t_free[2];
     uint64_t d2_full, d2_empty, e2_done, d3_full, d3_empty;
     uint64_t g_full[kNG], g_empty[kNG];
+    uint64_t cv_full[kNS];             // fp8: the stage's q, k tiles converted to bf16
     // chain
     uint64_t vk_full[kNVK], vk_empty[kNVK], a_full[2], a_empty[2], d_full[2], d_empty[2], o_full[2];
     uint64_t u_full, s_full, h_full;
+    uint64_t s8_full, s8_empty;        // fp8: the v, k code staging
     uint64_t drain;
     float gscal[kNG][2];   // per gate buffer: G_end, factorised (1) or not (0)
     int gitem[kNG];        // per gate buffer: the item, or -1 after the last
@@ -250,11 +258,59 @@ __device__ __forceinline__ bool wait_global(const int *word, int target, const C
     return false;
 }
 
+// ------------------------------------------------------------------ fp8 inputs
+// A chunk's q, k or v tile of E4M3 codes arrives by TMA as 64 token rows of
+// 128 bytes (128B-swizzled, 8 KB); the tensor-core products take bf16, so 64
+// threads widen it to scaled bf16 (x = scale * decode(code)) in the
+// 128B-swizzled layout of the bf16 path: codes [0, 64) of each row into tile
+// dst0, codes [64, 128) into dst1.
+
+// 16 codes (one 16-byte chunk) times `scale`, as 8 packed bf16 pairs (the
+// E4M3 to f16 widening is exact; one rounding, to bf16)
+__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &c, float scale, uint32_t (&w)[8])
+{
+    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const __half2_raw hr =
+                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(words[i] >> (16 * h)), __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+            w[2 * i + h] = pack_bf16(f.x * scale, f.y * scale);
+        }
+}
+
+// Thread t (of 64) takes the 16-code chunk t % 8 of rows t / 8 + 8 n.  Every
+// thread reads its chunks before the group's barrier and writes after it, so
+// a destination may overlap the source.
+__device__ __forceinline__ void e4m3_tile_to_bf16(const uint8_t *src, uint8_t *dst0, uint8_t *dst1, float scale,
+                                                  int t, int bar_id)
+{
+    const int j = t & 7, r0 = t >> 3, ph = r0 & 7;   // rows r0 + 8 n share the swizzle phase
+    uint4 c[8];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) c[n] = *reinterpret_cast<const uint4 *>(src + (r0 + 8 * n) * 128 + ((j ^ ph) << 4));
+    named_bar(bar_id, 64);
+    uint8_t *d = (j >> 2) ? dst1 : dst0;
+    const int m0 = 2 * (j & 3);   // the chunk's first 16-byte bf16 chunk in its 64-column tile
+    const uint32_t o0 = (uint32_t)((m0 ^ ph) << 4), o1 = (uint32_t)(((m0 + 1) ^ ph) << 4);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+        uint32_t w[8];
+        e4m3x16_to_bf16(c[n], scale, w);
+        uint8_t *row = d + (r0 + 8 * n) * 128;
+        *reinterpret_cast<uint4 *>(row + o0) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(row + o1) = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
+
 // ================================================================== workers
 
 // TMA: hands out the items (one per input stage: published on it_full before
 // its q, k tiles are loaded) and loads their q, k tiles; an item past the last
 // one marks the end.
+template <bool FP8>
 __device__ __forceinline__ void worker_tma(const Ctx &x, const CUtensorMap *tmQ, const CUtensorMap *tmK,
                                            const PoolParams &p)
 {
@@ -274,10 +330,16 @@ __device__ __forceinline__ void worker_tma(const Ctx &x, const CUtensorMap *tmQ,
         B.sitem[s] = k;
         mbar_arrive(&B.it_full[s]);
         uint8_t *st = x.smem + kWStage + s * kWStageBytes;
-        mbar_arrive_expect_tx(&B.st_full[s], 32768);
-        for (int kb = 0; kb < 2; ++kb) {
-            tma_load_3d(st + kb * 16384, tmQ, &B.st_full[s], kb * 64, it.c * kC, it.bh);
-            tma_load_3d(st + kb * 16384 + 8192, tmK, &B.st_full[s], kb * 64, it.c * kC, it.bh);
+        if (FP8) {   // the E4M3 q, k tiles into the stage's K spots, widened in place by the gate warps
+            mbar_arrive_expect_tx(&B.st_full[s], 16384);
+            tma_load_3d(st + 8192, tmQ, &B.st_full[s], 0, it.c * kC, it.bh);
+            tma_load_3d(st + 24576, tmK, &B.st_full[s], 0, it.c * kC, it.bh);
+        } else {
+            mbar_arrive_expect_tx(&B.st_full[s], 32768);
+            for (int kb = 0; kb < 2; ++kb) {
+                tma_load_3d(st + kb * 16384, tmQ, &B.st_full[s], kb * 64, it.c * kC, it.bh);
+                tma_load_3d(st + kb * 16384 + 8192, tmK, &B.st_full[s], kb * 64, it.c * kC, it.bh);
+            }
         }
         issued = i + 1;
     }
@@ -288,6 +350,7 @@ __device__ __forceinline__ void worker_tma(const Ctx &x, const CUtensorMap *tmQ,
 // Gate warps (64 threads): the gates of each item in log2 form, as soon as the
 // item is handed out: G (inclusive prefix sum of log2 a in scan order), gamma,
 // b, b gamma, e = 2^(G_end - G), and the row/column factors of the decay ratios.
+template <bool FP8>
 __device__ __forceinline__ void worker_gates(const Ctx &x, const PoolParams &p, int gpt)
 {
     Bars &B = *x.bars;
@@ -295,11 +358,31 @@ __device__ __forceinline__ void worker_gates(const Ctx &x, const PoolParams &p, 
     for (int i = 0;; ++i) {
         const int s = i % kNS, gj = i % kNG;
         bool ok = wait_bar(&B.it_full[s], (i / kNS) & 1, x.abort_flag, p.err, 2);
-        if (ok && i >= kNG) ok = wait_bar(&B.g_empty[gj], ((i / kNG) + 1) & 1, x.abort_flag, p.err, 3);
         // both gate warps leave together: a thread whose wait gave up never
         // leaves the other waiting at the group's barrier
         if (named_bar_any(kBarGate, 64, !ok || *x.abort_flag)) break;
         const int k = B.sitem[s];
+        if (FP8) {   // widen the stage's E4M3 q, k tiles to bf16 first (the next [Q;K] K^T waits on it)
+            if (k >= 0) {
+                ok = wait_bar(&B.st_full[s], (i / kNS) & 1, x.abort_flag, p.err, 36);
+                if (named_bar_any(kBarGate, 64, !ok || *x.abort_flag)) break;
+                const int bh = decode_item(p, k).bh;
+                uint8_t *st = x.smem + kWStage + s * kWStageBytes;
+                // q codes (in K's kb0 spot) into Q's tiles; then k codes (in K's kb1
+                // spot) into K's tiles, over both code tiles once they are read
+#pragma unroll 1
+                for (int rd = 0; rd < 2; ++rd)
+                    e4m3_tile_to_bf16(st + (rd ? 24576 : 8192), st + (rd ? 8192 : 0), st + (rd ? 24576 : 16384),
+                                      __ldg((rd ? p.k_scale : p.q_scale) + bh), gpt, kBarGate);
+                fence_proxy_async_smem();
+                named_bar(kBarGate, 64);
+            }
+            if (gpt == 0) mbar_arrive(&B.cv_full[s]);   // (the end marker too)
+        }
+        if (i >= kNG) {
+            ok = wait_bar(&B.g_empty[gj], ((i / kNG) + 1) & 1, x.abort_flag, p.err, 3);
+            if (named_bar_any(kBarGate, 64, !ok || *x.abort_flag)) break;
+        }
         if (k < 0) {   // past the last item: pass the end on
             if (gpt == 0) {
                 B.gitem[gj] = -1;
@@ -372,14 +455,15 @@ __device__ __forceinline__ void worker_gates(const Ctx &x, const PoolParams &p, 
 // places): 1 issued, 0 no such item (the end), -1 inputs not ready yet (only
 // when !block), -2 abort.
 __device__ __noinline__ int issue_qk(Bars *Bp, volatile int *abort_flag, int *err, uint32_t sbase, uint32_t tm,
-                                     int i, bool block)
+                                     int i, bool block, bool fp8)
 {
     Bars &B = *Bp;
     const int s = i % kNS, b1 = i & 1;
-    if (!block && !(mbar_test_wait(&B.st_full[s], (i / kNS) & 1) &&
+    uint64_t *ready = fp8 ? &B.cv_full[s] : &B.st_full[s];   // the stage's bf16 q, k tiles
+    if (!block && !(mbar_test_wait(ready, (i / kNS) & 1) &&
                     (i < 2 || mbar_test_wait(&B.d1_empty[b1], ((i >> 1) + 1) & 1))))
         return -1;
-    if (!wait_bar(&B.st_full[s], (i / kNS) & 1, abort_flag, err, 4)) return -2;
+    if (!wait_bar(ready, (i / kNS) & 1, abort_flag, err, 4)) return -2;
     if (B.sitem[s] < 0) return 0;
     if (i >= 2 && !wait_bar(&B.d1_empty[b1], ((i >> 1) + 1) & 1, abort_flag, err, 5)) return -2;
     const uint32_t sQK = sbase + kWStage + s * kWStageBytes;
@@ -391,6 +475,7 @@ __device__ __noinline__ int issue_qk(Bars *Bp, volatile int *abort_flag, int *er
     return 1;
 }
 
+template <bool FP8>
 __device__ __forceinline__ void worker_mma(const Ctx &x, const PoolParams &p)
 {
     Bars &B = *x.bars;
@@ -399,7 +484,7 @@ __device__ __forceinline__ void worker_mma(const Ctx &x, const PoolParams &p)
     int next = 0;    // next item whose [Q;K] K^T is to be issued
     auto step_m1 = [&](bool block) -> bool {   // false on abort
         if (last >= 0) return true;
-        const int r = issue_qk(x.bars, x.abort_flag, p.err, x.sbase, tm, next, block);
+        const int r = issue_qk(x.bars, x.abort_flag, p.err, x.sbase, tm, next, block, FP8);
         if (r == -2) return false;
         if (r == 0) last = next;
         if (r == 1) {
@@ -530,6 +615,7 @@ __device__ __forceinline__ void worker_solver(const Ctx &x, const PoolParams &p,
 // Finisher group (4 warps, warp w reads TMEM lane quarter qd = w % 4): per item,
 // P T1 and P T2 into the operand tiles, Q' = gamma Q - P T1 K and -W = -T1 K into
 // A2, then the item's slot in its scan's ring.
+template <bool FP8>
 __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &p, int ft, int qd)
 {
     Bars &B = *x.bars;
@@ -597,7 +683,7 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
         // ---- A2 = [gamma Q - P T1 K; -T1 K]
         // (the waits below also order this group's reads of the Q tile and of the
         // solver's T2 rows after the writes that published them)
-        wait_bar(&B.st_full[i % kNS], (i / kNS) & 1, x.abort_flag, p.err, 16);
+        wait_bar(FP8 ? &B.cv_full[i % kNS] : &B.st_full[i % kNS], (i / kNS) & 1, x.abort_flag, p.err, 16);
         wait_bar(&B.tp_full[b], (i >> 1) & 1, x.abort_flag, p.err, 17);
         wait_bar(&B.d3_full, i & 1, x.abort_flag, p.err, 18);
         if (ft == 0) tr(p, 0, 11, i);
@@ -675,7 +761,7 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
 
 // ================================================================== chains
 
-template <int DIR>
+template <int DIR, bool FP8>
 __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, const CUtensorMap *tmV,
                                           const PoolParams &p)
 {
@@ -684,14 +770,21 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
     const int *seq = p.slot_seq + (size_t)x.scan * kNSlot;
     for (int i = 0; i < x.NC; ++i) {
         const int st = i % kNVK, ab = i & 1, s = i % kNSlot;
-        if (i >= kNVK && !wait_bar(&B.vk_empty[st], ((i / kNVK) + 1) & 1, x.abort_flag, p.err, 21)) break;
         const int c = chunk_of<DIR>(x, i);
-        uint8_t *sv = x.smem + kCStage + st * 32768;
-        mbar_arrive_expect_tx(&B.vk_full[st], 32768);
-        tma_load_3d(sv, tmV, &B.vk_full[st], 0, c * kC, x.bh);
-        tma_load_3d(sv + 8192, tmV, &B.vk_full[st], 64, c * kC, x.bh);
-        tma_load_3d(sv + 16384, tmK, &B.vk_full[st], 0, c * kC, x.bh);
-        tma_load_3d(sv + 24576, tmK, &B.vk_full[st], 64, c * kC, x.bh);
+        if (FP8) {   // the E4M3 v, k tiles into the staging (widened into the V/K stage by the converters)
+            if (i >= 1 && !wait_bar(&B.s8_empty, (i - 1) & 1, x.abort_flag, p.err, 37)) break;
+            mbar_arrive_expect_tx(&B.s8_full, 16384);
+            tma_load_3d(x.smem + kC8, tmV, &B.s8_full, 0, c * kC, x.bh);
+            tma_load_3d(x.smem + kC8 + 8192, tmK, &B.s8_full, 0, c * kC, x.bh);
+        } else {
+            if (i >= kNVK && !wait_bar(&B.vk_empty[st], ((i / kNVK) + 1) & 1, x.abort_flag, p.err, 21)) break;
+            uint8_t *sv = x.smem + kCStage + st * 32768;
+            mbar_arrive_expect_tx(&B.vk_full[st], 32768);
+            tma_load_3d(sv, tmV, &B.vk_full[st], 0, c * kC, x.bh);
+            tma_load_3d(sv + 8192, tmV, &B.vk_full[st], 64, c * kC, x.bh);
+            tma_load_3d(sv + 16384, tmK, &B.vk_full[st], 0, c * kC, x.bh);
+            tma_load_3d(sv + 24576, tmK, &B.vk_full[st], 64, c * kC, x.bh);
+        }
         vk_issued = i + 1;
         if (i >= 2 && !wait_bar(&B.a_empty[ab], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 22)) break;
         tr(p, 1, 0, i);
@@ -709,9 +802,42 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
         a_issued = i + 1;
     }
     if (*x.abort_flag) {
-        for (int i = (vk_issued > kNVK ? vk_issued - kNVK : 0); i < vk_issued; ++i)
-            drain_copies(&B.vk_full[i % kNVK], (i / kNVK) & 1);
+        if (FP8) {   // one staging load in flight at most
+            if (vk_issued > 0) drain_copies(&B.s8_full, (vk_issued - 1) & 1);
+        } else {
+            for (int i = (vk_issued > kNVK ? vk_issued - kNVK : 0); i < vk_issued; ++i)
+                drain_copies(&B.vk_full[i % kNVK], (i / kNVK) & 1);
+        }
         for (int i = (a_issued > 2 ? a_issued - 2 : 0); i < a_issued; ++i) drain_copies(&B.a_full[i & 1], (i >> 1) & 1);
+    }
+}
+
+// Converters (2 warps, fp8 inputs): per chunk, the staged E4M3 v, k tiles
+// widened to scaled bf16 into the V/K stage the chain's products read.
+__device__ __forceinline__ void chain_convert(const Ctx &x, const PoolParams &p, int t)
+{
+    Bars &B = *x.bars;
+    const float sv = __ldg(p.v_scale + x.bh), sk = __ldg(p.k_scale + x.bh);
+#pragma unroll 1
+    for (int i = 0; i < x.NC; ++i) {
+        const int st = i % kNVK;
+        bool ok = true;
+        if (t == 0) {
+            ok = wait_bar(&B.s8_full, i & 1, x.abort_flag, p.err, 38);
+            if (ok && i >= kNVK) ok = wait_bar(&B.vk_empty[st], ((i / kNVK) + 1) & 1, x.abort_flag, p.err, 39);
+        }
+        if (named_bar_any(kBarConv, 64, !ok || *x.abort_flag)) break;
+        uint8_t *stage = x.smem + kCStage + st * 32768;   // [V0 | V1 | K0 | K1]
+#pragma unroll 1
+        for (int rd = 0; rd < 2; ++rd)
+            e4m3_tile_to_bf16(x.smem + kC8 + 8192 * rd, stage + 16384 * rd, stage + 16384 * rd + 8192, rd ? sk : sv,
+                              t, kBarConv);
+        fence_proxy_async_smem();
+        named_bar(kBarConv, 64);
+        if (t == 0) {
+            mbar_arrive(&B.s8_empty);   // the staging may take the next chunk's codes
+            mbar_arrive(&B.vk_full[st]);
+        }
     }
 }
 
@@ -975,6 +1101,9 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
 
 // ================================================================== kernel
 
+// FP8: q, k, v are E4M3 codes, widened in shared memory (a separate
+// instantiation, so that the bf16 kernel carries none of that code).
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -1040,21 +1169,21 @@ gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 
     if (!chain) {
         if (warp == 0) {
-            if (lane == 0) worker_tma(x, &tmQ, &tmK, p);
+            if (lane == 0) worker_tma<FP8>(x, &tmQ, &tmK, p);
         } else if (warp == 1) {
-            if (lane == 0) worker_mma(x, p);
+            if (lane == 0) worker_mma<FP8>(x, p);
         } else if (warp < 10) {
             worker_solver(x, p, tid - 64, warp & 3, (warp - 2) >> 2);
         } else if (warp < 14) {
-            worker_finisher(x, p, tid - 320, warp & 3);
+            worker_finisher<FP8>(x, p, tid - 320, warp & 3);
         } else {
-            worker_gates(x, p, tid - 448);
+            worker_gates<FP8>(x, p, tid - 448);
         }
     } else {
         if (warp == 0) {
             if (lane == 0) {
-                if (x.dir) chain_tma<1>(x, &tmK, &tmV, p);
-                else chain_tma<0>(x, &tmK, &tmV, p);
+                if (x.dir) chain_tma<1, FP8>(x, &tmK, &tmV, p);
+                else chain_tma<0, FP8>(x, &tmK, &tmV, p);
             }
         } else if (warp == 1) {
             if (lane == 0) chain_mma(x, p);
@@ -1066,6 +1195,8 @@ gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             const int ot = tid - 320, q = warp & 3;
             if (x.dir) chain_out<1>(x, p, &tmO, ot, q);
             else chain_out<0>(x, p, &tmO, ot, q);
+        } else if (FP8) {
+            chain_convert(x, p, tid - 448);
         }
     }
 
@@ -1096,17 +1227,21 @@ EncodeTiledFn get_encoder()
 }
 
 // 3D map over a [BH, T, 128] bf16 tensor; box = 64 (inner) x 64 (tokens) x 1, 128B swizzle.
-bool make_map(CUtensorMap *m, const void *base, int T, int BH)
+// 3D map over a [BH, T, 128] tensor of 2-byte (bf16) or 1-byte (E4M3 code)
+// elements; box = 128 bytes (64 bf16 or 128 codes) x 64 tokens x 1, 128B swizzle.
+bool make_map(CUtensorMap *m, const void *base, int T, int BH, bool bytes = false)
 {
     EncodeTiledFn enc = get_encoder();
     if (!enc) return false;
+    const cuuint64_t row = bytes ? 128 : 256;
     cuuint64_t dims[3] = {128, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {256, (cuuint64_t)T * 256};
-    cuuint32_t box[3] = {64, 64, 1};
+    cuuint64_t strides[2] = {row, (cuuint64_t)T * row};
+    cuuint32_t box[3] = {bytes ? 128u : 64u, 64, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -1127,8 +1262,11 @@ cudaError_t device_info(DevInfo **out)
     std::lock_guard<std::mutex> lock(mu);
     DevInfo &d = info[dev];
     if (!d.init) {
-        err = cudaFuncSetAttribute(gdn_chunk_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        err = cudaFuncSetAttribute(gdn_chunk_pool_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)kSmemAlloc);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(gdn_chunk_pool_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemAlloc);
         if (err == cudaSuccess) err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
         if (err != cudaSuccess) return err;
         d.init = true;
@@ -1148,12 +1286,14 @@ bool chunk_pool_supported(const FwdArgs &a)
            a.seg_chunks == 0;
 }
 
-cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream)
+cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream, const float *q_scale, const float *k_scale,
+                              const float *v_scale)
 {
     CUtensorMap mq, mk, mv, mo;
     const int BH_all = a.B * a.H;
-    if (!make_map(&mq, a.q, a.T, BH_all) || !make_map(&mk, a.k, a.T, BH_all) ||
-        !make_map(&mv, a.v, a.T, BH_all) || !make_map(&mo, a.o, a.T, BH_all))
+    const bool fp8 = q_scale != nullptr;
+    if (!make_map(&mq, a.q, a.T, BH_all, fp8) || !make_map(&mk, a.k, a.T, BH_all, fp8) ||
+        !make_map(&mv, a.v, a.T, BH_all, fp8) || !make_map(&mo, a.o, a.T, BH_all))
         return cudaErrorInvalidValue;
     DevInfo *info = nullptr;
     cudaError_t err = device_info(&info);
@@ -1192,6 +1332,9 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream)
         p.work = p.consumed + p.n_scans;
         p.counters = a.bidi ? p.work + 1 : nullptr;
         p.stall_chunk = h0 == 0 ? g_stall_chunk : -1;
+        p.q_scale = q_scale;
+        p.k_scale = k_scale;
+        p.v_scale = v_scale;
         err = device_error_word(&p.err);
         if (err != cudaSuccess) break;
         err = cudaMemsetAsync(flags, 0, flag_ints * sizeof(int), stream);
@@ -1208,7 +1351,8 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream)
         at[0].val.cooperative = 1;
         cfg.attrs = at;
         cfg.numAttrs = g_plain_launch ? 0 : 1;
-        err = cudaLaunchKernelEx(&cfg, gdn_chunk_pool_kernel, mq, mk, mv, mo, p);
+        err = fp8 ? cudaLaunchKernelEx(&cfg, gdn_chunk_pool_kernel<true>, mq, mk, mv, mo, p)
+                  : cudaLaunchKernelEx(&cfg, gdn_chunk_pool_kernel<false>, mq, mk, mv, mo, p);
         if (err == cudaSuccess) err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }

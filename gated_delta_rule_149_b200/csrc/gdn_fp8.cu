@@ -1,10 +1,12 @@
 // fp8 (E4M3) q, k, v with one fp32 scale per (batch, head): x = scale * x8.
 //
-// This form dequantises in a pre-pass (16 codes per thread step, through the
-// CUDA fp8 conversion) into bf16 workspace copies and runs the chunkwise
-// kernel on them; it accepts fp8 inputs but does not yet save their bandwidth
-// (the chunkwise kernel's tensor-core products pair q, k and v with bf16
-// operands, and both operands of one product must have the same type).
+// dk = dv = 128 (the pooled kernel): the kernel loads the codes by TMA, one
+// byte per element, and widens each tile to scaled bf16 in shared memory
+// before the tensor-core products (both operands of one product must have the
+// same type, and the other operands are bf16).  Other shapes (dv = 64, or the
+// single-CTA kernel forced): a pre-pass dequantises into bf16 workspace copies
+// (16 codes per thread step, through the CUDA fp8 conversion) and the
+// chunkwise kernel runs on them.
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -49,6 +51,8 @@ size_t align_up256(size_t n) { return (n + 255) & ~(size_t)255; }
 cudaError_t launch_fp8(const FwdArgs &a, const float *q_scale, const float *k_scale, const float *v_scale,
                        cudaStream_t stream)
 {
+    // dk = dv = 128: the pooled kernel loads the codes and widens them itself
+    if (chunk_pool_supported(a)) return launch_chunk_pool(a, stream, q_scale, k_scale, v_scale);
     const size_t BH = (size_t)a.B * a.H, nk = BH * a.T * a.dk, nv = BH * a.T * a.dv;
     const size_t bq = align_up256(nk * 2), bv = align_up256(nv * 2);
     uint8_t *ws = nullptr;

@@ -35,7 +35,10 @@ cudaError_t launch_chunk_tc(const FwdArgs &a, cudaStream_t stream);
 // preparation workers that serve every scan (bf16, dk = dv = 128, whole
 // sequences, no segments).  launch_chunk_tc hands such calls to it.
 bool chunk_pool_supported(const FwdArgs &a);
-cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream);
+// The pooled chunkwise kernel; with q_scale (and k_scale, v_scale) given, a.q,
+// a.k and a.v are E4M3 codes with one fp32 scale per head, widened in-kernel.
+cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream, const float *q_scale = nullptr,
+                              const float *k_scale = nullptr, const float *v_scale = nullptr);
 
 // Allocation-free variant of launch_chunk_tc: the bidirectional arrival
 // counters come from a fixed static device array of noalloc_capacity() ints.
