@@ -2,9 +2,10 @@
 // serial state chains (one CTA per scan) and a pool of preparation workers
 // that serve every scan.
 //
-// The recurrence (librediffusion PR #21 page, "What's added": the GDN
-// linear-attention recurrence; the causal-streaming and bidirectional forms
-// of the flashdreams SANA-WM page), per head, with H = S^T (dk x dv):
+// The recurrence (the GDN linear-attention recurrence that the librediffusion
+// PR #21 page names in "What's added", in the causal-streaming and
+// bidirectional forms of the flashdreams SANA-WM page; the pages print no
+// formula, this is the gated delta rule), per head, with H = S^T (dk x dv):
 //     H_t = a_t (I - b_t k_t k_t^T) H_{t-1} + b_t k_t v_t^T,   o_t = H_t^T q_t
 // is evaluated 64 tokens at a time in its WY/UT form.  Per chunk, in scan
 // order, with g = log2 a, G_i = sum of g up to and including token i,
@@ -129,6 +130,7 @@ constexpr bool kDbgOn = false;
 #endif
 
 constexpr uint32_t kIdM1 = idesc_bf16(128, 64, false, false);   // [Q;K] K^T
+constexpr uint32_t kIdM1f8 = idesc_e4m3(128, 64, false, false); // [Q;K] K^T on E4M3 codes
 constexpr uint32_t kIdM2 = idesc_bf16(64, 128, false, true);    // P [T1 | T2]
 constexpr uint32_t kIdM3 = idesc_bf16(128, 128, false, true);   // [P T1; T1] K
 constexpr uint32_t kIdA = idesc_bf16(128, 128, true, false);    // V^T A1^T
@@ -281,6 +283,22 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &c, float scale, uin
         }
 }
 
+// 16 codes times `scale`, as fp32
+__device__ __forceinline__ void e4m3x16_to_f32(const uint4 &c, float scale, float (&f)[16])
+{
+    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const __half2_raw hr =
+                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(words[i] >> (16 * h)), __NV_E4M3);
+            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+            f[4 * i + 2 * h] = v.x * scale;
+            f[4 * i + 2 * h + 1] = v.y * scale;
+        }
+}
+
 // Thread t (of 64) takes the 16-code chunk t % 8 of rows t / 8 + 8 n.  Every
 // thread reads its chunks before the group's barrier and writes after it, so
 // a destination may overlap the source.
@@ -330,10 +348,10 @@ __device__ __forceinline__ void worker_tma(const Ctx &x, const CUtensorMap *tmQ,
         B.sitem[s] = k;
         mbar_arrive(&B.it_full[s]);
         uint8_t *st = x.smem + kWStage + s * kWStageBytes;
-        if (FP8) {   // the E4M3 q, k tiles into the stage's K spots, widened in place by the gate warps
+        if (FP8) {   // the E4M3 q, k tiles: [Q8; K8], the A operand of [Q;K] K^T on codes
             mbar_arrive_expect_tx(&B.st_full[s], 16384);
-            tma_load_3d(st + 8192, tmQ, &B.st_full[s], 0, it.c * kC, it.bh);
-            tma_load_3d(st + 24576, tmK, &B.st_full[s], 0, it.c * kC, it.bh);
+            tma_load_3d(st, tmQ, &B.st_full[s], 0, it.c * kC, it.bh);
+            tma_load_3d(st + 8192, tmK, &B.st_full[s], 0, it.c * kC, it.bh);
         } else {
             mbar_arrive_expect_tx(&B.st_full[s], 32768);
             for (int kb = 0; kb < 2; ++kb) {
@@ -362,18 +380,13 @@ __device__ __forceinline__ void worker_gates(const Ctx &x, const PoolParams &p, 
         // leaves the other waiting at the group's barrier
         if (named_bar_any(kBarGate, 64, !ok || *x.abort_flag)) break;
         const int k = B.sitem[s];
-        if (FP8) {   // widen the stage's E4M3 q, k tiles to bf16 first (the next [Q;K] K^T waits on it)
+        if (FP8) {   // widen the stage's k codes to bf16 (for [P T1; T1] K) beside them
             if (k >= 0) {
                 ok = wait_bar(&B.st_full[s], (i / kNS) & 1, x.abort_flag, p.err, 36);
                 if (named_bar_any(kBarGate, 64, !ok || *x.abort_flag)) break;
-                const int bh = decode_item(p, k).bh;
                 uint8_t *st = x.smem + kWStage + s * kWStageBytes;
-                // q codes (in K's kb0 spot) into Q's tiles; then k codes (in K's kb1
-                // spot) into K's tiles, over both code tiles once they are read
-#pragma unroll 1
-                for (int rd = 0; rd < 2; ++rd)
-                    e4m3_tile_to_bf16(st + (rd ? 24576 : 8192), st + (rd ? 8192 : 0), st + (rd ? 24576 : 16384),
-                                      __ldg((rd ? p.k_scale : p.q_scale) + bh), gpt, kBarGate);
+                e4m3_tile_to_bf16(st + 8192, st + 16384, st + 24576, __ldg(p.k_scale + decode_item(p, k).bh), gpt,
+                                  kBarGate);
                 fence_proxy_async_smem();
                 named_bar(kBarGate, 64);
             }
@@ -459,18 +472,23 @@ __device__ __noinline__ int issue_qk(Bars *Bp, volatile int *abort_flag, int *er
 {
     Bars &B = *Bp;
     const int s = i % kNS, b1 = i & 1;
-    uint64_t *ready = fp8 ? &B.cv_full[s] : &B.st_full[s];   // the stage's bf16 q, k tiles
-    if (!block && !(mbar_test_wait(ready, (i / kNS) & 1) &&
+    if (!block && !(mbar_test_wait(&B.st_full[s], (i / kNS) & 1) &&
                     (i < 2 || mbar_test_wait(&B.d1_empty[b1], ((i >> 1) + 1) & 1))))
         return -1;
-    if (!wait_bar(ready, (i / kNS) & 1, abort_flag, err, 4)) return -2;
+    if (!wait_bar(&B.st_full[s], (i / kNS) & 1, abort_flag, err, 4)) return -2;
     if (B.sitem[s] < 0) return 0;
     if (i >= 2 && !wait_bar(&B.d1_empty[b1], ((i >> 1) + 1) & 1, abort_flag, err, 5)) return -2;
     const uint32_t sQK = sbase + kWStage + s * kWStageBytes;
     const uint64_t a = sw128_desc(sQK, 16, 1024), b = sw128_desc(sQK + 8192, 16, 1024);
     tc_fence_after();
-    mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a, b, kIdM1, false);
-    mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a + 1024, b + 1024, kIdM1, true);
+    if (fp8) {   // [Q8; K8] K8^T: one 128-byte row of codes per token, 32 codes per K step
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            mma_f8(tm + kTD1 + 64 * b1, a + (uint64_t)(2 * k), b + (uint64_t)(2 * k), kIdM1f8, k > 0 ? 1u : 0u);
+    } else {
+        mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a, b, kIdM1, false);
+        mma_run<4, 2, 2>(tm + kTD1 + 64 * b1, a + 1024, b + 1024, kIdM1, true);
+    }
     mma_commit(&B.d1_full[b1]);
     return 1;
 }
@@ -510,10 +528,17 @@ __device__ __forceinline__ void worker_mma(const Ctx &x, const PoolParams &p)
         if (next == j + 2 && !step_m1(false)) break;
         if (!wait_bar(&B.e2_done, j & 1, x.abort_flag, p.err, 8)) break;
         if (j >= 1 && !wait_bar(&B.d3_empty, (j - 1) & 1, x.abort_flag, p.err, 9)) break;
+        // fp8: K widened to bf16 by the gate warps
+        if (FP8 && !wait_bar(&B.cv_full[j % kNS], (j / kNS) & 1, x.abort_flag, p.err, 41)) break;
         tc_fence_after();
-        // [P T1; T1] K: B = K [token][dk] MN-major, dk groups 16 KB apart in the stage
-        mma_run<4, 2, 128>(tm + kTD3, sw128_desc(tb, 16, 1024),
-                           sw128_desc(x.sbase + kWStage + (j % kNS) * kWStageBytes + 8192, 16384, 1024), kIdM3, false);
+        // [P T1; T1] K: B = K [token][dk] MN-major, dk groups 16 KB apart in the
+        // stage (fp8: 8 KB apart, beside the codes)
+        {
+            const uint32_t st = x.sbase + kWStage + (j % kNS) * kWStageBytes;
+            mma_run<4, 2, 128>(tm + kTD3, sw128_desc(tb, 16, 1024),
+                               FP8 ? sw128_desc(st + 16384, 8192, 1024) : sw128_desc(st + 8192, 16384, 1024), kIdM3,
+                               false);
+        }
         mma_commit(&B.d3_full);
         mma_commit(&B.t_free[bj]);
         tr(p, 0, 18, j);
@@ -529,14 +554,15 @@ __device__ __forceinline__ void worker_mma(const Ctx &x, const PoolParams &p)
 // 2^(G_r - G_j) is a product of a row and a column factor when the chunk's
 // factors are all normal floats (`fact`), else one exp2 of the difference.
 __device__ __forceinline__ void mask_rows(uint32_t taddr, const float *gt, float *As, uint8_t *sP, int qd,
-                                          int lane, int hf, bool fact, int dir)
+                                          int lane, int hf, bool fact, int dir, float sc_p, float sc_a)
 {
     const int r = (qd & 1) * 32 + lane;                  // physical token row
     const int lr = dir ? 63 - r : r;                     // its scan position
     const bool pm = qd < 2;                              // P (else A)
     const bool useB = lr >= 32 && (dir ? (hf == 1) : (hf == 0));   // cross-half pairs
     const float *cf = gt + (useB ? gCB : gCA) * 64 + 32 * hf;
-    const float br = pm ? 1.f : gt[gBet * 64 + r];
+    // sc_p, sc_a: the input scales of the [Q;K] K^T rows (fp8 codes), else 1
+    const float br = pm ? sc_p : sc_a * gt[gBet * 64 + r];
     const float rf = br * gt[(useB ? gRB : gRA) * 64 + r];
     const int j0 = 32 * hf;                              // physical column of xv[0]
     float xv[32];
@@ -572,6 +598,7 @@ __device__ __forceinline__ void mask_rows(uint32_t taddr, const float *gt, float
 // Solver group (8 warps; warp w reads TMEM lane quarter qd = w % 4 and columns
 // [32 hf, +32) of each row it owns): per item, the masks of [Q;K] K^T, then
 // T = (I + A)^-1 written as T1 = T diag(b gamma) and T2 = T diag(b).
+template <bool FP8>
 __device__ __forceinline__ void worker_solver(const Ctx &x, const PoolParams &p, int pt, int qd, int hf)
 {
     Bars &B = *x.bars;
@@ -587,13 +614,21 @@ __device__ __forceinline__ void worker_solver(const Ctx &x, const PoolParams &p,
         wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 10);
         const int k = B.gitem[gi];
         if (named_bar_any(kBarA, kGroup, *x.abort_flag || k < 0)) return;
-        const int dir = decode_item(p, k).dir;
+        const Item itk = decode_item(p, k);
+        const int dir = itk.dir;
+        float sc_p = 1.f, sc_a = 1.f;   // fp8: [Q;K] K^T was formed on the codes
+        if (FP8) {
+            const float sk = __ldg(p.k_scale + itk.bh);
+            sc_p = __ldg(p.q_scale + itk.bh) * sk;
+            sc_a = sk * sk;
+        }
         const bool fact = B.gscal[gi][1] != 0.f;
         wait_bar(&B.d1_full[b], (i >> 1) & 1, x.abort_flag, p.err, 11);
         if (i >= 1) wait_bar(&B.p_free, (i - 1) & 1, x.abort_flag, p.err, 12);   // P of item i - 1 is read
         if (pt == 0) tr(p, 0, 1, i);
         tc_fence_after();
-        mask_rows(x.tmem + tm_lane + kTD1 + 64 * b + 32 * hf, gt, As, x.smem + kPP, qd, lane, hf, fact, dir);
+        mask_rows(x.tmem + tm_lane + kTD1 + 64 * b + 32 * hf, gt, As, x.smem + kPP, qd, lane, hf, fact, dir, sc_p,
+                  sc_a);
         tc_fence_before();
         fence_proxy_async_smem();
         if (named_bar_any(kBarA, kGroup, *x.abort_flag)) return;
@@ -681,9 +716,9 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
         if (ft == 0) tr(p, 0, 10, i);
 
         // ---- A2 = [gamma Q - P T1 K; -T1 K]
-        // (the waits below also order this group's reads of the Q tile and of the
-        // solver's T2 rows after the writes that published them)
-        wait_bar(FP8 ? &B.cv_full[i % kNS] : &B.st_full[i % kNS], (i / kNS) & 1, x.abort_flag, p.err, 16);
+        // (the waits below also order this group's reads of the Q tile (fp8: its
+        // codes) and of the solver's T2 rows after the writes that published them)
+        wait_bar(&B.st_full[i % kNS], (i / kNS) & 1, x.abort_flag, p.err, 16);
         wait_bar(&B.tp_full[b], (i >> 1) & 1, x.abort_flag, p.err, 17);
         wait_bar(&B.d3_full, i & 1, x.abort_flag, p.err, 18);
         if (ft == 0) tr(p, 0, 11, i);
@@ -691,6 +726,7 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
         {
             const int n = 32 * qd + lane;   // row of [P T1; T1] K
             const float gq = (n < 64) ? gt[gGam * 64 + n] : 0.f;
+            const float sq = FP8 ? __ldg(p.q_scale + it.bh) : 1.f;
             float v[32];
 #pragma unroll 1
             for (int kb = 0; kb < 2; ++kb) {
@@ -700,7 +736,17 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
                 for (int h2 = 0; h2 < 2; ++h2) {
                     tmem_ld32(x.tmem + tm_lane + kTD3 + 64 * kb + 32 * h2, v);
                     tmem_wait_ld();
-                    if (n < 64) {
+                    if (FP8 && n < 64) {   // gamma Q from the q codes: chunks 4 kb + 2 h2, + 1 of row n
+                        const uint8_t *qc = x.smem + kWStage + (i % kNS) * kWStageBytes + n * 128;
+#pragma unroll
+                        for (int hc = 0; hc < 2; ++hc) {
+                            const int j = 4 * kb + 2 * h2 + hc;
+                            float f[16];
+                            e4m3x16_to_f32(*reinterpret_cast<const uint4 *>(qc + ((j ^ (n & 7)) << 4)), sq, f);
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) v[16 * hc + e] = fmaf(gq, f[e], -v[16 * hc + e]);
+                        }
+                    } else if (n < 64) {
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             const uint4 w = *reinterpret_cast<const uint4 *>(qrow + sw128_off(n, 32 * h2 + 8 * q4));
@@ -1173,7 +1219,7 @@ gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         } else if (warp == 1) {
             if (lane == 0) worker_mma<FP8>(x, p);
         } else if (warp < 10) {
-            worker_solver(x, p, tid - 64, warp & 3, (warp - 2) >> 2);
+            worker_solver<FP8>(x, p, tid - 64, warp & 3, (warp - 2) >> 2);
         } else if (warp < 14) {
             worker_finisher<FP8>(x, p, tid - 320, warp & 3);
         } else {

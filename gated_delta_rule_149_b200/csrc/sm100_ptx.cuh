@@ -115,6 +115,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
                  : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f8f6f4 (8-bit A and B in the
+// formats the instruction descriptor names, fp32 accumulate; K = 32 per instruction)
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc], kind::f16: the A operand (M rows, one per
 // TMEM lane; K bf16 values packed two per 32-bit column, K/2 columns) is read
 // from tensor memory instead of shared memory.
@@ -311,6 +323,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
          | (1u << 7)                       // A format: bf16
          | (1u << 10)                      // B format: bf16
          | ((neg_a ? 1u : 0u) << 13)
+         | ((a_mn ? 1u : 0u) << 15)
+         | ((b_mn ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f8f6f4 with E4M3 A and B (format code 0) and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4)                       // D format: f32
+         | (0u << 7)                       // A format: E4M3
+         | (0u << 10)                      // B format: E4M3
          | ((a_mn ? 1u : 0u) << 15)
          | ((b_mn ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)

@@ -2,11 +2,13 @@
  * gdn.h -- C ABI of libgdn, the Gated-Delta-Net (GDN) linear-attention
  * recurrence on NVIDIA B200 (sm_100a).
  *
- * The operation (the "GDN (Gated-Delta-Net) linear-attention recurrence" of the
- * librediffusion PR #21 page, "What's added"; the streaming/bidirectional
- * forms of the flashdreams SANA-WM page, "Bidirectional variant", and the
- * causal linear-attention KV cache of the LongSANA diffusers PR #12723 page,
- * "PR feature"), per batch b and head h, with a dv x dk state S:
+ * The operation: the "GDN (Gated-Delta-Net) linear-attention recurrence" that
+ * the librediffusion PR #21 page names ("What's added"), in the streaming and
+ * bidirectional forms of the flashdreams SANA-WM page ("Bidirectional
+ * variant") and the causal linear-attention KV cache of the LongSANA diffusers
+ * PR #12723 page ("PR feature").  The pages print no formula; the update is
+ * the gated delta rule (Gated DeltaNet), per batch b and head h, with a
+ * dv x dk state S:
  *
  *     S_t = a_t * S_{t-1} * (I - b_t k_t k_t^T) + b_t v_t k_t^T
  *     o_t = S_t q_t
@@ -14,10 +16,16 @@
  * a_t = decay[b,h,t], b_t = beta[b,h,t].  The stored state is H = S^T, a
  * row-major [dk][dv] fp32 matrix per head.  No 1/sqrt(dk) factor is applied.
  *
+ * Precondition on the gates: decay in (0, 1] (a gate), beta finite (typically
+ * in [0, 1]).  The chunkwise kernels work with log2 decay: a decay below
+ * 2^-120 acts as 2^-120, and decays above 1 (growth) are computed as written
+ * only while every product of decays within a 64-token chunk stays a normal
+ * fp32 number (checked up to 1 + 1e-3); the library does not scan the gates.
+ *
  * Layouts (all row-major, contiguous, element strides implied by the sizes):
  *   q, k        [B, H, T, dk]      bf16 or fp32 (mode bit GDN_FP32)
  *   v, o        [B, H, T, dv]      same dtype as q
- *   beta, decay [B, H, T]          fp32; decay in (0, 1], beta in [0, 1] typical
+ *   beta, decay [B, H, T]          fp32 (see the precondition above)
  *   state_in    [B, H, dk, dv]     fp32, or NULL for a zero initial state
  *   state_out   causal: [B, H, dk, dv];  bidi: [2, B, H, dk, dv] =
  *               {forward final state, reverse final state}; or NULL to skip

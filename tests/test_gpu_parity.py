@@ -131,6 +131,18 @@ def test_bf16_no_decay_unit_gates(oracle_mod, kernel):
 
 
 @pytest.mark.parametrize("kernel", BF16_KERNELS)
+@pytest.mark.parametrize("bidi", [False, True])
+def test_bf16_decay_slightly_above_one(oracle_mod, kernel, bidi):
+    # the gates' precondition is decay in (0, 1]; growth up to 1 + 1e-3 per token
+    # keeps every within-chunk decay product a normal float and is computed as written
+    inp = make_custom(1, 2, 333, 128, 128, dtype="bf16", seed=14, bidi=bidi, state0=True)
+    g = torch.Generator().manual_seed(15)
+    inp.decay.copy_(1.0 + 1e-3 * torch.rand(inp.decay.shape, generator=g))
+    assert float(inp.decay.min()) > 1.0
+    check(oracle_mod, inp, bidi, kernel)
+
+
+@pytest.mark.parametrize("kernel", BF16_KERNELS)
 def test_bf16_zero_inputs_keep_zero(kernel):
     inp = make_custom(1, 2, 130, 128, 128, dtype="bf16", seed=7)
     d = to_dev(inp)
