@@ -83,6 +83,12 @@ constexpr int kNG = 3;                    // gate buffers
 constexpr int kNS = 3;                    // worker input stages
 constexpr uint32_t kGateFloats = 9 * 64;
 constexpr int kNSlot = 8;                 // ring slots per scan
+// Flag words polled across SMs (a scan's slot sequence words, a scan's count
+// of chunks taken out, the item counter) each get their own 128-byte line:
+// sharing lines made the kernel up to 50 % slower depending on where the
+// workspace landed.
+constexpr int kFlagStride = 32;
+static_assert(kNSlot <= kFlagStride, "a scan's slot words share its line");
 
 // ring slot: A1 [128 rows x 64] bf16, A2 [kb][128 rows x 64] bf16 (both 128B-swizzled
 // images), then e[64] and gamma_end (fp32)
@@ -142,9 +148,9 @@ struct PoolParams {
     float *state_out;
     __nv_bfloat16 *o;
     uint8_t *ring;       // [n_scans][kNSlot] slots
-    int *slot_seq;       // [n_scans][kNSlot]: chunk + 1 once the slot holds that chunk, zeroed
-    int *consumed;       // [n_scans]: chunks the scan's chain has taken out of its ring, zeroed
-    int *work;           // next item to hand out, zeroed
+    int *slot_seq;       // [n_scans][kFlagStride], first kNSlot used: chunk + 1 once the slot holds it, zeroed
+    int *consumed;       // [n_scans][kFlagStride], first used: chunks the scan's chain has taken out, zeroed
+    int *work;           // next item to hand out (own line), zeroed
     int *counters;       // bidi arrival counters [BH][n_chunks] of this launch's heads, zeroed
     int *err;            // device error word
     float *debug;        // optional: chunk-0 D and S of scan 0
@@ -672,7 +678,7 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
         bulk_wait0();
         fence_proxy_async_global();
         __threadfence();
-        st_release_gpu(p.slot_seq + (size_t)pend_scan * kNSlot + pend_c % kNSlot, pend_c + 1);
+        st_release_gpu(p.slot_seq + (size_t)pend_scan * kFlagStride + pend_c % kNSlot, pend_c + 1);
         pend_scan = -1;
     };
 #pragma unroll 1
@@ -786,7 +792,7 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
         // ---- the item's slot: A1, A2, e, gamma_end (bulk copies, published an item later)
         if (ft == 0) {
             // the slot's previous chunk must have been taken out by the chain
-            if (it.ci < kNSlot || wait_global(p.consumed + it.scan, it.ci - kNSlot + 1, x, p, 64)) {
+            if (it.ci < kNSlot || wait_global(p.consumed + (size_t)it.scan * kFlagStride, it.ci - kNSlot + 1, x, p, 64)) {
                 uint8_t *slot = p.ring + ((size_t)it.scan * kNSlot + it.ci % kNSlot) * kSlotBytes;
                 bulk_store(slot + kSlotA1, tb + 16384, 16384);
                 bulk_store(slot + kSlotA2, x.smem + kPA2, 32768);
@@ -813,7 +819,7 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
 {
     Bars &B = *x.bars;
     int vk_issued = 0, a_issued = 0;
-    const int *seq = p.slot_seq + (size_t)x.scan * kNSlot;
+    const int *seq = p.slot_seq + (size_t)x.scan * kFlagStride;
     for (int i = 0; i < x.NC; ++i) {
         const int st = i % kNVK, ab = i & 1, s = i % kNSlot;
         const int c = chunk_of<DIR>(x, i);
@@ -895,7 +901,7 @@ __device__ __forceinline__ void chain_mma(const Ctx &x, const PoolParams &p)
         const int st = i % kNVK, ab = i & 1, db = i & 1;
         if (!wait_bar(&B.vk_full[st], (i / kNVK) & 1, x.abort_flag, p.err, 24)) break;
         if (!wait_bar(&B.a_full[ab], (i >> 1) & 1, x.abort_flag, p.err, 25)) break;
-        st_release_gpu(p.consumed + x.scan, i + 1);   // the slot's data has landed: it may be refilled
+        st_release_gpu(p.consumed + (size_t)x.scan * kFlagStride, i + 1);   // the slot's data has landed: it may be refilled
         tr(p, 1, 2, i);
         if (i >= 2 && !wait_bar(&B.d_empty[db], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 26)) break;
         tr(p, 1, 3, i);
@@ -1353,7 +1359,7 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream, const float
 
     const size_t n_scans_max = (size_t)dirs * heads;
     const size_t ring_bytes = n_scans_max * kNSlot * kSlotBytes;
-    const size_t flag_ints = n_scans_max * kNSlot + n_scans_max + 1 + (a.bidi ? (size_t)heads * n_chunks : 0);
+    const size_t flag_ints = (2 * n_scans_max + 1) * kFlagStride + (a.bidi ? (size_t)heads * n_chunks : 0);
     uint8_t *ws = nullptr;
     err = ws_alloc(reinterpret_cast<void **>(&ws), ring_bytes + flag_ints * sizeof(int), stream);
     if (err != cudaSuccess) return err;
@@ -1374,9 +1380,9 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream, const float
         p.trace = g_prof_buf;
         p.ring = g_debug_ring ? static_cast<uint8_t *>(g_debug_ring) : ws;
         p.slot_seq = flags;
-        p.consumed = flags + (size_t)p.n_scans * kNSlot;
-        p.work = p.consumed + p.n_scans;
-        p.counters = a.bidi ? p.work + 1 : nullptr;
+        p.consumed = flags + (size_t)p.n_scans * kFlagStride;
+        p.work = p.consumed + (size_t)p.n_scans * kFlagStride;
+        p.counters = a.bidi ? p.work + kFlagStride : nullptr;
         p.stall_chunk = h0 == 0 ? g_stall_chunk : -1;
         p.q_scale = q_scale;
         p.k_scale = k_scale;
