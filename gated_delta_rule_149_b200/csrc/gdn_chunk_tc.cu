@@ -738,15 +738,17 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
                 first = false;   // stored above, or added below
             }
         }
-        if (mine) {
-            if (first) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-            } else if (add) {
-                // the first writer's stored partial plus this direction's fp32
-                // partial, rounded to bf16 once (read past L1: the partial was
-                // written by another SM)
+        // second writer: the fp32 partial is read from TMEM again (the tile is
+        // released only after this step), so that it need not stay in registers
+        // across the waits above; the load is warp-wide (every lane takes part).
+        // It adds the first writer's stored partial (read past L1: written by
+        // another SM) and rounds to bf16 once.
+        if (__any_sync(0xffffffffu, add)) {
+            float xa[32];
+            tc_fence_after();
+            tmem_ld32(x.tmem + tm_lane + kColO0 + 64 * bj + 32 * chf, xa);
+            tmem_wait_ld();
+            if (mine && add) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(orow + 8 * q));
@@ -755,11 +757,15 @@ __device__ __forceinline__ void chain_role(const Ctx &x, const TcParams &p, int 
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const float2 f = __bfloat1622float2(h2[u]);
-                        r4[u] = pack_bf16(f.x + xv[8 * q + 2 * u], f.y + xv[8 * q + 2 * u + 1]);
+                        r4[u] = pack_bf16(f.x + xa[8 * q + 2 * u], f.y + xa[8 * q + 2 * u + 1]);
                     }
                     *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(r4[0], r4[1], r4[2], r4[3]);
                 }
             }
+        } else if (mine && first) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
         tc_fence_before();
         PROF_MARK(25);

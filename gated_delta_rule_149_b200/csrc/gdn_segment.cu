@@ -37,6 +37,15 @@ namespace {
 
 constexpr int kDKs = 128;   // the chunkwise kernel's key size
 
+// SMs of the current device (grid-stride helper kernels launch one block per SM)
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;   // a launch error, if any, surfaces at the launch itself
+    return n;
+}
+
 __global__ void identity_fill_kernel(float *out, size_t n_mats)
 {
     const size_t n = n_mats * kDKs * kDKs;
@@ -186,7 +195,7 @@ cudaError_t launch_segmented(const FwdArgs &a, int n_segments, cudaStream_t stre
     if (err == cudaSuccess) err = cudaStreamWaitEvent(side->s, side->fork, 0);
     if (err == cudaSuccess) err = cudaMemsetAsync(Vz, 0, BH * (size_t)a.T * a.dk * 2, side->s);
     if (err == cudaSuccess) {
-        identity_fill_kernel<<<148, 256, 0, side->s>>>(Pin, nP);
+        identity_fill_kernel<<<sm_count(), 256, 0, side->s>>>(Pin, nP);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }
@@ -301,7 +310,7 @@ cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream)
     if (err == cudaSuccess) err = cudaStreamWaitEvent(side->s, side->fork, 0);
     if (err == cudaSuccess) err = cudaMemsetAsync(Vz, 0, ntok * a.dk * 2, side->s);
     if (err == cudaSuccess) {
-        identity_fill_kernel<<<148, 256, 0, side->s>>>(Pin, BHF);
+        identity_fill_kernel<<<sm_count(), 256, 0, side->s>>>(Pin, BHF);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }
@@ -343,7 +352,7 @@ cudaError_t launch_blockcausal(const FwdArgs &a, int block, cudaStream_t stream)
     // read-out with identity tokens
     if (err == cudaSuccess) err = cudaMemsetAsync(Zb, 0, ntok * 4, stream);
     if (err == cudaSuccess) {
-        fill_kernel<<<148, 256, 0, stream>>>(On, ntok, 1.f);
+        fill_kernel<<<sm_count(), 256, 0, stream>>>(On, ntok, 1.f);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }
@@ -384,19 +393,20 @@ __global__ void fill_bf16_kernel(__nv_bfloat16 *out, size_t n, float value)
 }
 
 // every column of the [rows][64] output is z_in[row]
-__global__ void broadcast_cols_kernel(float *out, const float *z, size_t rows)
+__global__ void broadcast_cols_kernel(float *out, const float *z, size_t rows, int width)
 {
-    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < rows * 64; e += (size_t)gridDim.x * blockDim.x)
-        out[e] = z[e / 64];
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < rows * width; e += (size_t)gridDim.x * blockDim.x)
+        out[e] = z[e / width];
 }
 
 // o[row][c] /= (den[row][0] + eps), 8 bf16 values per thread step
-__global__ void divide_rows_kernel(__nv_bfloat16 *o, const __nv_bfloat16 *den, size_t rows, int dv, float eps)
+__global__ void divide_rows_kernel(__nv_bfloat16 *o, const __nv_bfloat16 *den, size_t rows, int dv, int den_width,
+                                   float eps)
 {
     const int per = dv / 8;
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < rows * per; e += (size_t)gridDim.x * blockDim.x) {
         const size_t row = e / per;
-        const float inv = 1.f / (__bfloat162float(den[row * 64]) + eps);
+        const float inv = 1.f / (__bfloat162float(den[row * den_width]) + eps);
         uint4 w = *reinterpret_cast<const uint4 *>(o + e * 8);
         __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&w);
 #pragma unroll
@@ -414,8 +424,13 @@ cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *
                               cudaStream_t stream)
 {
     const size_t BH = (size_t)a.B * a.H, ntok = BH * (size_t)a.T, ndir = a.bidi ? 2 : 1;
-    const size_t b_ones = align_up(ntok * 64 * 2), b_den = b_ones;
-    const size_t b_zin = align_up(BH * a.dk * 64 * 4), b_zout = align_up(ndir * BH * a.dk * 64 * 4);
+    // the value of ones: 128 wide when the pooled kernel can run the pass (it
+    // serves dv = 128 only; every column then carries the same z), else 64
+    FwdArgs az = a;
+    az.dv = 128;
+    const int zw = chunk_pool_supported(az) ? 128 : 64;
+    const size_t b_ones = align_up(ntok * zw * 2), b_den = b_ones;
+    const size_t b_zin = align_up(BH * a.dk * zw * 4), b_zout = align_up(ndir * BH * a.dk * zw * 4);
     uint8_t *ws = nullptr;
     cudaError_t err = ws_alloc(reinterpret_cast<void **>(&ws), b_ones + b_den + b_zin + b_zout, stream);
     if (err != cudaSuccess) return err;
@@ -424,11 +439,13 @@ cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *
     float *zin = reinterpret_cast<float *>(ws + b_ones + b_den);
     float *zout = reinterpret_cast<float *>(ws + b_ones + b_den + b_zin);
 
-    // causal: the denominator pass runs beside the numerator pass on a second
-    // stream.  Bidirectional: after it, on the caller's stream (a bidirectional
-    // launch counts on having every one of its CTAs resident at once).
-    int dev = 0;
+    // causal: the denominator pass is enqueued beside the numerator pass on a
+    // second stream (they overlap as far as their grids leave SMs free; two
+    // pooled launches each take every SM and run one after the other).
+    // Bidirectional: after it, on the caller's stream.
+    int dev = 0, sms = 0;
     err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     std::lock_guard<std::mutex> lock(g_side_mu);
     SideStream *side = nullptr;
     if (err == cudaSuccess && !a.bidi) err = side_stream(dev, &side);
@@ -440,19 +457,18 @@ cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *
     }
     if (err == cudaSuccess && a.bidi) err = launch_chunk_tc(a, stream);   // numerator first
     if (err == cudaSuccess) {
-        fill_bf16_kernel<<<148, 256, 0, ds>>>(ones, ntok * 64, 1.f);
+        fill_bf16_kernel<<<sms, 256, 0, ds>>>(ones, ntok * zw, 1.f);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }
     if (err == cudaSuccess && state_z_in) {
-        broadcast_cols_kernel<<<148, 256, 0, ds>>>(zin, state_z_in, BH * a.dk);
+        broadcast_cols_kernel<<<sms, 256, 0, ds>>>(zin, state_z_in, BH * a.dk, zw);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }
     if (err == cudaSuccess) {
-        FwdArgs az = a;
         az.v = ones;
-        az.dv = 64;
+        az.dv = zw;
         az.o = den;
         az.state_in = state_z_in ? zin : nullptr;
         az.state_out = state_z_out ? zout : nullptr;
@@ -468,13 +484,13 @@ cudaError_t launch_normalized(const FwdArgs &a, const float *state_z_in, float *
         }
     }
     if (err == cudaSuccess) {
-        divide_rows_kernel<<<592, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(a.o), den, ntok, a.dv, eps);
+        divide_rows_kernel<<<sms * 4, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(a.o), den, ntok, a.dv, zw, eps);
         err = cudaGetLastError();
         if (err == cudaSuccess) count_launches(1);
     }
-    // z out: column 0 of every [dk][64] state
+    // z out: column 0 of every [dk][zw] state
     if (err == cudaSuccess && state_z_out)
-        err = cudaMemcpy2DAsync(state_z_out, 4, zout, 64 * 4, 4, ndir * BH * a.dk, cudaMemcpyDeviceToDevice, stream);
+        err = cudaMemcpy2DAsync(state_z_out, 4, zout, zw * 4, 4, ndir * BH * a.dk, cudaMemcpyDeviceToDevice, stream);
     const cudaError_t e2 = ws_free(ws, stream);
     return err != cudaSuccess ? err : e2;
 }
