@@ -97,12 +97,14 @@ def workload_config(wl, world):
             "parallelism": f"replicas x{world} (independent scans, no collective)"}
 
 
-def kernel_source_sha():
-    """Hash of the chunkwise kernel's device code (its source and the PTX
-    wrappers it includes; comments and whitespace removed), so that a recorded
-    traffic figure stays tied to the kernel it was taken on."""
+def kernel_source_sha(kernel="pool"):
+    """Hash of the main kernel's device code (its source and the headers it
+    includes; comments and whitespace removed), so that a recorded traffic
+    figure stays tied to the kernel it was taken on.  kernel: "pool" (the pooled
+    kernel, dk = dv = 128) or "single" (the single-CTA kernel)."""
     h = hashlib.sha256()
-    for name in ("gdn_chunk_pool.cu", "gdn_chunk_tc.cu", "gdn_chunk_common.cuh", "sm100_ptx.cuh"):
+    main = "gdn_chunk_pool.cu" if kernel == "pool" else "gdn_chunk_tc.cu"
+    for name in (main, "gdn_chunk_common.cuh", "sm100_ptx.cuh"):
         p = os.path.join(ROOT, "gated_delta_rule_149_b200", "csrc", name)
         if os.path.exists(p):
             src = open(p).read()
@@ -529,7 +531,7 @@ def run_gpu(args, world, rank, local):
     hbm_peak, tc_peak, peak_kind = load_peaks()
     call_s = statistics.mean(per_call) * 1e-3
     achieved = bytes_ / call_s / 1e9
-    sha = kernel_source_sha()
+    sha = kernel_source_sha("single" if args.kernel == "single" or wl.dv != 128 or recurrent else "pool")
     traffic = recorded_traffic(wl.name, sha)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": traffic,
