@@ -45,6 +45,9 @@
 // to it and rounds once, after an arrival counter shows the first is visible
 // (the forward scan writes first in the first half of the sequence).  The
 // launch is cooperative: every CTA is resident, or the launch is refused.
+// fp8 inputs (the FP8 instantiation): q, k, v arrive as E4M3 codes with one
+// scale per head; workers form [Q;K] K^T on the codes (kind::f8f6f4) and widen
+// only k to bf16, chains widen v and k; every other product is the bf16 one.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -1419,9 +1422,9 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream, const float
 // gdn_debug_ring: a device buffer of at least dirs*B*H*8*49664 bytes that the
 // pooled kernel uses as its operand ring instead of workspace (NULL: off), so a
 // test can read back the prepared operands of each scan's last eight chunks.
-// gdn_debug_kernel_select: 0 or 2 pick the kernel by shape (the pooled kernel
-// for dk = dv = 128 whole sequences), 1 forces the single-CTA chunkwise kernel
-// for every bf16 call.
+// gdn_debug_kernel_select: 0 picks the kernel by shape (the pooled kernel for
+// dk = dv = 128 whole sequences), 1 forces the single-CTA chunkwise kernel for
+// every bf16 call.
 // gdn_debug_stall: chunk c >= 0 makes scan 0's chain of the pooled kernel wait
 // for chunk c's operands with a target nothing reaches, so the wait runs out
 // (with a lowered limit, see gdn_debug_wait_limit) and the call ends with

@@ -379,9 +379,9 @@ def gdn_workspace_reserved(device=None):
 
 
 def debug_kernel_select(which):
-    """Test hook: 0 (or 2) picks the bf16 chunkwise kernel by shape (the pooled
-    kernel for dk = dv = 128 whole-sequence calls), 1 forces the single-CTA
-    chunkwise kernel for every bf16 call (for A/B comparisons of the two)."""
+    """Test hook: 0 picks the bf16 chunkwise kernel by shape (the pooled kernel
+    for dk = dv = 128 whole-sequence calls), 1 forces the single-CTA chunkwise
+    kernel for every bf16 call (for A/B comparisons of the two)."""
     load_library().gdn_debug_kernel_select(int(which))
 
 

@@ -15,9 +15,9 @@ extern "C" {
 
 /*
  * gdn_debug_kernel_select -- which chunkwise kernel bf16 calls use: 0 (default)
- * or 2 choose by shape (the pooled kernel for whole sequences with
- * dk = dv = 128, the single-CTA kernel otherwise); 1 forces the single-CTA
- * kernel for every bf16 call.
+ * chooses by shape (the pooled kernel for whole sequences with dk = dv = 128,
+ * the single-CTA kernel otherwise); 1 forces the single-CTA kernel for every
+ * bf16 call.  Other values act as 0.
  */
 void gdn_debug_kernel_select(int which);
 
