@@ -67,3 +67,18 @@ def test_fp8_and_frame_block_forms(oracle_mod):
     args = argparse.Namespace(normalized=False, block=40)
     r = bench.sampled_parity(args, inp.wl, inp, torch.from_numpy(o_ref).float(), torch.from_numpy(s_ref).float())
     assert r["pass"], r
+
+
+def test_algorithmic_bytes_and_source_hash():
+    import bench
+    from gated_delta_rule_149_b200.inputs import WORKLOADS
+    wl = WORKLOADS["bidi_720p"]
+    b16, b8 = bench.algorithmic_bytes(wl), bench.algorithmic_bytes(wl, fp8=True)
+    # bf16: 2 directions x ((2 dk + dv) x 2 B + 8 B of gates) + dv x 2 B of o, per token-head, plus states
+    states = wl.B * wl.H * wl.dk * wl.dv * 4 * 2
+    assert b16 == wl.B * wl.H * wl.T * (2 * ((2 * 128 + 128) * 2 + 8) + 128 * 2) + states
+    # fp8 codes: q, k, v at one byte, o still bf16
+    assert b16 - b8 == wl.B * wl.H * wl.T * 2 * (2 * 128 + 128)
+    # the hash covers the kernel that ran, and ignores comments
+    assert bench.kernel_source_sha("pool") != bench.kernel_source_sha("single")
+    assert bench.kernel_source_sha("pool") == bench.kernel_source_sha("pool")
