@@ -4,7 +4,8 @@
    state chain of the pooled kernel told to wait for a slot sequence value
    nothing writes, the kernel records a timeout in the device error word and
    returns (no hang); gdn_device_status reports GDN_ERR_DEVICE_TIMEOUT, and the
-   next normal call on the same context matches the oracle.
+   next normal call on the same context matches the oracle.  Causal and
+   bidirectional bf16 calls, and a causal fp8 call (the fp8 instantiation).
 2. Co-residency: the kernels whose CTAs wait for one another are launched
    cooperatively, so a call made while another stream keeps every SM busy with
    matrix products still finishes correctly (no wait runs out), and so do the
@@ -15,9 +16,9 @@ import time
 import pytest
 import torch
 
-from gated_delta_rule_149_b200 import gdn, gdn_device_status, gdn_forward
+from gated_delta_rule_149_b200 import gdn, gdn_device_status, gdn_forward, gdn_forward_fp8
 from gated_delta_rule_149_b200.gdn import GDNError
-from gated_delta_rule_149_b200.inputs import make_custom
+from gated_delta_rule_149_b200.inputs import make_custom, quantize_e4m3
 from parity_util import TOL, f64, oracle_forward, rel_l2, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -32,8 +33,8 @@ def _check_parity(oracle_mod, inp, bidi, o, s):
     assert e_s <= TOL["bf16"], f"state rel-L2 {e_s:.3e}"
 
 
-@pytest.mark.parametrize("bidi", [False, True])
-def test_wait_runs_out_and_the_next_call_is_correct(oracle_mod, bidi):
+@pytest.mark.parametrize("bidi,fp8", [(False, False), (True, False), (False, True)])
+def test_wait_runs_out_and_the_next_call_is_correct(oracle_mod, bidi, fp8):
     torch.cuda.set_device(0)
     inp = make_custom(1, 2, 1024, 128, 128, dtype="bf16", seed=31, bidi=bidi, state0=True)
     d = to_dev(inp)
@@ -42,7 +43,12 @@ def test_wait_runs_out_and_the_next_call_is_correct(oracle_mod, bidi):
     gdn.debug_stall(3)
     try:
         t0 = time.perf_counter()
-        gdn_forward(d["q"], d["k"], d["v"], d["beta"], d["decay"], d["state0"], bidi=bidi)
+        if fp8:   # the fp8 instantiation (its code widening runs in both CTA kinds)
+            codes = [quantize_e4m3(x) for x in (inp.q, inp.k, inp.v)]
+            gdn_forward_fp8(*(c.cuda() for c, _ in codes), *(sc.cuda() for _, sc in codes), d["beta"],
+                            d["decay"], d["state0"])
+        else:
+            gdn_forward(d["q"], d["k"], d["v"], d["beta"], d["decay"], d["state0"], bidi=bidi)
         with pytest.raises(GDNError) as err:
             gdn_device_status()
         elapsed = time.perf_counter() - t0
