@@ -27,8 +27,8 @@ Also measured, and printed on the same JSON line:
                (rank 0, N = 1 only);
   clocks       SM clock and throttle reasons sampled (NVML) during the timed
                region.
---impl reference times the CPU oracle alone (the reference arm of this build:
-there is no upstream code to run).
+--impl reference times the CPU oracle alone (the reference arm: there is no
+upstream code to run).
 """
 import argparse
 import hashlib

@@ -9,8 +9,8 @@
  * Definition followed.  The librediffusion PR #21 page ("What's added") names
  * the operation -- a GDN (Gated-Delta-Net) linear-attention recurrence kernel
  * -- but none of the pages prints its formula.  The update below is the gated
- * delta rule as the task defines it (the standard Gated DeltaNet recurrence),
- * per head, with S a dv x dk matrix:
+ * delta rule (the standard Gated DeltaNet recurrence), per head, with S a
+ * dv x dk matrix:
  *
  *     S_t = a_t * S_{t-1} * (I - b_t k_t k_t^T) + b_t v_t k_t^T
  *     o_t = S_t q_t

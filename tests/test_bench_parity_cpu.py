@@ -57,7 +57,7 @@ def test_fp8_and_frame_block_forms(oracle_mod):
     r = bench.sampled_parity(args, inp.wl, inp, torch.from_numpy(o_ref).float(), torch.from_numpy(s_ref).float(),
                              fp8=(q8, k8, v8, sq, sk, sv))
     assert r["pass"] and r["rel_l2_o"] < 1e-6, r
-    # the same result judged as a plain bf16 call fails: the check uses the fp8 definition
+    # the same result checked as a plain bf16 call fails: the check uses the fp8 definition
     assert bench.sampled_parity(args, inp.wl, inp, torch.from_numpy(o_ref).float(),
                                 torch.from_numpy(s_ref).float())["rel_l2_o"] > 1e-3
 
