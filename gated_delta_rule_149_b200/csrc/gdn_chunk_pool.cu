@@ -11,27 +11,25 @@
 // order, with g = log2 a, G_i = sum of g up to and including token i,
 // gamma_i = 2^G_i, e_i = 2^(G_end - G_i):
 //     A  = strict-lower [ b_i 2^(G_i - G_j) k_i.k_j ],  P = lower [ 2^(G_i - G_j) q_i.k_j ]
-//     T  = (I + A)^-1,  T1 = T diag(b gamma),  T2 = T diag(b)
-//     U  = T2 V - T1 K H_prev                      (the delta-rule values)
-//     O  = diag(gamma) Q H_prev + P U              (the outputs)
-//     H  = gamma_end H_prev + K^T diag(e) U        (the next state)
-// Substituting U into O gives both from one product with the previous state:
-//     [O; U] = [P T2; T2] V + [Q'; -W] H_prev,   Q' = diag(gamma) Q - P T1 K,  W = T1 K,
-// so everything except that product and the state update is independent of
-// the state: a chunk's operands A1 = [P T2; T2] (128 x 64) and
-// A2 = [Q'; -W] (128 x dk) can be formed by any SM, ahead of the chain.
+//     T  = (I + A)^-1,  T1 = T diag(b gamma),  T2 = T diag(b),  W = T1 K
+//     U  = T2 V - W H_prev                          (the delta-rule values)
+//     O  = diag(gamma) Q H_prev + P U               (the outputs)
+//     H  = gamma_end H_prev + K^T diag(e) U         (the next state)
+// P, T2 and W do not depend on the state: any SM can form them ahead of the
+// chain, which is left with the products against the state.
 //
 // Roles (CTA = blockIdx.x):
-//   CTA < n_scans, chain of scan CTA: loads V, K and the scan's prepared
+//   CTA < n_scans, chain of scan CTA: loads V, K, Q and the scan's prepared
 //       operands of each chunk, and runs
-//           D = V^T A1^T + H^T A2^T   (M = dv = 128, N = 128: O^T and U^T)
-//           S = Ubar^T K              (Ubar = diag(e) U; M = dv, N = dk)
-//           H^T <- gamma_end H^T + S  (fp32 in registers)
-//       with H^T and Ubar^T as bf16 A operands in TMEM, and writes O.
+//           U^T = V^T T2^T - H^T W^T     (M = dv = 128, N = 64)
+//           S = Ubar^T K                 (Ubar = diag(e) U; M = dv, N = dk)
+//           H^T <- gamma_end H^T + S     (fp32 in registers)
+//           O^T = H^T Q'^T + U^T P^T     (Q' = diag(gamma) Q; off the state's path)
+//       with H^T, Ubar^T and U^T as bf16 A operands in TMEM, and writes O.
 //   CTA >= n_scans, worker: takes (scan, chunk) items from a global counter in
-//       chunk-major order and prepares them: gates, the masks of [Q;K] K^T,
-//       the 64 x 64 solve, the products P [T1 | T2] and [P T1; T1] K and their
-//       epilogues (tcgen05 MMAs, fp32 accumulators in TMEM); writes A1, A2, e
+//       chunk-major order and prepares them: gates, the masks of [Q;K] K^T
+//       (P and A), the 64 x 64 solve, W^T = K^T T1^T and its epilogue
+//       (tcgen05 MMAs, fp32 accumulators in TMEM); writes P, T2, -W^T, e, gamma
 //       and gamma_end into the scan's ring of slots in global memory (a few
 //       chunks per scan, so it stays in L2).
 // A preparation is a long chain of dependent steps, independent from chunk to
@@ -47,7 +45,7 @@
 // launch is cooperative: every CTA is resident, or the launch is refused.
 // fp8 inputs (the FP8 instantiation): q, k, v arrive as E4M3 codes with one
 // scale per head; workers form [Q;K] K^T on the codes (kind::f8f6f4) and widen
-// only k to bf16, chains widen v and k; every other product is the bf16 one.
+// only k to bf16, chains widen v, k and q; every other product is the bf16 one.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -76,9 +74,9 @@ bool g_plain_launch = false;
 namespace {
 
 // 16 warps: TMA, MMA, group A (8 warps: two per TMEM lane quarter), group B
-// (4 warps: one per quarter), 2 gate warps (workers).  Four warps per SM
-// sub-partition leave 128 registers a thread (a chain's state threads hold 64
-// fp32 values).
+// (4 warps: one per quarter), 2 gate warps (workers) or converters (chains).
+// Four warps per SM sub-partition leave 128 registers a thread (a chain's
+// state threads hold 64 fp32 values).
 constexpr int kThreads = 512;
 constexpr int kGroup = 256, kGroupB = 128;
 constexpr int kBarA = 1, kBarB = 2, kBarGate = 3, kBarConv = 4;   // named barriers
@@ -93,41 +91,46 @@ constexpr int kNSlot = 8;                 // ring slots per scan
 constexpr int kFlagStride = 32;
 static_assert(kNSlot <= kFlagStride, "a scan's slot words share its line");
 
-// ring slot: A1 [128 rows x 64] bf16, A2 [kb][128 rows x 64] bf16 (both 128B-swizzled
-// images), then e[64] and gamma_end (fp32)
-constexpr uint32_t kSlotA1 = 0, kSlotA2 = 16384, kSlotGates = 49152, kSlotBytes = 49664;
+// ring slot: P [64 x 64] and T2 [64 x 64] bf16 (128B-swizzled, token rows),
+// -W^T [128 keys x 64 tokens] bf16 (128B-swizzled), then the gate block (fp32):
+// e[64], gamma_end, 3 unused, gamma[64]
+constexpr uint32_t kSlotP = 0, kSlotT2 = 8192, kSlotW = 16384, kSlotGates = 32768;
+constexpr uint32_t kGateBlockBytes = 528, kSlotCopy = kSlotGates + kGateBlockBytes, kSlotBytes = 33792;
+constexpr int kGamOff = 68;               // gamma's first float in the gate block
 
 // shared memory (from a 1024-aligned base)
 constexpr uint32_t kOffBar = 0;
 // worker
 constexpr uint32_t kWStage = 1024;                        // kNS x [kb0: Q|K][kb1: Q|K]
 constexpr uint32_t kWStageBytes = 32768;
-constexpr uint32_t kPP = kWStage + kNS * kWStageBytes;    // 8 KB P
-constexpr uint32_t kPTB = kPP + 8192;                     // 2 x [PT1 | T1 | PT2 | T2], 8 KB each
-constexpr uint32_t kPA2 = kPTB + 65536;                   // A2 staging [kb][128 rows]
-constexpr uint32_t kPA = kPA2 + 32768;                    // fp32 [64][kLDA] solve buffer
+constexpr uint32_t kPTB = kWStage + kNS * kWStageBytes;   // 2 x [P | T1 | T2], 8 KB each
+constexpr uint32_t kTBBytes = 24576;
+constexpr uint32_t kPW = kPTB + 2 * kTBBytes;             // -W^T staging [128 keys][64 tokens]
+constexpr uint32_t kPA = kPW + 16384;                     // fp32 [64][kLDA] solve buffer
 constexpr uint32_t kPGates = kPA + 64 * kLDA * 4;
-constexpr uint32_t kPGst = kPGates + kNG * kGateFloats * 4;   // 512 B: e, gamma_end of the slot
-constexpr uint32_t kPEnd = kPGst + 512;
+constexpr uint32_t kPGst = kPGates + kNG * kGateFloats * 4;   // the slot's gate block
+constexpr uint32_t kPEnd = kPGst + 1024;
 // chain
-constexpr int kNVK = 2;                                   // V/K stages
-constexpr uint32_t kCStage = 1024;                        // kNVK x [V0 | V1 | K0 | K1]
-constexpr uint32_t kCA = kCStage + kNVK * 32768;          // 2 ring-slot images
-constexpr uint32_t kCABytes = 50176;
+constexpr int kNVK = 2;                                   // V/K/Q stages
+constexpr uint32_t kCStage = 1024;                        // kNVK x [V0 | V1 | K0 | K1 | Q0 | Q1]
+constexpr uint32_t kCStageBytes = 49152;
+constexpr uint32_t kCA = kCStage + kNVK * kCStageBytes;   // 2 ring-slot images
+constexpr uint32_t kCABytes = kSlotBytes;
 constexpr uint32_t kCO = kCA + 2 * kCABytes;              // 2 output tiles [dv block][64 tokens][64]
 constexpr uint32_t kCEnd = kCO + 2 * 16384;
-constexpr uint32_t kC8 = kCEnd;                           // fp8 inputs: staging of one chunk's v, k codes
-constexpr uint32_t kCEnd8 = kC8 + 16384;
+constexpr uint32_t kC8 = kCEnd;                           // fp8 inputs: staging of one chunk's v, k, q codes
+constexpr uint32_t kCEnd8 = kC8 + 24576;
 constexpr uint32_t kSmemBytes = (kPEnd > kCEnd8 ? kPEnd : kCEnd8);
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
-static_assert(kPP % 1024 == 0 && kPTB % 1024 == 0 && kPA2 % 1024 == 0 && kCA % 1024 == 0 &&
-              kCABytes % 1024 == 0 && kCO % 1024 == 0 && kC8 % 1024 == 0 && kPGst % 16 == 0,
+static_assert(kPTB % 1024 == 0 && kTBBytes % 1024 == 0 && kPW % 1024 == 0 && kCA % 1024 == 0 &&
+              kCABytes % 1024 == 0 && kCO % 1024 == 0 && kC8 % 1024 == 0 && kPGst % 16 == 0 &&
+              kSlotCopy % 16 == 0 && kSlotCopy <= kSlotBytes,
               "tile alignment");
 
 // TMEM columns
-constexpr uint32_t kTD1 = 0, kTD2 = 128, kTD3 = 256;                 // worker
-constexpr uint32_t kTD = 0, kTS = 256, kTH = 384, kTUb = 448;         // chain
+constexpr uint32_t kTD1 = 0, kTD3 = 256;                             // worker
+constexpr uint32_t kTD = 0, kTS = 256, kTH = 384, kTUb = 448, kTUr = 480;   // chain: kTD = 2 x [O^T | U^T]
 constexpr uint32_t kTmemCols = 512;
 
 // Chunk-0 products of scan 0 can be dumped for debugging in builds with
@@ -140,10 +143,10 @@ constexpr bool kDbgOn = false;
 
 constexpr uint32_t kIdM1 = idesc_bf16(128, 64, false, false);   // [Q;K] K^T
 constexpr uint32_t kIdM1f8 = idesc_e4m3(128, 64, false, false); // [Q;K] K^T on E4M3 codes
-constexpr uint32_t kIdM2 = idesc_bf16(64, 128, false, true);    // P [T1 | T2]
-constexpr uint32_t kIdM3 = idesc_bf16(128, 128, false, true);   // [P T1; T1] K
-constexpr uint32_t kIdA = idesc_bf16(128, 128, true, false);    // V^T A1^T
-constexpr uint32_t kIdB = idesc_bf16(128, 128, false, false);   // H^T A2^T (A in TMEM)
+constexpr uint32_t kIdW = idesc_bf16(128, 64, true, false);     // K^T T1^T (A = K MN-major)
+constexpr uint32_t kIdU1 = idesc_bf16(128, 64, true, false);    // V^T T2^T (A = V MN-major)
+constexpr uint32_t kIdU2 = idesc_bf16(128, 64, false, true);    // H^T (-W^T) (A in TMEM, B MN-major)
+constexpr uint32_t kIdO = idesc_bf16(128, 64, false, false);    // H^T Q'^T, U^T P^T (A in TMEM)
 constexpr uint32_t kIdC = idesc_bf16(128, 128, false, true);    // Ubar^T K (A in TMEM)
 
 struct PoolParams {
@@ -169,14 +172,15 @@ struct PoolParams {
 
 struct Bars {
     // worker
-    uint64_t it_full[kNS], st_full[kNS], st_empty[kNS], d1_full[2], d1_empty[2], tp_full[2], p_free, t_free[2];
-    uint64_t d2_full, d2_empty, e2_done, d3_full, d3_empty;
+    uint64_t it_full[kNS], st_full[kNS], st_empty[kNS], d1_full[2], d1_empty[2], tp_full[2], t_free[2];
+    uint64_t d3_full, d3_empty;
     uint64_t g_full[kNG], g_empty[kNG];
-    uint64_t cv_full[kNS];             // fp8: the stage's q, k tiles converted to bf16
+    uint64_t cv_full[kNS];             // fp8: the stage's k tile widened to bf16
     // chain
-    uint64_t vk_full[kNVK], vk_empty[kNVK], a_full[2], a_empty[2], d_full[2], d_empty[2], o_full[2];
+    uint64_t vk_full[kNVK], vk_empty[kNVK], q_full[kNVK], a_full[2], a_empty[2];
+    uint64_t du_full[2], do_full[2], d_empty[2], o_full[2];
     uint64_t u_full, s_full, h_full;
-    uint64_t s8_full, s8_empty;        // fp8: the v, k code staging
+    uint64_t s8_full, s8_empty;        // fp8: the v, k, q code staging
     uint64_t drain;
     float gscal[kNG][2];   // per gate buffer: G_end, factorised (1) or not (0)
     int gitem[kNG];        // per gate buffer: the item, or -1 after the last
@@ -292,27 +296,12 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &c, float scale, uin
         }
 }
 
-// 16 codes times `scale`, as fp32
-__device__ __forceinline__ void e4m3x16_to_f32(const uint4 &c, float scale, float (&f)[16])
-{
-    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const __half2_raw hr =
-                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(words[i] >> (16 * h)), __NV_E4M3);
-            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
-            f[4 * i + 2 * h] = v.x * scale;
-            f[4 * i + 2 * h + 1] = v.y * scale;
-        }
-}
-
 // Thread t (of 64) takes the 16-code chunk t % 8 of rows t / 8 + 8 n.  Every
 // thread reads its chunks before the group's barrier and writes after it, so
-// a destination may overlap the source.
+// a destination may overlap the source.  row_scale (optional): a factor per
+// row, applied with scale.
 __device__ __forceinline__ void e4m3_tile_to_bf16(const uint8_t *src, uint8_t *dst0, uint8_t *dst1, float scale,
-                                                  int t, int bar_id)
+                                                  int t, int bar_id, const float *row_scale = nullptr)
 {
     const int j = t & 7, r0 = t >> 3, ph = r0 & 7;   // rows r0 + 8 n share the swizzle phase
     uint4 c[8];
@@ -325,10 +314,34 @@ __device__ __forceinline__ void e4m3_tile_to_bf16(const uint8_t *src, uint8_t *d
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
         uint32_t w[8];
-        e4m3x16_to_bf16(c[n], scale, w);
+        e4m3x16_to_bf16(c[n], row_scale ? scale * row_scale[r0 + 8 * n] : scale, w);
         uint8_t *row = d + (r0 + 8 * n) * 128;
         *reinterpret_cast<uint4 *>(row + o0) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4 *>(row + o1) = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
+
+// Row r of a [64 tokens][128] bf16 tile held as two 128B-swizzled 64-column
+// blocks 8 KB apart, times g, in place (one rounding).  The row's 16-byte
+// chunks are visited in swizzle order, so 8 consecutive rows take 8 different
+// bank groups.
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t w, float g)
+{
+    return pack_bf16(__uint_as_float(w << 16) * g, __uint_as_float(w & 0xffff0000u) * g);
+}
+__device__ __forceinline__ void scale_row_bf16(uint8_t *tile, int r, float g)
+{
+    uint4 w[16];   // every chunk loaded before the first store
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+        w[m] = *reinterpret_cast<const uint4 *>(tile + (m >> 3) * 8192 + r * 128 + (((m & 7) ^ (r & 7)) << 4));
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        w[m].x = scale_bf16x2(w[m].x, g);
+        w[m].y = scale_bf16x2(w[m].y, g);
+        w[m].z = scale_bf16x2(w[m].z, g);
+        w[m].w = scale_bf16x2(w[m].w, g);
+        *reinterpret_cast<uint4 *>(tile + (m >> 3) * 8192 + r * 128 + (((m & 7) ^ (r & 7)) << 4)) = w[m];
     }
 }
 
@@ -469,10 +482,10 @@ __device__ __forceinline__ void worker_gates(const Ctx &x, const PoolParams &p, 
     }
 }
 
-// MMA issue, per item j: P [T1 | T2] of item j, then [Q;K] K^T of item j + 2 (its
-// D1 buffer is free once item j's masks are read, which P [T1 | T2] follows),
-// then [P T1; T1] K of item j (after the finisher has read P [T1 | T2]).  The
-// [Q;K] K^T products run two items ahead of the solver.
+// MMA issue, per item j: W^T = K^T T1^T of item j once its solve is done,
+// with [Q;K] K^T of item j + 2 beside it (its D1 buffer is free once item j's
+// masks are read, which the solve follows).  The [Q;K] K^T products run two
+// items ahead of the solver.
 // [Q;K] K^T of item i (one thread; out of line, as it is issued from several
 // places): 1 issued, 0 no such item (the end), -1 inputs not ready yet (only
 // when !block), -2 abort.
@@ -524,29 +537,20 @@ __device__ __forceinline__ void worker_mma(const Ctx &x, const PoolParams &p)
     for (int j = 0; ok && (last < 0 || j < last); ++j) {
         const int bj = j & 1;
         if (!wait_bar(&B.tp_full[bj], (j >> 1) & 1, x.abort_flag, p.err, 6)) break;
-        if (j >= 1 && !wait_bar(&B.d2_empty, (j - 1) & 1, x.abort_flag, p.err, 7)) break;
-        const uint32_t tb = x.sbase + kPTB + bj * 32768;
-        tc_fence_after();
-        // P [T1 | T2]: B is MN-major, the T1 and T2 tiles are its two 64-column groups
-        mma_run<4, 2, 128>(tm + kTD2, sw128_desc(x.sbase + kPP, 16, 1024),
-                           sw128_desc(tb + 8192, 16384, 1024), kIdM2, false);
-        mma_commit(&B.d2_full);
-        mma_commit(&B.p_free);
-        tr(p, 0, 17, j);
-        // item j + 2's [Q;K] K^T now if its tiles are in, else after [P T1; T1] K
+        // item j + 2's [Q;K] K^T now if its tiles are in, else after W^T
         if (next == j + 2 && !step_m1(false)) break;
-        if (!wait_bar(&B.e2_done, j & 1, x.abort_flag, p.err, 8)) break;
         if (j >= 1 && !wait_bar(&B.d3_empty, (j - 1) & 1, x.abort_flag, p.err, 9)) break;
         // fp8: K widened to bf16 by the gate warps
         if (FP8 && !wait_bar(&B.cv_full[j % kNS], (j / kNS) & 1, x.abort_flag, p.err, 41)) break;
         tc_fence_after();
-        // [P T1; T1] K: B = K [token][dk] MN-major, dk groups 16 KB apart in the
-        // stage (fp8: 8 KB apart, beside the codes)
+        // W^T = K^T T1^T: A = K [token][dk] MN-major, dk groups 16 KB apart in the
+        // stage (fp8: 8 KB apart, beside the codes); B = T1 (K-major)
         {
             const uint32_t st = x.sbase + kWStage + (j % kNS) * kWStageBytes;
-            mma_run<4, 2, 128>(tm + kTD3, sw128_desc(tb, 16, 1024),
-                               FP8 ? sw128_desc(st + 16384, 8192, 1024) : sw128_desc(st + 8192, 16384, 1024), kIdM3,
-                               false);
+            const uint32_t tb = x.sbase + kPTB + bj * kTBBytes;
+            mma_run<4, 128, 2>(tm + kTD3,
+                               FP8 ? sw128_desc(st + 16384, 8192, 1024) : sw128_desc(st + 8192, 16384, 1024),
+                               sw128_desc(tb + 8192, 16, 1024), kIdW, false);
         }
         mma_commit(&B.d3_full);
         mma_commit(&B.t_free[bj]);
@@ -618,7 +622,7 @@ __device__ __forceinline__ void worker_solver(const Ctx &x, const PoolParams &p,
     for (int i = 0;; ++i) {
         const int b = i & 1, gi = i % kNG;
         const float *gt = gates_buf(x, gi);
-        uint8_t *tb = x.smem + kPTB + b * 32768;
+        uint8_t *tb = x.smem + kPTB + b * kTBBytes;   // [P | T1 | T2]
         if (pt == 0) tr(p, 0, 0, i);
         wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 10);
         const int k = B.gitem[gi];
@@ -633,22 +637,19 @@ __device__ __forceinline__ void worker_solver(const Ctx &x, const PoolParams &p,
         }
         const bool fact = B.gscal[gi][1] != 0.f;
         wait_bar(&B.d1_full[b], (i >> 1) & 1, x.abort_flag, p.err, 11);
-        if (i >= 1) wait_bar(&B.p_free, (i - 1) & 1, x.abort_flag, p.err, 12);   // P of item i - 1 is read
+        // this buffer's P, T1, T2 must be done with (item i - 2: its W^T product and its ring copies)
+        if (i >= 2) wait_bar(&B.t_free[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 13);
         if (pt == 0) tr(p, 0, 1, i);
         tc_fence_after();
-        mask_rows(x.tmem + tm_lane + kTD1 + 64 * b + 32 * hf, gt, As, x.smem + kPP, qd, lane, hf, fact, dir, sc_p,
-                  sc_a);
+        mask_rows(x.tmem + tm_lane + kTD1 + 64 * b + 32 * hf, gt, As, tb, qd, lane, hf, fact, dir, sc_p, sc_a);
         tc_fence_before();
         fence_proxy_async_smem();
         if (named_bar_any(kBarA, kGroup, *x.abort_flag)) return;
         if (pt == 0) mbar_arrive(&B.d1_empty[b]);
         if (pt == 0) tr(p, 0, 2, i);
-        // T1 / T2 of this buffer must be done with (item i - 2: its products and its ring copy)
-        if (i >= 2) wait_bar(&B.t_free[b], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 13);
-        if (pt == 0) tr(p, 0, 3, i);
-        solve_diag_blocks<kBarA, kGroup>(As, gt, tb + 8192, tb + 24576, nullptr, dir, pt);
+        solve_diag_blocks<kBarA, kGroup>(As, gt, tb + 8192, tb + 16384, nullptr, dir, pt);
         if (pt == 0) tr(p, 0, 4, i);
-        solve_off_diag_strips(As, gt, tb + 8192, tb + 24576, dir, pt);
+        solve_off_diag_strips(As, gt, tb + 8192, tb + 16384, dir, pt);
         fence_proxy_async_smem();
         if (named_bar_any(kBarA, kGroup, *x.abort_flag)) return;
         if (pt == 0) mbar_arrive(&B.tp_full[b]);
@@ -657,8 +658,9 @@ __device__ __forceinline__ void worker_solver(const Ctx &x, const PoolParams &p,
 }
 
 // Finisher group (4 warps, warp w reads TMEM lane quarter qd = w % 4): per item,
-// P T1 and P T2 into the operand tiles, Q' = gamma Q - P T1 K and -W = -T1 K into
-// A2, then the item's slot in its scan's ring.
+// -W^T into its staging tile and the gate block, then the item's slot in its
+// scan's ring: P, T2, -W^T and the gate block by bulk copies, published to the
+// chain once they have completed (at the start of the next item).
 template <bool FP8>
 __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &p, int ft, int qd)
 {
@@ -666,18 +668,13 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
     const int lane = ft & 31;
     const uint32_t tm_lane = (uint32_t)(qd * 32) << 16;
     int pend_scan = -1, pend_c = 0, pend_b = -1;   // leader: the item whose ring copies are in flight
-    // leader: once the copies have read their sources, the A1 tile goes back to the
-    // solver and A2 staging is free again
-    auto release_sources = [&]() {
-        if (pend_b < 0) return;
-        bulk_wait_read0();
-        mbar_arrive(&B.t_free[pend_b]);
-        pend_b = -1;
-    };
-    // leader: once the copies have completed, the slot is published to the scan's chain
+    // leader: once the copies have read their sources, the P / T2 buffer goes back
+    // to the solver (the staging tiles are free); once they have completed, the
+    // slot is published to the scan's chain
     auto publish = [&]() {
         if (pend_scan < 0) return;
-        release_sources();
+        bulk_wait_read0();
+        mbar_arrive(&B.t_free[pend_b]);
         bulk_wait0();
         fence_proxy_async_global();
         __threadfence();
@@ -687,100 +684,40 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
 #pragma unroll 1
     for (int i = 0;; ++i) {
         const int b = i & 1, gi = i % kNG;
-        uint8_t *tb = x.smem + kPTB + b * 32768;
         const float *gt = gates_buf(x, gi);
         wait_bar(&B.g_full[gi], (i / kNG) & 1, x.abort_flag, p.err, 14);
         const int k = B.gitem[gi];
+        // the previous item's copies complete before the staging tiles are rewritten
+        if (ft == 0) publish();
         if (named_bar_any(kBarB, kGroupB, *x.abort_flag || k < 0)) break;
         const Item it = decode_item(p, k);
 
-        // ---- P [T1 | T2] (M = 64: lanes 0-15 of quarter qd hold rows 16 qd ..)
-        if (ft == 0) tr(p, 0, 8, i);
-        wait_bar(&B.d2_full, i & 1, x.abort_flag, p.err, 15);
-        if (ft == 0) tr(p, 0, 9, i);
-        tc_fence_after();
-        {
-            float v[32];
-            const int r = 16 * qd + lane;
-#pragma unroll 1
-            for (int part = 0; part < 2; ++part) {   // PT1 above T1, PT2 above T2
-#pragma unroll 1
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    tmem_ld32(x.tmem + tm_lane + kTD2 + 64 * part + 32 * h2, v);
-                    tmem_wait_ld();
-                    if (lane < 16) store_half_row_bf16(tb + 16384 * part, r, h2, v);
-                }
-            }
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        // the previous item's ring copies complete here (measured: the best place;
-        // releasing the A1 tile earlier stalls the finisher's leader instead)
-        if (ft == 0) publish();
-        if (named_bar_any(kBarB, kGroupB, *x.abort_flag)) break;
-        if (ft == 0) {
-            mbar_arrive(&B.e2_done);
-            mbar_arrive(&B.d2_empty);
-        }
-        if (ft == 0) tr(p, 0, 10, i);
-
-        // ---- A2 = [gamma Q - P T1 K; -T1 K]
-        // (the waits below also order this group's reads of the Q tile (fp8: its
-        // codes) and of the solver's T2 rows after the writes that published them)
-        wait_bar(&B.st_full[i % kNS], (i / kNS) & 1, x.abort_flag, p.err, 16);
-        wait_bar(&B.tp_full[b], (i >> 1) & 1, x.abort_flag, p.err, 17);
-        wait_bar(&B.d3_full, i & 1, x.abort_flag, p.err, 18);
+        // ---- -W^T: row n = key n, columns = the chunk's tokens
         if (ft == 0) tr(p, 0, 11, i);
+        wait_bar(&B.d3_full, i & 1, x.abort_flag, p.err, 18);
         tc_fence_after();
         {
-            const int n = 32 * qd + lane;   // row of [P T1; T1] K
-            const float gq = (n < 64) ? gt[gGam * 64 + n] : 0.f;
-            const float sq = FP8 ? __ldg(p.q_scale + it.bh) : 1.f;
+            const int n = 32 * qd + lane;
             float v[32];
 #pragma unroll 1
-            for (int kb = 0; kb < 2; ++kb) {
-                const uint8_t *qrow = x.smem + kWStage + (i % kNS) * kWStageBytes + kb * 16384;   // Q, key block kb
-                uint8_t *a2 = x.smem + kPA2 + kb * 16384;
-#pragma unroll 1
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    tmem_ld32(x.tmem + tm_lane + kTD3 + 64 * kb + 32 * h2, v);
-                    tmem_wait_ld();
-                    if (FP8 && n < 64) {   // gamma Q from the q codes: chunks 4 kb + 2 h2, + 1 of row n
-                        const uint8_t *qc = x.smem + kWStage + (i % kNS) * kWStageBytes + n * 128;
+            for (int h2 = 0; h2 < 2; ++h2) {
+                tmem_ld32(x.tmem + tm_lane + kTD3 + 32 * h2, v);
+                tmem_wait_ld();
 #pragma unroll
-                        for (int hc = 0; hc < 2; ++hc) {
-                            const int j = 4 * kb + 2 * h2 + hc;
-                            float f[16];
-                            e4m3x16_to_f32(*reinterpret_cast<const uint4 *>(qc + ((j ^ (n & 7)) << 4)), sq, f);
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) v[16 * hc + e] = fmaf(gq, f[e], -v[16 * hc + e]);
-                        }
-                    } else if (n < 64) {
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const uint4 w = *reinterpret_cast<const uint4 *>(qrow + sw128_off(n, 32 * h2 + 8 * q4));
-                            const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const float2 f = __bfloat1622float2(w2[u]);
-                                v[8 * q4 + 2 * u] = fmaf(gq, f.x, -v[8 * q4 + 2 * u]);
-                                v[8 * q4 + 2 * u + 1] = fmaf(gq, f.y, -v[8 * q4 + 2 * u + 1]);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = -v[e];
-                    }
-                    store_half_row_bf16(a2, n, h2, v);
-                }
+                for (int e = 0; e < 32; ++e) v[e] = -v[e];
+                store_half_row_bf16(x.smem + kPW, n, h2, v);
             }
         }
+        // gate block: e, gamma_end, gamma
         if (ft < 16) {
             *reinterpret_cast<float4 *>(x.smem + kPGst + 16 * ft) =
                 *reinterpret_cast<const float4 *>(gt + gEb * 64 + 4 * ft);
         } else if (ft == 16) {
             *reinterpret_cast<float4 *>(x.smem + kPGst + 256) =
                 make_float4(exp2f(B.gscal[gi][0]), 0.f, 0.f, 0.f);
+        } else if (ft < 33) {
+            *reinterpret_cast<float4 *>(x.smem + kPGst + 4 * kGamOff + 16 * (ft - 17)) =
+                *reinterpret_cast<const float4 *>(gt + gGam * 64 + 4 * (ft - 17));
         }
         tc_fence_before();
         fence_proxy_async_smem();
@@ -792,14 +729,16 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
         }
         if (ft == 0) tr(p, 0, 12, i);
 
-        // ---- the item's slot: A1, A2, e, gamma_end (bulk copies, published an item later)
+        // ---- the item's slot (bulk copies, published at the start of the next item)
         if (ft == 0) {
             // the slot's previous chunk must have been taken out by the chain
             if (it.ci < kNSlot || wait_global(p.consumed + (size_t)it.scan * kFlagStride, it.ci - kNSlot + 1, x, p, 64)) {
                 uint8_t *slot = p.ring + ((size_t)it.scan * kNSlot + it.ci % kNSlot) * kSlotBytes;
-                bulk_store(slot + kSlotA1, tb + 16384, 16384);
-                bulk_store(slot + kSlotA2, x.smem + kPA2, 32768);
-                bulk_store(slot + kSlotGates, x.smem + kPGst, 512);
+                const uint8_t *tb = x.smem + kPTB + b * kTBBytes;
+                bulk_store(slot + kSlotP, tb, 8192);
+                bulk_store(slot + kSlotT2, tb + 16384, 8192);
+                bulk_store(slot + kSlotW, x.smem + kPW, 16384);
+                bulk_store(slot + kSlotGates, x.smem + kPGst, kGateBlockBytes);
                 bulk_commit();
                 pend_scan = it.scan;
                 pend_c = it.ci;
@@ -817,8 +756,8 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
 // ================================================================== chains
 
 template <int DIR, bool FP8>
-__device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, const CUtensorMap *tmV,
-                                          const PoolParams &p)
+__device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                                          const CUtensorMap *tmV, const PoolParams &p)
 {
     Bars &B = *x.bars;
     int vk_issued = 0, a_issued = 0;
@@ -826,19 +765,22 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
     for (int i = 0; i < x.NC; ++i) {
         const int st = i % kNVK, ab = i & 1, s = i % kNSlot;
         const int c = chunk_of<DIR>(x, i);
-        if (FP8) {   // the E4M3 v, k tiles into the staging (widened into the V/K stage by the converters)
+        if (FP8) {   // the E4M3 v, k, q tiles into the staging (widened into the stage by the converters)
             if (i >= 1 && !wait_bar(&B.s8_empty, (i - 1) & 1, x.abort_flag, p.err, 37)) break;
-            mbar_arrive_expect_tx(&B.s8_full, 16384);
+            mbar_arrive_expect_tx(&B.s8_full, 24576);
             tma_load_3d(x.smem + kC8, tmV, &B.s8_full, 0, c * kC, x.bh);
             tma_load_3d(x.smem + kC8 + 8192, tmK, &B.s8_full, 0, c * kC, x.bh);
+            tma_load_3d(x.smem + kC8 + 16384, tmQ, &B.s8_full, 0, c * kC, x.bh);
         } else {
             if (i >= kNVK && !wait_bar(&B.vk_empty[st], ((i / kNVK) + 1) & 1, x.abort_flag, p.err, 21)) break;
-            uint8_t *sv = x.smem + kCStage + st * 32768;
-            mbar_arrive_expect_tx(&B.vk_full[st], 32768);
+            uint8_t *sv = x.smem + kCStage + st * kCStageBytes;
+            mbar_arrive_expect_tx(&B.vk_full[st], 49152);
             tma_load_3d(sv, tmV, &B.vk_full[st], 0, c * kC, x.bh);
             tma_load_3d(sv + 8192, tmV, &B.vk_full[st], 64, c * kC, x.bh);
             tma_load_3d(sv + 16384, tmK, &B.vk_full[st], 0, c * kC, x.bh);
             tma_load_3d(sv + 24576, tmK, &B.vk_full[st], 64, c * kC, x.bh);
+            tma_load_3d(sv + 32768, tmQ, &B.vk_full[st], 0, c * kC, x.bh);
+            tma_load_3d(sv + 40960, tmQ, &B.vk_full[st], 64, c * kC, x.bh);
         }
         vk_issued = i + 1;
         if (i >= 2 && !wait_bar(&B.a_empty[ab], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 22)) break;
@@ -849,11 +791,10 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
         fence_proxy_async_global();
         const uint8_t *slot = x.ring + (size_t)s * kSlotBytes;
         uint8_t *dst = x.smem + kCA + ab * kCABytes;
-        mbar_arrive_expect_tx(&B.a_full[ab], kSlotBytes);
+        mbar_arrive_expect_tx(&B.a_full[ab], kSlotCopy);
         bulk_load(dst, slot, 16384, &B.a_full[ab]);
         bulk_load(dst + 16384, slot + 16384, 16384, &B.a_full[ab]);
-        bulk_load(dst + 32768, slot + 32768, 16384, &B.a_full[ab]);
-        bulk_load(dst + 49152, slot + 49152, 512, &B.a_full[ab]);
+        bulk_load(dst + kSlotGates, slot + kSlotGates, kGateBlockBytes, &B.a_full[ab]);
         a_issued = i + 1;
     }
     if (*x.abort_flag) {
@@ -867,35 +808,54 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmK, 
     }
 }
 
-// Converters (2 warps, fp8 inputs): per chunk, the staged E4M3 v, k tiles
-// widened to scaled bf16 into the V/K stage the chain's products read.
+// Converters (2 warps): per chunk, Q' = diag(gamma) Q in the stage (the B
+// operand of H^T Q'^T; gamma comes with the ring slot); with fp8 inputs, the
+// staged E4M3 v, k tiles widened to scaled bf16 into the stage first, and q
+// widened with its scale times gamma.
+template <bool FP8>
 __device__ __forceinline__ void chain_convert(const Ctx &x, const PoolParams &p, int t)
 {
     Bars &B = *x.bars;
-    const float sv = __ldg(p.v_scale + x.bh), sk = __ldg(p.k_scale + x.bh);
+    const float sv = FP8 ? __ldg(p.v_scale + x.bh) : 1.f, sk = FP8 ? __ldg(p.k_scale + x.bh) : 1.f;
+    const float sq = FP8 ? __ldg(p.q_scale + x.bh) : 1.f;
 #pragma unroll 1
     for (int i = 0; i < x.NC; ++i) {
-        const int st = i % kNVK;
+        const int st = i % kNVK, ab = i & 1;
+        uint8_t *stage = x.smem + kCStage + st * kCStageBytes;   // [V0 | V1 | K0 | K1 | Q0 | Q1]
         bool ok = true;
-        if (t == 0) {
-            ok = wait_bar(&B.s8_full, i & 1, x.abort_flag, p.err, 38);
-            if (ok && i >= kNVK) ok = wait_bar(&B.vk_empty[st], ((i / kNVK) + 1) & 1, x.abort_flag, p.err, 39);
-        }
-        if (named_bar_any(kBarConv, 64, !ok || *x.abort_flag)) break;
-        uint8_t *stage = x.smem + kCStage + st * 32768;   // [V0 | V1 | K0 | K1]
+        if (FP8) {
+            if (t == 0) {
+                ok = wait_bar(&B.s8_full, i & 1, x.abort_flag, p.err, 38);
+                if (ok && i >= kNVK) ok = wait_bar(&B.vk_empty[st], ((i / kNVK) + 1) & 1, x.abort_flag, p.err, 39);
+            }
+            if (named_bar_any(kBarConv, 64, !ok || *x.abort_flag)) break;
 #pragma unroll 1
-        for (int rd = 0; rd < 2; ++rd)
-            e4m3_tile_to_bf16(x.smem + kC8 + 8192 * rd, stage + 16384 * rd, stage + 16384 * rd + 8192, rd ? sk : sv,
-                              t, kBarConv);
+            for (int rd = 0; rd < 2; ++rd)
+                e4m3_tile_to_bf16(x.smem + kC8 + 8192 * rd, stage + 16384 * rd, stage + 16384 * rd + 8192,
+                                  rd ? sk : sv, t, kBarConv);
+            fence_proxy_async_smem();
+            named_bar(kBarConv, 64);
+            if (t == 0) mbar_arrive(&B.vk_full[st]);
+        } else if (t == 0) {
+            ok = wait_bar(&B.vk_full[st], (i / kNVK) & 1, x.abort_flag, p.err, 39);
+        }
+        if (t == 0 && ok) ok = wait_bar(&B.a_full[ab], (i >> 1) & 1, x.abort_flag, p.err, 40);
+        if (named_bar_any(kBarConv, 64, !ok || *x.abort_flag)) break;
+        const float *gam = reinterpret_cast<const float *>(x.smem + kCA + ab * kCABytes + kSlotGates) + kGamOff;
+        if (FP8) e4m3_tile_to_bf16(x.smem + kC8 + 16384, stage + 32768, stage + 40960, sq, t, kBarConv, gam);
+        else scale_row_bf16(stage + 32768, t, gam[t]);
         fence_proxy_async_smem();
         named_bar(kBarConv, 64);
         if (t == 0) {
-            mbar_arrive(&B.s8_empty);   // the staging may take the next chunk's codes
-            mbar_arrive(&B.vk_full[st]);
+            if (FP8) mbar_arrive(&B.s8_empty);   // the staging may take the next chunk's codes
+            mbar_arrive(&B.q_full[st]);
         }
     }
 }
 
+// MMA issue, per chunk: U^T (its state-free part first, then the product with
+// H^T), H^T Q'^T (while H^T is still the previous state), S = Ubar^T K once the
+// state group has formed Ubar^T, then U^T P^T (off the state's path).
 __device__ __forceinline__ void chain_mma(const Ctx &x, const PoolParams &p)
 {
     Bars &B = *x.bars;
@@ -908,24 +868,32 @@ __device__ __forceinline__ void chain_mma(const Ctx &x, const PoolParams &p)
         tr(p, 1, 2, i);
         if (i >= 2 && !wait_bar(&B.d_empty[db], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 26)) break;
         tr(p, 1, 3, i);
-        const uint32_t sv = x.sbase + kCStage + st * 32768;
+        const uint32_t sv = x.sbase + kCStage + st * kCStageBytes;
         const uint32_t sa = x.sbase + kCA + ab * kCABytes;
-        const uint32_t dD = tm + kTD + 128 * db;
+        const uint32_t dO = tm + kTD + 128 * db, dU = dO + 64;
         tc_fence_after();
-        // D = V^T A1^T: A = V (MN-major, dv groups 8 KB apart), B = A1 (K-major)
-        mma_run<4, 128, 2>(dD, sw128_desc(sv, 8192, 1024), sw128_desc(sa + kSlotA1, 16, 1024), kIdA, false);
+        // U^T = V^T T2^T: A = V (MN-major, dv groups 8 KB apart), B = T2 (K-major)
+        mma_run<4, 128, 2>(dU, sw128_desc(sv, 8192, 1024), sw128_desc(sa + kSlotT2, 16, 1024), kIdU1, false);
         if (!wait_bar(&B.h_full, i & 1, x.abort_flag, p.err, 27)) break;
         tr(p, 1, 4, i);
         tc_fence_after();
-        // D += H^T A2^T: A = H^T (bf16 in TMEM), B = A2 (K-major, key blocks 16 KB apart)
+        // U^T += H^T (-W^T): A = H^T (bf16 in TMEM), B = -W^T [key][token] (MN-major)
         {
-            const uint64_t dA2 = sw128_desc(sa + kSlotA2, 16, 1024);
+            const uint64_t dW = sw128_desc(sa + kSlotW, 8192, 1024);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mma_bf16_ta(dU, tm + kTH + 8 * k, dW + (uint64_t)(k * 128), kIdU2, 1u);
+        }
+        mma_commit(&B.du_full[db]);
+        // O^T = H^T Q'^T: B = Q' [token][dk] (K-major, key blocks 8 KB apart)
+        if (!wait_bar(&B.q_full[st], (i / kNVK) & 1, x.abort_flag, p.err, 42)) break;
+        tc_fence_after();
+        {
+            const uint64_t dQ = sw128_desc(sv + 32768, 16, 1024);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                mma_bf16_ta(dD, tm + kTH + 8 * k, dA2 + (uint64_t)((k >> 2) * 1024 + (k & 3) * 2), kIdB, 1u);
+                mma_bf16_ta(dO, tm + kTH + 8 * k, dQ + (uint64_t)((k >> 2) * 512 + (k & 3) * 2), kIdO,
+                            k > 0 ? 1u : 0u);
         }
-        mma_commit(&B.d_full[db]);
-        mma_commit(&B.a_empty[ab]);
         if (!wait_bar(&B.u_full, i & 1, x.abort_flag, p.err, 28)) break;
         tr(p, 1, 5, i);
         tc_fence_after();
@@ -938,14 +906,22 @@ __device__ __forceinline__ void chain_mma(const Ctx &x, const PoolParams &p)
         }
         mma_commit(&B.s_full);
         mma_commit(&B.vk_empty[st]);
+        // O^T += U^T P^T: A = U^T (bf16 in TMEM), B = P (K-major)
+        {
+            const uint64_t dP = sw128_desc(sa + kSlotP, 16, 1024);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mma_bf16_ta(dO, tm + kTUr + 8 * k, dP + (uint64_t)(2 * k), kIdO, 1u);
+        }
+        mma_commit(&B.do_full[db]);
+        mma_commit(&B.a_empty[ab]);
     }
     drain_mmas(B);
 }
 
 // State group (8 warps): H^T in fp32 registers, thread (quarter q, half h) holds
 // row d = 32 q + lane, key columns [64 h, +64).  U epilogue: tokens [32 h, +32)
-// of U^T, scaled by e, into Ubar^T (bf16, TMEM); state epilogue: H^T <-
-// gamma_end H^T + S into registers and its bf16 copy into TMEM.
+// of U^T into U^T and, scaled by e, Ubar^T (both bf16, TMEM); state epilogue:
+// H^T <- gamma_end H^T + S into registers and its bf16 copy into TMEM.
 template <int DIR>
 __device__ __forceinline__ void chain_state(const Ctx &x, const PoolParams &p, int ct, int q, int h)
 {
@@ -978,14 +954,14 @@ __device__ __forceinline__ void chain_state(const Ctx &x, const PoolParams &p, i
         const float *eg = reinterpret_cast<const float *>(x.smem + kCA + ab * kCABytes + kSlotGates);
         // ---- Ubar^T (e and gamma_end come with the chunk's ring slot)
         wait_bar(&B.a_full[ab], (i >> 1) & 1, x.abort_flag, p.err, 34);
-        wait_bar(&B.d_full[db], (i >> 1) & 1, x.abort_flag, p.err, 31);
+        wait_bar(&B.du_full[db], (i >> 1) & 1, x.abort_flag, p.err, 31);
         if (ct == 0) tr(p, 1, 8, i);
         tc_fence_after();
         {
-            uint32_t w[16];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 float u[16];
+                uint32_t we[8], wr[8];
                 tmem_ld16(x.tmem + tl + kTD + 128 * db + 64 + 32 * h + 16 * h2, u);
                 tmem_wait_ld();
                 if (dbg && i == 0)
@@ -994,11 +970,14 @@ __device__ __forceinline__ void chain_state(const Ctx &x, const PoolParams &p, i
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     const float4 ev = e4[m];
-                    w[8 * h2 + 2 * m] = pack_bf16(u[4 * m] * ev.x, u[4 * m + 1] * ev.y);
-                    w[8 * h2 + 2 * m + 1] = pack_bf16(u[4 * m + 2] * ev.z, u[4 * m + 3] * ev.w);
+                    we[2 * m] = pack_bf16(u[4 * m] * ev.x, u[4 * m + 1] * ev.y);
+                    we[2 * m + 1] = pack_bf16(u[4 * m + 2] * ev.z, u[4 * m + 3] * ev.w);
+                    wr[2 * m] = pack_bf16(u[4 * m], u[4 * m + 1]);
+                    wr[2 * m + 1] = pack_bf16(u[4 * m + 2], u[4 * m + 3]);
                 }
+                tmem_st8(x.tmem + tl + kTUb + 16 * h + 8 * h2, we);
+                tmem_st8(x.tmem + tl + kTUr + 16 * h + 8 * h2, wr);
             }
-            tmem_st16(x.tmem + tl + kTUb + 16 * h, w);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -1068,6 +1047,7 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
     int nload0 = 0, nload1 = 0;       // partial loads waited for, per staging tile
     int nissued0 = 0, nissued1 = 0;   // leader: partial loads issued, per staging tile
     int loaded_ahead = -1;            // leader: the chunk whose partial load is already in flight
+    int pub_c = -1;                   // leader: a first writer's chunk stored but not yet published
     const bool bidi = p.counters != nullptr;
     // every CTA is resident: the forward scan reaches the first half of the
     // chunks first, the reverse scan the second half
@@ -1092,7 +1072,7 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
                 load_partial(c, ob);
             }
         }
-        wait_bar(&B.d_full[db], (i >> 1) & 1, x.abort_flag, p.err, 33);
+        wait_bar(&B.do_full[db], (i >> 1) & 1, x.abort_flag, p.err, 33);
         // the staging tile's store of two chunks ago must have read it before it is rewritten
         if (lead) bulk_wait_read1();
         if (named_bar_any(kBarB, kGroupB, *x.abort_flag)) break;
@@ -1109,13 +1089,18 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
             tmem_wait_ld();
             if (dbg && i == 0)
                 for (int j = 0; j < 32; ++j) p.debug[d * 128 + 32 * h2 + j] = v[j];
+            if (!first) {   // the first writer's partial: every load before the first store
+                __nv_bfloat16 pv[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                __nv_bfloat16 *e = reinterpret_cast<__nv_bfloat16 *>(stg + dblk + sw128_off(32 * h2 + j, d & 63));
-                float y = v[j];
-                if (!first) y += __bfloat162float(*e);
-                *e = __float2bfloat16_rn(y);
+                for (int j = 0; j < 32; ++j)
+                    pv[j] = *reinterpret_cast<const __nv_bfloat16 *>(stg + dblk + sw128_off(32 * h2 + j, d & 63));
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] += __bfloat162float(pv[j]);
             }
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                *reinterpret_cast<__nv_bfloat16 *>(stg + dblk + sw128_off(32 * h2 + j, d & 63)) =
+                    __float2bfloat16_rn(v[j]);
         }
         tc_fence_before();
         fence_proxy_async_smem();
@@ -1125,12 +1110,26 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
             tma_store_3d(tmO, stg, 0, c * kC, x.bh);
             tma_store_3d(tmO, stg + 8192, 64, c * kC, x.bh);
             bulk_commit();
-            if (bidi && first) {
-                // publish the partial once its writes are performed
-                bulk_wait0();
+            // a first writer's partial is published once its writes are performed:
+            // the previous one now (its store has had a chunk's time), this one
+            // at the next chunk if that is a first-writer chunk too (it does not
+            // wait for the other scan), else now
+            if (pub_c >= 0) {
+                bulk_wait1();
                 fence_proxy_async_global();
                 __threadfence();
-                atomicAdd(counter(c), 1);
+                atomicAdd(counter(pub_c), 1);
+                pub_c = -1;
+            }
+            if (bidi && first) {
+                if (i + 1 < x.NC && first_of(chunk_of<DIR>(x, i + 1))) {
+                    pub_c = c;
+                } else {
+                    bulk_wait0();
+                    fence_proxy_async_global();
+                    __threadfence();
+                    atomicAdd(counter(c), 1);
+                }
             }
             // request the next tile's partial now if its first writer is done
             if (bidi && i + 1 < x.NC) {
@@ -1149,6 +1148,11 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
     }
     if (lead) {
         bulk_wait0();   // every store performed before the CTA exits
+        if (pub_c >= 0 && !*x.abort_flag) {
+            fence_proxy_async_global();
+            __threadfence();
+            atomicAdd(counter(pub_c), 1);
+        }
         for (int k = nload0; k < nissued0; ++k) drain_copies(&B.o_full[0], k & 1);   // after an abort
         for (int k = nload1; k < nissued1; ++k) drain_copies(&B.o_full[1], k & 1);
     }
@@ -1188,13 +1192,14 @@ gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         const int nbar = (int)(offsetof(Bars, gscal) / sizeof(uint64_t));
         for (int k = 0; k < nbar; ++k) mbar_init(&all[k], 1);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&B.t_free[b], 2);    // [P T1; T1] K done, ring copy read A1
-            mbar_init(&B.a_empty[b], 2);   // D += H^T A2^T done, state epilogue done
+            mbar_init(&B.t_free[b], 2);    // W^T product done, ring copies read P and T2
+            mbar_init(&B.a_empty[b], 2);   // the chunk's products done, state epilogue done
             mbar_init(&B.d_empty[b], 2);   // output epilogue, U epilogue
         }
         B.abort_flag = 0;
         fence_mbar_init();
         if (chain) {
+            prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmO);
@@ -1212,8 +1217,8 @@ gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         for (int i = tid; i < 64 * kLDA; i += kThreads) As0[i] = 0.f;
         // T1, T2: the triangle the solve never writes stays zero throughout
         for (int b = 0; b < 2; ++b) {
-            uint32_t *t1 = reinterpret_cast<uint32_t *>(smem + kPTB + b * 32768 + 8192);
-            uint32_t *t2 = reinterpret_cast<uint32_t *>(smem + kPTB + b * 32768 + 24576);
+            uint32_t *t1 = reinterpret_cast<uint32_t *>(smem + kPTB + b * kTBBytes + 8192);
+            uint32_t *t2 = reinterpret_cast<uint32_t *>(smem + kPTB + b * kTBBytes + 16384);
             for (int i = tid; i < 8192 / 4; i += kThreads) t1[i] = t2[i] = 0u;
         }
     }
@@ -1237,8 +1242,8 @@ gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     } else {
         if (warp == 0) {
             if (lane == 0) {
-                if (x.dir) chain_tma<1, FP8>(x, &tmK, &tmV, p);
-                else chain_tma<0, FP8>(x, &tmK, &tmV, p);
+                if (x.dir) chain_tma<1, FP8>(x, &tmQ, &tmK, &tmV, p);
+                else chain_tma<0, FP8>(x, &tmQ, &tmK, &tmV, p);
             }
         } else if (warp == 1) {
             if (lane == 0) chain_mma(x, p);
@@ -1250,8 +1255,8 @@ gdn_chunk_pool_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             const int ot = tid - 320, q = warp & 3;
             if (x.dir) chain_out<1>(x, p, &tmO, ot, q);
             else chain_out<0>(x, p, &tmO, ot, q);
-        } else if (FP8) {
-            chain_convert(x, p, tid - 448);
+        } else {
+            chain_convert<FP8>(x, p, tid - 448);
         }
     }
 
@@ -1419,7 +1424,7 @@ cudaError_t launch_chunk_pool(const FwdArgs &a, cudaStream_t stream, const float
 }  // namespace gdn
 
 // Test hooks (declared in gdn_debug.h).
-// gdn_debug_ring: a device buffer of at least dirs*B*H*8*49664 bytes that the
+// gdn_debug_ring: a device buffer of at least dirs*B*H*8*33792 bytes that the
 // pooled kernel uses as its operand ring instead of workspace (NULL: off), so a
 // test can read back the prepared operands of each scan's last eight chunks.
 // gdn_debug_kernel_select: 0 picks the kernel by shape (the pooled kernel for

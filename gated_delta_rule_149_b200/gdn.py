@@ -386,7 +386,7 @@ def debug_kernel_select(which):
 
 
 def debug_ring(buf):
-    """Test hook: a CUDA uint8 tensor of at least dirs*B*H*8*49664 bytes that the
+    """Test hook: a CUDA uint8 tensor of at least dirs*B*H*8*33792 bytes that the
     pooled kernel uses as its operand ring (None: workspace), so that the
     prepared operands of the last eight chunks of every scan can be read back."""
     load_library().gdn_debug_ring(None if buf is None else ctypes.c_void_p(buf.data_ptr()))

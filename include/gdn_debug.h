@@ -22,7 +22,7 @@ extern "C" {
 void gdn_debug_kernel_select(int which);
 
 /*
- * gdn_debug_ring -- a device buffer of at least dirs*B*H*8*49664 bytes (dirs
+ * gdn_debug_ring -- a device buffer of at least dirs*B*H*8*33792 bytes (dirs
  * = 2 for GDN_BIDI, else 1) that the pooled kernel uses as its operand ring
  * instead of workspace, so that a test can read back the operands prepared
  * for each scan's last eight chunks.  NULL (default) turns it off.  Caller-owned.
