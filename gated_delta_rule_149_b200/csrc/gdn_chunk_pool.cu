@@ -261,6 +261,10 @@ __device__ __forceinline__ void st_release_gpu(int *addr, int v)
 {
     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
 }
+__device__ __forceinline__ void st_relaxed_gpu(int *addr, int v)
+{
+    asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
 
 // Bounded wait until a device-wide word reaches `target`; on timeout the error
 // is recorded and the CTA's abort flag raised.  false on timeout or abort.
@@ -677,7 +681,6 @@ __device__ __forceinline__ void worker_finisher(const Ctx &x, const PoolParams &
         mbar_arrive(&B.t_free[pend_b]);
         bulk_wait0();
         fence_proxy_async_global();
-        __threadfence();
         st_release_gpu(p.slot_seq + (size_t)pend_scan * kFlagStride + pend_c % kNSlot, pend_c + 1);
         pend_scan = -1;
     };
@@ -864,7 +867,10 @@ __device__ __forceinline__ void chain_mma(const Ctx &x, const PoolParams &p)
         const int st = i % kNVK, ab = i & 1, db = i & 1;
         if (!wait_bar(&B.vk_full[st], (i / kNVK) & 1, x.abort_flag, p.err, 24)) break;
         if (!wait_bar(&B.a_full[ab], (i >> 1) & 1, x.abort_flag, p.err, 25)) break;
-        st_release_gpu(p.consumed + (size_t)x.scan * kFlagStride, i + 1);   // the slot's data has landed: it may be refilled
+        // the slot's data has landed (the bulk copy that read it completed): it
+        // may be refilled.  A relaxed store: no write of this thread needs
+        // ordering before it, and a release here cost ~1k cycles a chunk.
+        st_relaxed_gpu(p.consumed + (size_t)x.scan * kFlagStride, i + 1);
         tr(p, 1, 2, i);
         if (i >= 2 && !wait_bar(&B.d_empty[db], ((i >> 1) + 1) & 1, x.abort_flag, p.err, 26)) break;
         tr(p, 1, 3, i);
