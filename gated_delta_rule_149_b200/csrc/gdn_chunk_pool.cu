@@ -1035,11 +1035,15 @@ __device__ __forceinline__ void chain_state(const Ctx &x, const PoolParams &p, i
 }
 
 // Output group (4 warps): thread (quarter q) owns column d = 32 q + lane of each
-// chunk's O tile.  The tile is assembled in shared memory as [dv block][token]
-// rows (the TMA layout of o) and written with one TMA store.  Bidirectional:
-// the first writer of a tile stores its bf16 partial and then publishes it on
-// the tile's counter; the second loads that partial by TMA (requested a chunk
-// ahead), adds its fp32 partial and rounds once.
+// chunk's O tile.  A tile with no partial to add (causal calls, and a
+// bidirectional tile's first writer) is written straight to o, one 2-byte
+// store per token (a warp instruction covers 64 contiguous bytes of a row:
+// two whole sectors); a first writer then publishes its bf16 partial on the
+// tile's counter, after the group's barrier, with one thread's release
+// (cumulative: it covers the stores the barrier ordered before it).  The
+// second writer loads that partial by TMA (requested a chunk ahead) into a
+// 128B-swizzled staging tile ([dv block][token] rows, the TMA layout of o),
+// adds its fp32 partial, rounds once and stores the tile with TMA.
 template <int DIR>
 __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, const CUtensorMap *tmO, int ot, int q)
 {
@@ -1050,15 +1054,19 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
     const bool dbg = kDbgOn && p.debug != nullptr && x.scan == 0;
     // this thread's column in a staging tile: dv block d / 64, column d % 64
     const uint32_t dblk = (uint32_t)(d >> 6) * 8192u;
+    __nv_bfloat16 *col = p.o + (size_t)x.bh * x.T * 128 + d;   // o[bh][t][d] at col + 128 t
     int nload0 = 0, nload1 = 0;       // partial loads waited for, per staging tile
     int nissued0 = 0, nissued1 = 0;   // leader: partial loads issued, per staging tile
     int loaded_ahead = -1;            // leader: the chunk whose partial load is already in flight
-    int pub_c = -1;                   // leader: a first writer's chunk stored but not yet published
+    int pending = -1;                 // a first writer's tile published at the next chunk's first barrier
     const bool bidi = p.counters != nullptr;
     // every CTA is resident: the forward scan reaches the first half of the
     // chunks first, the reverse scan the second half
     auto first_of = [&](int c) { return DIR == ((2 * c < x.NC) ? 0 : 1); };
     auto counter = [&](int c) { return p.counters + (size_t)x.bhl * x.NC + c; };
+    auto release_add = [&](int c) {
+        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter(c)) : "memory");
+    };
     auto load_partial = [&](int c, int ob) {
         uint8_t *stg = x.smem + kCO + ob * 16384;
         fence_proxy_async_global();
@@ -1080,14 +1088,20 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
         }
         wait_bar(&B.do_full[db], (i >> 1) & 1, x.abort_flag, p.err, 33);
         // the staging tile's store of two chunks ago must have read it before it is rewritten
-        if (lead) bulk_wait_read1();
+        if (lead && !first) bulk_wait_read1();
         if (named_bar_any(kBarB, kGroupB, *x.abort_flag)) break;
+        if (pending >= 0) {   // the previous chunk's stores: every thread's were issued before the barrier
+            if (lead) release_add(pending);
+            pending = -1;
+        }
         if (!first) {
             int &nl = ob ? nload1 : nload0;
             wait_bar(&B.o_full[ob], nl & 1, x.abort_flag, p.err, 35);
             ++nl;
         }
         tc_fence_after();
+        __nv_bfloat16 *orow = col + (size_t)c * kC * 128;
+        const int n = (x.T - c * kC) < kC ? (x.T - c * kC) : kC;   // the chunk's tokens (ragged tail)
 #pragma unroll 1
         for (int h2 = 0; h2 < 2; ++h2) {
             float v[32];
@@ -1095,72 +1109,57 @@ __device__ __forceinline__ void chain_out(const Ctx &x, const PoolParams &p, con
             tmem_wait_ld();
             if (dbg && i == 0)
                 for (int j = 0; j < 32; ++j) p.debug[d * 128 + 32 * h2 + j] = v[j];
-            if (!first) {   // the first writer's partial: every load before the first store
+            if (first) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (32 * h2 + j < n) orow[(size_t)(32 * h2 + j) * 128] = __float2bfloat16_rn(v[j]);
+            } else {   // the first writer's partial: every load before the first store
                 __nv_bfloat16 pv[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
                     pv[j] = *reinterpret_cast<const __nv_bfloat16 *>(stg + dblk + sw128_off(32 * h2 + j, d & 63));
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] += __bfloat162float(pv[j]);
+                for (int j = 0; j < 32; ++j)
+                    *reinterpret_cast<__nv_bfloat16 *>(stg + dblk + sw128_off(32 * h2 + j, d & 63)) =
+                        __float2bfloat16_rn(v[j] + __bfloat162float(pv[j]));
             }
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                *reinterpret_cast<__nv_bfloat16 *>(stg + dblk + sw128_off(32 * h2 + j, d & 63)) =
-                    __float2bfloat16_rn(v[j]);
         }
         tc_fence_before();
-        fence_proxy_async_smem();
+        if (!first) fence_proxy_async_smem();
         if (named_bar_any(kBarB, kGroupB, *x.abort_flag)) break;
         if (lead) {
             mbar_arrive(&B.d_empty[db]);
-            tma_store_3d(tmO, stg, 0, c * kC, x.bh);
-            tma_store_3d(tmO, stg + 8192, 64, c * kC, x.bh);
-            bulk_commit();
-            // a first writer's partial is published once its writes are performed:
-            // the previous one now (its store has had a chunk's time), this one
-            // at the next chunk if that is a first-writer chunk too (it does not
-            // wait for the other scan), else now
-            if (pub_c >= 0) {
-                bulk_wait1();
-                fence_proxy_async_global();
-                __threadfence();
-                atomicAdd(counter(pub_c), 1);
-                pub_c = -1;
+            if (!first) {
+                tma_store_3d(tmO, stg, 0, c * kC, x.bh);
+                tma_store_3d(tmO, stg + 8192, 64, c * kC, x.bh);
+                bulk_commit();
             }
-            if (bidi && first) {
-                if (i + 1 < x.NC && first_of(chunk_of<DIR>(x, i + 1))) {
-                    pub_c = c;
-                } else {
-                    bulk_wait0();
-                    fence_proxy_async_global();
-                    __threadfence();
-                    atomicAdd(counter(c), 1);
-                }
-            }
-            // request the next tile's partial now if its first writer is done
-            if (bidi && i + 1 < x.NC) {
-                const int cn = chunk_of<DIR>(x, i + 1);
-                if (!first_of(cn)) {
-                    int seen;
-                    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(counter(cn)) : "memory");
-                    if (seen >= 1) {
-                        bulk_wait_read1();   // tile (i + 1) & 1: its store of chunk i - 1 has read it
-                        load_partial(cn, (i + 1) & 1);
-                        loaded_ahead = i + 1;
-                    }
+        }
+        if (bidi && first) {
+            // published at the next chunk when that is a first-writer chunk too
+            // (it does not wait for the other scan), else now
+            if (i + 1 < x.NC && first_of(chunk_of<DIR>(x, i + 1))) pending = c;
+            else if (lead) release_add(c);
+        }
+        // request the next tile's partial now if its first writer is done
+        if (lead && bidi && i + 1 < x.NC) {
+            const int cn = chunk_of<DIR>(x, i + 1);
+            if (!first_of(cn)) {
+                int seen;
+                asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(counter(cn)) : "memory");
+                if (seen >= 1) {
+                    bulk_wait_read1();   // tile (i + 1) & 1: its store of chunk i - 1 has read it
+                    load_partial(cn, (i + 1) & 1);
+                    loaded_ahead = i + 1;
                 }
             }
         }
     }
     if (lead) {
         bulk_wait0();   // every store performed before the CTA exits
-        if (pub_c >= 0 && !*x.abort_flag) {
-            fence_proxy_async_global();
-            __threadfence();
-            atomicAdd(counter(pub_c), 1);
-        }
         for (int k = nload0; k < nissued0; ++k) drain_copies(&B.o_full[0], k & 1);   // after an abort
         for (int k = nload1; k < nissued1; ++k) drain_copies(&B.o_full[1], k & 1);
+        if (pending >= 0 && !*x.abort_flag) release_add(pending);
     }
 }
 
