@@ -180,7 +180,8 @@ struct Bars {
     uint64_t vk_full[kNVK], vk_empty[kNVK], q_full[kNVK], a_full[2], a_empty[2];
     uint64_t du_full[2], do_full[2], d_empty[2], o_full[2];
     uint64_t u_full, s_full, h_full;
-    uint64_t s8_full, s8_empty;        // fp8: the v, k, q code staging
+    uint64_t s8_full, s8_empty;        // fp8: the v, k code staging
+    uint64_t q8_full, q8_empty;        // fp8: the q code staging
     uint64_t drain;
     float gscal[kNG][2];   // per gate buffer: G_end, factorised (1) or not (0)
     int gitem[kNG];        // per gate buffer: the item, or -1 after the last
@@ -763,17 +764,22 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmQ, 
                                           const CUtensorMap *tmV, const PoolParams &p)
 {
     Bars &B = *x.bars;
-    int vk_issued = 0, a_issued = 0;
+    int vk_issued = 0, q_issued = 0, a_issued = 0;
     const int *seq = p.slot_seq + (size_t)x.scan * kFlagStride;
     for (int i = 0; i < x.NC; ++i) {
         const int st = i % kNVK, ab = i & 1, s = i % kNSlot;
         const int c = chunk_of<DIR>(x, i);
-        if (FP8) {   // the E4M3 v, k, q tiles into the staging (widened into the stage by the converters)
+        if (FP8) {   // the E4M3 v, k tiles, and apart from them the q tile, into the staging
+            // (widened into the stage by the converters; q waits for the slot's gamma)
             if (i >= 1 && !wait_bar(&B.s8_empty, (i - 1) & 1, x.abort_flag, p.err, 37)) break;
-            mbar_arrive_expect_tx(&B.s8_full, 24576);
+            mbar_arrive_expect_tx(&B.s8_full, 16384);
             tma_load_3d(x.smem + kC8, tmV, &B.s8_full, 0, c * kC, x.bh);
             tma_load_3d(x.smem + kC8 + 8192, tmK, &B.s8_full, 0, c * kC, x.bh);
-            tma_load_3d(x.smem + kC8 + 16384, tmQ, &B.s8_full, 0, c * kC, x.bh);
+            vk_issued = i + 1;
+            if (i >= 1 && !wait_bar(&B.q8_empty, (i - 1) & 1, x.abort_flag, p.err, 43)) break;
+            mbar_arrive_expect_tx(&B.q8_full, 8192);
+            tma_load_3d(x.smem + kC8 + 16384, tmQ, &B.q8_full, 0, c * kC, x.bh);
+            q_issued = i + 1;
         } else {
             if (i >= kNVK && !wait_bar(&B.vk_empty[st], ((i / kNVK) + 1) & 1, x.abort_flag, p.err, 21)) break;
             uint8_t *sv = x.smem + kCStage + st * kCStageBytes;
@@ -801,8 +807,9 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmQ, 
         a_issued = i + 1;
     }
     if (*x.abort_flag) {
-        if (FP8) {   // one staging load in flight at most
+        if (FP8) {   // one load of each staging in flight at most
             if (vk_issued > 0) drain_copies(&B.s8_full, (vk_issued - 1) & 1);
+            if (q_issued > 0) drain_copies(&B.q8_full, (q_issued - 1) & 1);
         } else {
             for (int i = (vk_issued > kNVK ? vk_issued - kNVK : 0); i < vk_issued; ++i)
                 drain_copies(&B.vk_full[i % kNVK], (i / kNVK) & 1);
@@ -813,8 +820,9 @@ __device__ __forceinline__ void chain_tma(const Ctx &x, const CUtensorMap *tmQ, 
 
 // Converters (2 warps): per chunk, Q' = diag(gamma) Q in the stage (the B
 // operand of H^T Q'^T; gamma comes with the ring slot); with fp8 inputs, the
-// staged E4M3 v, k tiles widened to scaled bf16 into the stage first, and q
-// widened with its scale times gamma.
+// staged E4M3 v, k tiles widened to scaled bf16 into the stage first (their
+// staging then takes the next chunk's codes), and q widened with its scale
+// times gamma.
 template <bool FP8>
 __device__ __forceinline__ void chain_convert(const Ctx &x, const PoolParams &p, int t)
 {
@@ -838,7 +846,11 @@ __device__ __forceinline__ void chain_convert(const Ctx &x, const PoolParams &p,
                                   rd ? sk : sv, t, kBarConv);
             fence_proxy_async_smem();
             named_bar(kBarConv, 64);
-            if (t == 0) mbar_arrive(&B.vk_full[st]);
+            if (t == 0) {
+                mbar_arrive(&B.s8_empty);   // the staging may take the next chunk's v, k codes
+                mbar_arrive(&B.vk_full[st]);
+                ok = wait_bar(&B.q8_full, i & 1, x.abort_flag, p.err, 44);
+            }
         } else if (t == 0) {
             ok = wait_bar(&B.vk_full[st], (i / kNVK) & 1, x.abort_flag, p.err, 39);
         }
@@ -850,7 +862,7 @@ __device__ __forceinline__ void chain_convert(const Ctx &x, const PoolParams &p,
         fence_proxy_async_smem();
         named_bar(kBarConv, 64);
         if (t == 0) {
-            if (FP8) mbar_arrive(&B.s8_empty);   // the staging may take the next chunk's codes
+            if (FP8) mbar_arrive(&B.q8_empty);   // the q staging may take the next chunk's codes
             mbar_arrive(&B.q_full[st]);
         }
     }
